@@ -1,0 +1,60 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle/pe_oracle.c (on the CPU),
+builds it, and runs the pin suite against it in a child process; the suite has
+to fail.  The real oracle is never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "pe_oracle.c")
+
+MUTANTS = {
+    "window_inner_order_swapped": ("(g_h % m) * m + (g_w % m)", "(g_w % m) * m + (g_h % m)"),
+    "window_outer_order_w_major": ("(g_t * (h / m) + g_h / m) * (w / m) + g_w / m",
+                                   "(g_t * (w / m) + g_w / m) * (h / m) + g_h / m"),
+    "bias_dropped": ("out[r * E + e] = acc + (bias ? (double)bias[e] : 0.0);",
+                     "out[r * E + e] = acc;"),
+    "bias_dropped_patches": ("out[n * E + e] = acc + (bias ? (double)bias[e] : 0.0);",
+                             "out[n * E + e] = acc;"),
+    "norm_sign": ("volatile float d = x - mean;", "volatile float d = x + mean;"),
+    "norm_reciprocal_multiply": ("volatile float q = d / std;",
+                                 "volatile float q = d * (1.0f / std);"),
+    "pad_repeats_first_frame": ("const int src = tau < T ? tau : T - 1;",
+                                "const int src = tau < T ? tau : 0;"),
+    "conv_i_j_transposed": ("const int64_t y = g_h * p + i, xx = g_w * p + j;",
+                            "const int64_t y = g_h * p + j, xx = g_w * p + i;"),
+    "patch_x_k_order_t_major": ("oracle_bf16_round(x[n * K + k])",
+                                "oracle_bf16_round(x[n * K + (((int64_t)t * C + c) * p + i) * p + j])"),
+    "weight_not_rounded": ("oracle_bf16_round_array(w, wb, (int64_t)E * K);\n    const int64_t ncell",
+                           "memcpy(wb, w, sizeof(float) * (size_t)(E * K));\n    const int64_t ncell"),
+    "bf16_truncates": ("u = (u + 0x7fffu + ((u >> 16) & 1u)) & 0xffff0000u;",
+                       "u = u & 0xffff0000u;"),
+    "bf16_ties_away": ("u = (u + 0x7fffu + ((u >> 16) & 1u)) & 0xffff0000u;",
+                       "u = (u + 0x8000u) & 0xffff0000u;"),
+    "input_not_rounded": ("const double xv = (double)oracle_bf16_round(x[n * K + k]);",
+                          "const double xv = (double)x[n * K + k];"),
+    "patchify_drops_time_offset": ("const int64_t tau = g_t * tp + t;\n                        rows",
+                                   "const int64_t tau = g_t * tp;\n                        rows"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"pattern for {name} not found in the oracle source"
+    mut = tmp_path / f"{name}.c"
+    mut.write_text(src.replace(old, new))
+    lib = oracle.compile_source(str(mut), str(tmp_path / f"lib{name}.so"))
+    env = dict(os.environ, PE_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
