@@ -1,0 +1,350 @@
+"""Benchmark of the fused frames -> embedding PatchEmbed on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+host plan + one fused kernel launch (patchify, normalise, merge-order rows,
+bf16 tcgen05 contraction, bias/cast epilogue) over every item of the workload.
+The default workload is the grouped batch of 16 images (one launch).
+
+For N > 1 (torchrun, one process per GPU) every rank embeds its own copy of the
+workload (weak scaling, no data-path collective); the value is all patches of
+all ranks divided by the slowest rank's device time.
+
+Rank 0 prints one JSON line.  Timing: W untimed warm-up steps; K timed steps,
+each bracketed by CUDA events on the launching stream, with an L2 flush (a
+write larger than L2) before every step outside the events; barrier +
+synchronize around the timed region; max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "PatchEmbed patches/s and TFLOP/s (% of B200 dense bf16 peak), 1 GPU"
+UNIT = "patches/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((mhz, int(reasons), util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        names = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def oracle_sample_rate(wl, n_rows: int, seed: int):
+    """Time the CPU oracle on n_rows sampled output rows of the workload.
+    Returns (rows/s, seconds, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    rows = rng.choice(wl.N, size=min(n_rows, wl.N), replace=False)
+    mask = np.zeros(wl.N, np.uint8)
+    mask[rows] = 1
+    t0 = time.perf_counter()
+    if wl.patches is not None:
+        oracle.conv3d_patches(wl.patches, wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
+    else:
+        oracle.conv3d_grouped([(it.frames, it.grid) for it in wl.items], wl.merge, wl.mean, wl.std,
+                              wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, dt, oracle.num_threads()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = workloads.ALL[args.workload]()
+    rows_per_step = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample_rate(wl, max(16, rows_per_step // 8), 1000)
+    times, nrows = [], 0
+    threads = 1
+    for s in range(args.steps):
+        r, dt, threads = oracle_sample_rate(wl, rows_per_step, 2000 + s)
+        times.append(dt)
+        nrows += int(round(r * dt))
+    total = sum(times)
+    value = nrows / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_per_step} seeded random output rows of {wl.name} per step "
+                                   f"(of {wl.N}); direct fp64 Conv3d, OpenMP over rows"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def config_of(wl, world):
+    cfg = {"workload": wl.name, "N_patches": wl.N, "K": wl.K, "E": wl.E, "patch": wl.p,
+           "temporal_patch": wl.tp, "merge": wl.merge, "items": max(1, len(wl.items)),
+           "out_dtype": "bf16" if wl.out_dtype == torch.bfloat16 else "f32",
+           "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
+           "l2": "flushed before every timed step (write of 2x L2 outside the events)"}
+    return cfg
+
+
+def run_ours(args, rank, world, local):
+    import vlm_vision_patch_b200 as vp
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    wl = workloads.ALL[args.workload]()
+    pe = vp.PatchEmbed(wl.E, wl.C, wl.tp, wl.p, wl.bias is not None)
+    pe.set_weight(wl.weight.to(dev), None if wl.bias is None else wl.bias.to(dev))
+    pe.set_norm(wl.mean, wl.std)
+    out = torch.empty((wl.N, wl.E), dtype=wl.out_dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    if wl.patches is not None:
+        x_dev = wl.patches.to(dev)
+
+        def step():
+            pe.forward_patches(x_dev, out=out)
+        in_bytes = wl.patches.numel() * wl.patches.element_size()
+    else:
+        frames_dev = [it.frames.to(dev) for it in wl.items]
+        grids = [it.grid for it in wl.items]
+
+        def step():
+            pe.forward_frames_grouped(frames_dev, grids, wl.merge, out=out)
+        in_bytes = sum(it.frames.numel() * it.frames.element_size() for it in wl.items)
+    out_bytes = out.numel() * out.element_size()
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if pe.last_error() != 0:
+        raise RuntimeError("device pipeline timeout during warm-up")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush_buf.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+    times = [a.elapsed_time(b) for a, b in evs]
+    if pe.last_error() != 0:
+        raise RuntimeError("device pipeline timeout during the timed steps")
+    total_ms = sum(times)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    total_max_ms = float(t.item())
+    patches = wl.N * args.steps * world
+    value = patches / (total_max_ms / 1e3)
+
+    # end to end through the public API with host buffers (pinned), per step:
+    # H2D of the step's frames, the forward, D2H of the embeddings
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    if wl.patches is not None:
+        host_in = [wl.patches.pin_memory()]
+        dev_in = [x_dev]
+    else:
+        host_in = [it.frames.pin_memory() for it in wl.items]
+        dev_in = frames_dev
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        for h_, d_ in zip(host_in, dev_in):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for h_, d_ in zip(host_in, dev_in):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(e2e_ms, op=pg.ReduceOp.MAX)
+    e2e_value = wl.N * e2e_steps * world / (float(e2e_ms.item()) / 1e3)
+
+    result = None
+    if rank == 0:
+        peaks, src = load_peaks()
+        flop = 2.0 * wl.N * wl.K * wl.E
+        mean_ms = statistics.mean(times)
+        achieved = flop / (mean_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            r, dt, th = oracle_sample_rate(wl, args.cpu_rows, 7)
+            cpu = {"value": r, "unit": UNIT, "cores": th, "kind": "oracle",
+                   "sample": f"{args.cpu_rows} seeded random output rows of {wl.name} (of {wl.N}), "
+                             f"{dt:.1f} s; direct fp64 Conv3d, OpenMP over rows"}
+        traffic = None
+        tfile = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tfile):
+            try:
+                traffic = json.load(open(tfile)).get(wl.name)
+            except Exception:
+                traffic = None
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded U[0,1) frames, N(0,0.02) weights)",
+            "config": config_of(wl, world),
+            "tflops": achieved,
+            "pct_of_peak": {"bf16_burst_measured": achieved / peak,
+                            "bf16_sustained_measured": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
+            "step_ms": {"mean": mean_ms, "median": statistics.median(times), "min": min(times)},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{src} bf16 dense (burst), MEASURED_PEAKS.json" if src == "measured"
+                         else "fallback 1590 TFLOP/s"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
+                    "d2h_bytes_per_step": out_bytes},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(result), flush=True)
+    if pg:
+        pg.destroy_process_group()
+    pe.close()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="grouped_16_images", choices=sorted(workloads.ALL))
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,202 @@
+/*
+ * pe.h -- C ABI of the B200 (sm_100a) vision PatchEmbed library (libpe.so).
+ *
+ * The operation.  Qwen2-VL / Qwen2.5-VL embed every video patch of C channels,
+ * tp frames and p x p pixels with a Conv3d whose kernel equals its stride, so
+ * each output row is the dot product of one flattened patch with one flattened
+ * filter (Qwen2.5VL-Vision Encode-PatchEmbed: the Conv3d description and the
+ * python验证 check; Optimize VLM PatchEmbed: Qwen3VLVisionPatchEmbed, "it's
+ * actually Linear projection"; patch详解 §4.3):
+ *
+ *     out[n, e] = bias[e] + sum_k  x[n, k] * W[e, k],   K = C * tp * p * p,
+ *
+ * with k(c, t, i, j) = ((c * tp + t) * p + i) * p + j, the view(-1, C, tp, p, p)
+ * order of the patch vectors and of the flattened [E, C, tp, p, p] weight.
+ *
+ * Arithmetic.  Operands are rounded to bf16 (round to nearest even) and
+ * multiplied on the tensor cores with fp32 accumulation; the bias is added in
+ * fp32; the result is stored as fp32 or rounded to bf16.  The pages cast the
+ * input to the weight's dtype before the conv (Qwen3VLVisionPatchEmbed.forward).
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are raw pointers.  "dev" means CUDA device memory of
+ *     the current device, "host" means ordinary host memory.  The caller owns
+ *     every input and output buffer; the library owns only what a handle holds
+ *     (packed weight, fp32 bias, normalisation constants, tensor-map
+ *     descriptors, a small device workspace and a device error word).
+ *   - Calls that take a stream are asynchronous on that stream and never
+ *     synchronise it.  Argument and shape errors are detected on the host and
+ *     returned before anything is launched or written.
+ *   - Dense row-major layouts only.  Device pointers must be 16-byte aligned.
+ *   - No C++ exception crosses this interface.  A CUDA error maps to
+ *     PE_ERR_CUDA.
+ *   - A handle may be used by concurrent forward calls on different streams,
+ *     except that grouped calls with more than PE_INLINE_ITEMS items upload
+ *     their item table into the handle's workspace and must therefore be
+ *     serialised (same stream).  pe_set_weight / pe_set_norm must not run
+ *     concurrently with anything else on the same handle.
+ */
+#ifndef PE_H_
+#define PE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st *pe_stream_t;
+
+typedef struct pe_handle pe_handle;
+
+typedef enum {
+    PE_OK = 0,
+    PE_ERR_INVALID_ARG = 1,    /* NULL pointer, non-positive size, bad enum value      */
+    PE_ERR_SHAPE = 2,          /* sizes inconsistent with the handle or the grid       */
+    PE_ERR_DTYPE = 3,          /* dtype not supported for this argument                */
+    PE_ERR_ALIGN = 4,          /* a device pointer is not 16-byte aligned              */
+    PE_ERR_NO_WEIGHT = 5,      /* forward called before pe_set_weight                  */
+    PE_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed                    */
+    PE_ERR_UNSUPPORTED = 7,    /* valid request outside what the kernels implement     */
+    PE_ERR_DEVICE_TIMEOUT = 8  /* a kernel gave up waiting on its pipeline (bounded wait) */
+} pe_status;
+
+typedef enum { PE_F32 = 0, PE_BF16 = 1 } pe_dtype;
+
+/* Grouped calls with at most this many items pass their item table inside the
+ * kernel launch; larger groups upload it into the handle's device workspace. */
+#define PE_INLINE_ITEMS 16
+
+/* Largest patch side the fused frames path accepts (p must also be even). */
+#define PE_MAX_PATCH 32
+
+/*
+ * pe_create -- allocate a handle for a PatchEmbed with hidden size E (out
+ * channels), C input channels, temporal patch tp and spatial patch p; has_bias
+ * != 0 makes pe_set_weight require a bias.  The constructor arguments are the
+ * module's config fields in_channels, temporal_patch_size, patch_size,
+ * hidden_size and bias (Qwen2.5VL-Vision Encode-PatchEmbed, the candle
+ * Qwen2_5VisionPatchEmbed::new; Optimize VLM PatchEmbed, Qwen3VLVisionPatchEmbed).
+ * Requires 1 <= C <= 4, 1 <= tp <= 4, 1 <= p, 16 <= E <= 65535 and E % 8 == 0,
+ * K = C*tp*p*p <= 8192.  Selects the current CUDA device; the handle must be
+ * used on that device.  *out receives the handle (NULL on failure).
+ * Errors: PE_ERR_INVALID_ARG, PE_ERR_UNSUPPORTED, PE_ERR_CUDA.
+ */
+pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out);
+
+/*
+ * pe_set_weight -- pack the Conv3d weight.
+ *   w    : dev [E, C, tp, p, p], dtype w_dt (PE_F32 or PE_BF16), dense.
+ *   bias : dev [E] of dtype b_dt, or NULL.  Must be non-NULL iff the handle was
+ *          created with has_bias.
+ * The weight is rounded to bf16 (RNE) into a handle-owned [E, Kpad] buffer
+ * (Kpad = K rounded up to 64, zero padded) -- the flatten(1, 4) of the candle
+ * module on Qwen2.5VL-Vision Encode-PatchEmbed -- and the bias is widened
+ * exactly to fp32.  Asynchronous on `stream`; w and bias may be freed once the
+ * stream has passed this point.  Errors: PE_ERR_INVALID_ARG, PE_ERR_DTYPE,
+ * PE_ERR_ALIGN, PE_ERR_CUDA.
+ */
+pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *bias,
+                        pe_dtype b_dt, pe_stream_t stream);
+
+/*
+ * pe_set_norm -- per-channel pixel normalisation used by the frames calls:
+ * x_hat = bf16_rne( fp32( fp32(x - mean[c]) / std[c] ) ), IEEE fp32 subtract
+ * and divide.  mean, std: host [C] fp32; std[c] must be finite and > 0.
+ * Default after pe_create: mean 0, std 1 (x_hat = bf16_rne(x)).
+ * Errors: PE_ERR_INVALID_ARG.
+ */
+pe_status pe_set_norm(pe_handle *h, const float *mean, const float *std);
+
+/*
+ * pe_forward_patches -- out = x @ W^T (+ bias) on already patchified rows.
+ *   x   : dev [N, K] of dtype x_dt (PE_BF16 or PE_F32), rows in
+ *         view(-1, C, tp, p, p) order as the Qwen2-VL processor emits
+ *         pixel_values (mytransformer README §3.2: pixel_values [N, 1176]).
+ *   out : dev [N, E] of dtype out_dt.
+ * Rows are processed in the given order; N may be 0 (nothing is launched).
+ * Errors: PE_ERR_INVALID_ARG, PE_ERR_DTYPE, PE_ERR_ALIGN, PE_ERR_NO_WEIGHT,
+ * PE_ERR_CUDA.
+ */
+pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
+                             void *out, pe_dtype out_dt, pe_stream_t stream);
+
+/*
+ * pe_forward_frames -- fused patchify + normalise + embed of one image/video.
+ *   frames   : dev [T, C, H, W] of dtype f_dt (PE_BF16 or PE_F32), dense.
+ *   grid_thw : host [3] = (gt, gh, gw) in patch units.  Requires H == gh*p,
+ *              W == gw*p and ceil(T / tp) == gt (patch详解 §4.5).  When T is not
+ *              a multiple of tp the last frame is repeated, so a single image
+ *              (T = 1) is duplicated to tp frames.
+ *   merge    : 1 or 2.  With merge = m > 1 the rows come in spatial-merge order:
+ *              m x m windows consecutive, windows row-major over
+ *              (t, h/m, w/m), (dh, dw) row-major inside a window (mytransformer
+ *              README §3.2 PatchMerger and §4.1; Qwen2.5VL语言模型 MRoPE example:
+ *              merged grid row-major, h outer).  gh and gw must be multiples of m.
+ *   out      : dev [gt*gh*gw, E] of dtype out_dt.
+ * Requires p even and p <= PE_MAX_PATCH.  The [N, K] patch matrix is never
+ * written to memory.  Errors: as pe_forward_patches plus PE_ERR_SHAPE,
+ * PE_ERR_UNSUPPORTED.
+ */
+pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H,
+                            int W, const int32_t grid_thw[3], int merge, void *out,
+                            pe_dtype out_dt, pe_stream_t stream);
+
+/*
+ * pe_forward_frames_grouped -- pe_forward_frames over n items in ONE launch; the
+ * rows of item i follow those of items 0..i-1 (the packed sequence of the vision
+ * forward with grid_thw of shape (num_images_or_videos, 3): Optimize VLM
+ * PatchEmbed, the vision model's forward).
+ *   frames   : host array of n dev pointers, item i is [THW[3i], C, THW[3i+1], THW[3i+2]]
+ *   THW      : host [n, 3] frame dims (T, H, W) per item
+ *   grid_thw : host [n, 3] patch grid per item
+ *   out      : dev [sum_i gt_i*gh_i*gw_i, E]
+ * All items share f_dt, merge and out_dt.  Errors: as pe_forward_frames.
+ */
+pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                    const int32_t *THW, const int32_t *grid_thw, int merge,
+                                    void *out, pe_dtype out_dt, pe_stream_t stream);
+
+/*
+ * pe_patchify -- test hook: the fused producer's gather and normalisation
+ * written out to memory instead of feeding the tensor cores.
+ *   rows : dev [sum_i N_i, K] of dtype rows_dt (PE_BF16 or PE_F32; values are
+ *          bf16-exact either way), row order and k order as in the forward calls.
+ * Other arguments as pe_forward_frames_grouped.
+ */
+pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                      const int32_t *THW, const int32_t *grid_thw, int merge, void *rows,
+                      pe_dtype rows_dt, pe_stream_t stream);
+
+/*
+ * pe_num_patches -- sum_i gt_i * gh_i * gw_i over host grid_thw [n, 3];
+ * 0 for n == 0; -1 on a NULL pointer with n > 0, negative n or a
+ * non-positive entry.
+ */
+int64_t pe_num_patches(const int32_t *grid_thw, int n);
+
+/*
+ * pe_last_error -- read and clear the handle's device error word.  Call after
+ * synchronising the streams the handle ran on.  Returns PE_OK, or
+ * PE_ERR_DEVICE_TIMEOUT if a kernel stopped waiting on its pipeline (it then
+ * wrote an incomplete output and left the device usable), or PE_ERR_CUDA if
+ * the word could not be read.
+ */
+pe_status pe_last_error(pe_handle *h);
+
+/* Static English text for a status code (never NULL). */
+const char *pe_status_string(pe_status s);
+
+/* Release the handle and everything it owns.  NULL is a no-op.  Synchronises
+ * the device first so no launch still uses the handle's buffers. */
+void pe_destroy(pe_handle *h);
+
+/* Device this handle was created on, or -1 for NULL. */
+int pe_device(const pe_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PE_H_ */

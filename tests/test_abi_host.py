@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds for
+sm_100a, loads, exports every entry point the header declares, and its pure
+host functions behave."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from vlm_vision_patch_b200 import build, _binding
+    build.build()
+    return _binding.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_matches_binding_exports():
+    from vlm_vision_patch_b200 import _binding
+    assert declared_functions() == sorted(_binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from vlm_vision_patch_b200 import _binding
+    out = subprocess.run(["nm", "-D", "--defined-only", _binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (pe_[a-z_]+)\b", out))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert hasattr(lib, f)
+
+
+def test_library_is_built_for_sm100a(lib):
+    from vlm_vision_patch_b200 import _binding
+    out = subprocess.run(["cuobjdump", "--list-elf", _binding.LIB_PATH], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+def test_status_strings(lib):
+    from vlm_vision_patch_b200 import _binding
+    seen = set()
+    for code in range(9):
+        s = _binding.status_string(code)
+        assert s and s != "unknown status"
+        seen.add(s)
+    assert len(seen) == 9
+    assert _binding.status_string(99) == "unknown status"
+
+
+def test_num_patches(lib):
+    from vlm_vision_patch_b200 import _binding
+    assert _binding.pe_num_patches([(1, 36, 54)]) == 1944
+    assert _binding.pe_num_patches([(1, 16, 64), (4, 14, 14)]) == 1024 + 784
+    assert _binding.pe_num_patches([]) == 0
+    assert _binding.pe_num_patches([(1, 0, 4)]) == -1
+    assert lib.pe_num_patches(None, 1) == -1
+
+
+def test_null_handle_calls_are_rejected(lib):
+    assert lib.pe_last_error(None) == 1
+    assert lib.pe_set_norm(None, None, None) == 1
+    assert lib.pe_forward_patches(None, None, 1, 0, None, 1, None) == 1
+    assert lib.pe_device(None) == -1
+    lib.pe_destroy(None)
+    h = ctypes.c_void_p()
+    assert lib.pe_create(1280, 3, 2, 14, 0, None) == 1
+    assert lib.pe_create(1004, 3, 2, 14, 0, ctypes.byref(h)) == 1     # E % 8 != 0
+    assert lib.pe_create(1280, 5, 2, 14, 0, ctypes.byref(h)) == 1     # C > 4
+    assert h.value is None
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_create_without_gpu_fails_cleanly(lib):
+    h = ctypes.c_void_p()
+    rc = lib.pe_create(1280, 3, 2, 14, 0, ctypes.byref(h))
+    assert rc != 0 and h.value is None

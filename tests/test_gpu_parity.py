@@ -1,0 +1,319 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Tolerance (per output element): |gpu - oracle| <= 1e-3 * sum_k |x_k * w_k| for
+fp32 output, plus one bf16 ulp of the oracle value for bf16 output.  Integer,
+one-hot and patchify cases are bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from vlm_vision_patch_b200 import PatchEmbed, PEError
+from tests.gpu_util import assert_within_tolerance, mask_of, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _pe(wl_or_args, weight, bias, mean=None, std=None):
+    E, C, tp, p = wl_or_args
+    pe = PatchEmbed(E, C, tp, p, bias is not None)
+    pe.set_weight(weight.to(DEV).contiguous(), None if bias is None else bias.to(DEV).contiguous())
+    if mean is not None:
+        pe.set_norm(mean, std)
+    return pe
+
+
+def _bits32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").float().numpy().view(np.uint32)
+
+
+# --------------------------------------------------------------- patches form
+
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("N", [1, 128, 300])
+def test_patches_integer_inputs_bit_exact(x_dtype, N):
+    """Small integers keep every product and partial sum exact in fp32, so the
+    fp32 output must equal the oracle bit for bit, and bf16 output must be its
+    bf16 rounding (Optimize VLM PatchEmbed's randint check, R1 == R2)."""
+    C, tp, p, E = 3, 2, 14, 1280
+    K = C * tp * p * p
+    x = workloads.small_ints((N, K), 31, 0, 2)
+    w = workloads.small_ints((E, C, tp, p, p), 32, -4, 4)
+    b = workloads.small_ints((E,), 33, -100, 100)
+    ref, _ = oracle.conv3d_patches(x, w, b, C, tp, p)
+    pe = _pe((E, C, tp, p), w, b)
+    xd = x.to(x_dtype).to(DEV)
+    out32 = pe.forward_patches(xd, out_dtype=torch.float32)
+    out16 = pe.forward_patches(xd, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    assert np.array_equal(out32.cpu().double().numpy(), ref)
+    ref16 = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16)
+    assert torch.equal(out16.cpu(), ref16)
+
+
+def test_patches_one_hot_recovers_weight():
+    C, tp, p, E = 3, 2, 14, 1280
+    K = C * tp * p * p
+    w = workloads.normal((E, C, tp, p, p), 34, std=0.02)
+    b = workloads.normal((E,), 35, std=0.02)
+    pe = _pe((E, C, tp, p), w, b)
+    x = torch.eye(K, dtype=torch.bfloat16, device=DEV)
+    out = pe.forward_patches(x, out_dtype=torch.float32)
+    ref, _ = oracle.conv3d_patches(torch.eye(K), w, b, C, tp, p)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().double().numpy(), ref)
+    zero = pe.forward_patches(torch.zeros(5, K, dtype=torch.bfloat16, device=DEV), out_dtype=torch.float32)
+    assert torch.equal(zero.cpu(), b.float().expand(5, E))
+
+
+def test_patches_fp32_1024_workload():
+    """pixel_values [1024, 1176] fp32 N(0,1), Kaiming-uniform fp32 weight, fp32 out."""
+    wl = workloads.patches_fp32_1024()
+    pe = _pe((wl.E, wl.C, wl.tp, wl.p), wl.weight, wl.bias)
+    out = pe.forward_patches(wl.patches.to(DEV), out_dtype=torch.float32)
+    ref, mag = oracle.conv3d_patches(wl.patches, wl.weight, wl.bias, wl.C, wl.tp, wl.p)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    assert_within_tolerance(out, ref, mag, what=wl.name)
+
+
+@pytest.mark.parametrize("C,tp,p,E,N,bias,x_dtype,out_dtype", [
+    (3, 2, 14, 1280, 129, False, torch.bfloat16, torch.bfloat16),
+    (3, 2, 16, 1152, 1000, True, torch.bfloat16, torch.float32),
+    (3, 1, 3, 72, 257, True, torch.float32, torch.float32),      # K=27: no TMA, ragged K
+    (1, 2, 4, 16, 5, False, torch.bfloat16, torch.bfloat16),     # K=32
+    (3, 2, 2, 40, 130, True, torch.bfloat16, torch.float32),     # K=24, E tail chunk
+    (2, 2, 14, 200, 384, False, torch.float32, torch.bfloat16),  # K=784, E=200 (partial tile)
+])
+def test_patches_shapes(C, tp, p, E, N, bias, x_dtype, out_dtype):
+    K = C * tp * p * p
+    x = workloads.normal((N, K), 40 + N)
+    w = workloads.normal((E, C, tp, p, p), 41 + E, std=0.05)
+    b = workloads.normal((E,), 42, std=0.05) if bias else None
+    pe = _pe((E, C, tp, p), w, b)
+    out = pe.forward_patches(x.to(x_dtype).to(DEV), out_dtype=out_dtype)
+    ref, mag = oracle.conv3d_patches(x.to(x_dtype), w, b, C, tp, p)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    assert_within_tolerance(out, ref, mag, what=f"patches {C},{tp},{p},{E},{N}")
+
+
+def test_patches_empty_and_bn_override(monkeypatch):
+    C, tp, p, E = 3, 2, 14, 256
+    w = workloads.normal((E, C, tp, p, p), 43, std=0.02)
+    pe = _pe((E, C, tp, p), w, None)
+    out = pe.forward_patches(torch.empty(0, C * tp * p * p, dtype=torch.bfloat16, device=DEV))
+    assert out.shape == (0, E)
+    x = workloads.normal((517, C * tp * p * p), 44)
+    ref, mag = oracle.conv3d_patches(x, w, None, C, tp, p)
+    for bn in ("64", "128", "256"):
+        monkeypatch.setenv("PE_BN", bn)
+        o = pe.forward_patches(x.to(torch.bfloat16).to(DEV), out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert_within_tolerance(o, ref, mag, what=f"BN={bn}")
+
+
+# ---------------------------------------------------------------- frames form
+
+def _run_frames(wl, out_dtype=None, rows=None):
+    pe = _pe((wl.E, wl.C, wl.tp, wl.p), wl.weight, wl.bias, wl.mean, wl.std)
+    od = out_dtype or wl.out_dtype
+    frames = [it.frames.to(DEV) for it in wl.items]
+    grids = [it.grid for it in wl.items]
+    if len(frames) == 1:
+        out = pe.forward_frames(frames[0], grids[0], wl.merge, out_dtype=od)
+    else:
+        out = pe.forward_frames_grouped(frames, grids, wl.merge, out_dtype=od)
+    mask = None if rows is None else mask_of(rows, wl.N)
+    ref, mag = oracle.conv3d_grouped([(it.frames, it.grid) for it in wl.items], wl.merge, wl.mean, wl.std,
+                                     wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    return pe, out, ref, mag
+
+
+@pytest.mark.parametrize("name", ["image_224x896", "video_8x224_p16", "image_448_e1152"])
+def test_frames_workloads_all_rows(name):
+    wl = workloads.ALL[name]()
+    _, out, ref, mag = _run_frames(wl)
+    assert_within_tolerance(out, ref, mag, what=name)
+
+
+def test_frames_fp32_out_and_fp32_frames():
+    wl = workloads.image_224x896()
+    for it in wl.items:
+        it.frames = it.frames.float()
+    _, out, ref, mag = _run_frames(wl, out_dtype=torch.float32)
+    assert out.dtype == torch.float32
+    assert_within_tolerance(out, ref, mag, what="fp32 frames / fp32 out")
+
+
+@pytest.mark.parametrize("T,gh,gw,merge,p,tp,E,bias", [
+    (3, 4, 6, 2, 14, 2, 1280, True),     # odd T: last frame repeated
+    (1, 6, 2, 1, 14, 2, 256, False),     # raster order
+    (5, 2, 4, 2, 16, 2, 128, True),
+    (2, 8, 10, 2, 4, 2, 64, False),      # small even p (generic kernel)
+    (1, 2, 2, 2, 14, 2, 1280, False),    # 4 rows only
+    (4, 10, 14, 2, 6, 1, 96, True),      # tp = 1
+])
+def test_frames_small_shapes(T, gh, gw, merge, p, tp, E, bias):
+    C = 3
+    gt = -(-T // tp)
+    wl = workloads.Workload(f"frames_{T}_{gh}_{gw}_{p}", E, C, tp, p,
+                            workloads.normal((E, C, tp, p, p), 50 + p, std=0.02, dtype=torch.bfloat16),
+                            workloads.normal((E,), 51, std=0.02) if bias else None, torch.bfloat16, merge=merge,
+                            items=[workloads.Item(workloads.uniform01((T, C, gh * p, gw * p), 52 + T), (gt, gh, gw))],
+                            mean=workloads.CLIP_MEAN, std=workloads.CLIP_STD)
+    _, out, ref, mag = _run_frames(wl)
+    assert_within_tolerance(out, ref, mag, what=wl.name)
+
+
+def test_grouped_16_images_sampled_rows():
+    """The 16-image grouped workload at full size, checked on sampled rows
+    (every item boundary included)."""
+    wl = workloads.grouped_16_images()
+    bounds, off = [], 0
+    for it in wl.items:
+        n = it.grid[0] * it.grid[1] * it.grid[2]
+        bounds += [off, off + 1, off + n - 1]
+        off += n
+    rows = sample_rows(wl.N, 3000, 60, bounds)
+    _, out, ref, mag = _run_frames(wl, rows=rows)
+    assert_within_tolerance(out, ref, mag, rows=rows, what=wl.name)
+
+
+def test_grouped_small_items_all_rows():
+    C, tp, p, E = 3, 2, 14, 1280
+    grids = [(1, 2, 2), (2, 4, 6), (1, 8, 2), (1, 2, 16), (3, 6, 6)]
+    items = [workloads.Item(workloads.uniform01((2 * g[0] - (i % 2 if g[0] > 1 else 0), C, g[1] * p, g[2] * p),
+                                                70 + i), g) for i, g in enumerate(grids)]
+    wl = workloads.Workload("grouped_small", E, C, tp, p,
+                            workloads.normal((E, C, tp, p, p), 71, std=0.02, dtype=torch.bfloat16), None,
+                            torch.bfloat16, merge=2, items=items, mean=workloads.CLIP_MEAN,
+                            std=workloads.CLIP_STD)
+    _, out, ref, mag = _run_frames(wl)
+    assert_within_tolerance(out, ref, mag, what=wl.name)
+
+
+def test_grouped_many_items_device_table():
+    """More items than fit in the launch parameters: the item table goes through
+    the handle's device workspace."""
+    C, tp, p, E = 3, 2, 14, 256
+    rng = np.random.default_rng(80)
+    grids = [(1, int(2 * rng.integers(1, 4)), int(2 * rng.integers(1, 4))) for _ in range(40)]
+    items = [workloads.Item(workloads.uniform01((1, C, g[1] * p, g[2] * p), 81 + i), g) for i, g in enumerate(grids)]
+    wl = workloads.Workload("grouped_40", E, C, tp, p,
+                            workloads.normal((E, C, tp, p, p), 82, std=0.02, dtype=torch.bfloat16), None,
+                            torch.bfloat16, merge=2, items=items, mean=workloads.CLIP_MEAN,
+                            std=workloads.CLIP_STD)
+    _, out, ref, mag = _run_frames(wl)
+    assert_within_tolerance(out, ref, mag, what=wl.name)
+
+
+def test_long_video_sampled_rows():
+    """[64, 3, 896, 896] frames, grid [32, 64, 64] -> 131072 rows, sampled."""
+    wl = workloads.long_video_64x896()
+    rows = sample_rows(wl.N, 768, 90)
+    _, out, ref, mag = _run_frames(wl, rows=rows)
+    assert_within_tolerance(out, ref, mag, rows=rows, what=wl.name)
+
+
+def test_frames_deterministic():
+    wl = workloads.image_448_e1152()
+    pe = _pe((wl.E, wl.C, wl.tp, wl.p), wl.weight, wl.bias, wl.mean, wl.std)
+    f = wl.items[0].frames.to(DEV)
+    a = pe.forward_frames(f, wl.items[0].grid, 2)
+    b = pe.forward_frames(f, wl.items[0].grid, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ patchify
+
+@pytest.mark.parametrize("T,gh,gw,merge,p,tp,fdt", [
+    (1, 16, 64, 2, 14, 2, torch.bfloat16),
+    (3, 4, 6, 2, 14, 2, torch.bfloat16),
+    (8, 14, 14, 2, 16, 2, torch.bfloat16),
+    (2, 6, 4, 1, 14, 2, torch.float32),
+    (5, 4, 8, 2, 4, 2, torch.float32),
+    (2, 6, 6, 2, 6, 1, torch.bfloat16),
+])
+def test_patchify_bit_exact(T, gh, gw, merge, p, tp, fdt):
+    C = 3
+    gt = -(-T // tp)
+    frames = workloads.uniform01((T, C, gh * p, gw * p), 100 + p + T).to(fdt)
+    pe = PatchEmbed(64, C, tp, p, False)
+    pe.set_norm(workloads.CLIP_MEAN, workloads.CLIP_STD)
+    rows = pe.patchify([frames.to(DEV)], [(gt, gh, gw)], merge, rows_dtype=torch.float32)
+    ref = oracle.patchify(frames, (gt, gh, gw), merge, workloads.CLIP_MEAN, workloads.CLIP_STD, C, tp, p)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits32(rows), ref.view(np.uint32))
+    rows16 = pe.patchify([frames.to(DEV)], [(gt, gh, gw)], merge, rows_dtype=torch.bfloat16)
+    assert np.array_equal(_bits32(rows16), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("mean,std", [(workloads.CLIP_MEAN, workloads.CLIP_STD),
+                                      ((0.5, -0.25, 3.0), (0.5, 0.1, 7.0)),
+                                      ((0.0, 0.0, 0.0), (1.0, 1.0, 1.0))])
+def test_normalization_exhaustive_bf16(mean, std):
+    """Every finite bf16 value in every channel: the kernel's fp32 (x-mean)/std
+    then bf16 rounding equals the oracle's IEEE divide bit for bit."""
+    vals = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32)
+    vals = vals[np.isfinite(vals)]
+    n = vals.size                                   # 65024 values
+    W = 128                                         # p = 2 -> gw = 64
+    H = -(-n // W)
+    H = -(-H // 4) * 4
+    buf = np.zeros(H * W, dtype=np.float32)
+    buf[:n] = vals
+    frames = torch.from_numpy(np.stack([np.roll(buf, 977 * c) for c in range(3)]).reshape(1, 3, H, W))
+    frames = frames.to(torch.bfloat16)
+    pe = PatchEmbed(64, 3, 1, 2, False)
+    pe.set_norm(mean, std)
+    rows = pe.patchify([frames.to(DEV)], [(1, H // 2, W // 2)], 2, rows_dtype=torch.float32)
+    ref = oracle.patchify(frames, (1, H // 2, W // 2), 2, mean, std, 3, 1, 2)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits32(rows), ref.view(np.uint32))
+
+
+# --------------------------------------------------------------- error paths
+
+def test_error_paths():
+    pe = PatchEmbed(256, 3, 2, 14, False)
+    K = 3 * 2 * 14 * 14
+    x = torch.zeros(4, K, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(PEError) as e:
+        pe.forward_patches(x)
+    assert e.value.status == "PE_ERR_NO_WEIGHT"
+    w = workloads.normal((256, 3, 2, 14, 14), 1, std=0.02).to(DEV)
+    with pytest.raises(PEError) as e:
+        pe.set_weight(w, torch.zeros(256, device=DEV))          # handle has no bias
+    assert e.value.status == "PE_ERR_INVALID_ARG"
+    pe.set_weight(w)
+    f = torch.zeros(1, 3, 224, 224, dtype=torch.bfloat16, device=DEV)
+    for grid, merge, code in [((1, 16, 15), 2, "PE_ERR_SHAPE"), ((1, 15, 16), 2, "PE_ERR_SHAPE"),
+                              ((2, 16, 16), 2, "PE_ERR_SHAPE"), ((1, 16, 16), 3, "PE_ERR_INVALID_ARG")]:
+        with pytest.raises(PEError) as e:
+            pe.forward_frames(f, grid, merge)
+        assert e.value.status == code
+    with pytest.raises(PEError) as e:
+        pe.forward_patches(x.view(-1)[1:1 + 3 * K].view(3, K))   # misaligned pointer
+    assert e.value.status == "PE_ERR_ALIGN"
+    with pytest.raises(PEError) as e:
+        pe.set_norm((0.5, 0.5, 0.5), (1.0, 0.0, 1.0))
+    assert e.value.status == "PE_ERR_INVALID_ARG"
+    with pytest.raises(PEError) as e:
+        PatchEmbed(1004, 3, 2, 14)                                  # E % 8 != 0
+    assert e.value.status == "PE_ERR_INVALID_ARG"
+    odd = PatchEmbed(64, 3, 2, 3, False)
+    odd.set_weight(workloads.normal((64, 3, 2, 3, 3), 2).to(DEV))
+    with pytest.raises(PEError) as e:
+        odd.forward_frames(torch.zeros(2, 3, 6, 6, device=DEV), (1, 2, 2), 2)
+    assert e.value.status == "PE_ERR_UNSUPPORTED"
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0

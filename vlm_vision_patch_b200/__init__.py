@@ -1,0 +1,123 @@
+"""B200-native vision PatchEmbed (Qwen2-VL / Qwen2.5-VL) over the libpe.so C ABI.
+
+``PatchEmbed`` is a convenience wrapper holding one ``pe_handle``; every method
+forwards to the same-named C entry point (``_binding``) with torch tensors
+turned into raw device pointers and the current CUDA stream.  PyTorch only
+provides device memory and streams here; all arithmetic runs in libpe.so.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import _binding as B
+from ._binding import PE_BF16, PE_F32, PEError, load  # noqa: F401
+
+__all__ = ["PatchEmbed", "PEError", "PE_F32", "PE_BF16", "load", "num_patches"]
+
+
+def _dt(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return PE_F32
+    if t == torch.bfloat16:
+        return PE_BF16
+    raise TypeError(f"unsupported dtype {t}; use torch.float32 or torch.bfloat16")
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def num_patches(grid_thw: Sequence[Sequence[int]]) -> int:
+    return B.pe_num_patches(grid_thw)
+
+
+class PatchEmbed:
+    """Conv3d(C, E, kernel=stride=(tp, p, p)) as one fused sm_100a kernel."""
+
+    def __init__(self, E: int, C: int = 3, tp: int = 2, p: int = 14, bias: bool = False):
+        self.E, self.C, self.tp, self.p, self.has_bias = E, C, tp, p, bias
+        self.K = C * tp * p * p
+        self.h = B.pe_create(E, C, tp, p, bias)
+
+    # ------------------------------------------------------------ lifetime
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            B.pe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------ state
+    def set_weight(self, w: torch.Tensor, bias: Optional[torch.Tensor] = None, stream=None) -> None:
+        B.pe_set_weight(self.h, _dev(w, "weight"), _dt(w.dtype),
+                        None if bias is None else _dev(bias, "bias"),
+                        _dt(bias.dtype) if bias is not None else PE_F32, _stream(stream))
+
+    def set_norm(self, mean: Sequence[float], std: Sequence[float]) -> None:
+        B.pe_set_norm(self.h, mean, std)
+
+    def last_error(self) -> int:
+        return B.pe_last_error(self.h)
+
+    # ------------------------------------------------------------ forward
+    def _out(self, n: int, out, out_dtype, device):
+        if out is None:
+            out = torch.empty((n, self.E), dtype=out_dtype, device=device)
+        return out
+
+    def forward_patches(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+        out = self._out(x.shape[0], out, out_dtype, x.device)
+        B.pe_forward_patches(self.h, _dev(x, "x"), _dt(x.dtype), x.shape[0], _dev(out, "out"),
+                             _dt(out.dtype), _stream(stream))
+        return out
+
+    def forward_frames(self, frames: torch.Tensor, grid_thw: Sequence[int], merge: int = 2,
+                       out: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
+                       stream=None) -> torch.Tensor:
+        T, C, H, W = frames.shape
+        n = int(grid_thw[0]) * int(grid_thw[1]) * int(grid_thw[2])
+        out = self._out(n, out, out_dtype, frames.device)
+        B.pe_forward_frames(self.h, _dev(frames, "frames"), _dt(frames.dtype), T, H, W, grid_thw, merge,
+                            _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        return out
+
+    def forward_frames_grouped(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]],
+                               merge: int = 2, out: Optional[torch.Tensor] = None,
+                               out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+        n = sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
+        out = self._out(n, out, out_dtype, frames[0].device)
+        dts = {f.dtype for f in frames}
+        if len(dts) != 1:
+            raise TypeError("all items must share one dtype")
+        B.pe_forward_frames_grouped(self.h, [_dev(f, "frames") for f in frames], _dt(frames[0].dtype),
+                                    [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames], grid_thw,
+                                    merge, _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        return out
+
+    def patchify(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]], merge: int = 2,
+                 rows_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+        n = sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
+        rows = torch.empty((n, self.K), dtype=rows_dtype, device=frames[0].device)
+        B.pe_patchify(self.h, [_dev(f, "frames") for f in frames], _dt(frames[0].dtype),
+                      [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames], grid_thw, merge,
+                      _dev(rows, "rows"), _dt(rows.dtype), _stream(stream))
+        return rows

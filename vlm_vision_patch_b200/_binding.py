@@ -1,0 +1,159 @@
+"""ctypes binding of libpe.so: argument marshalling only.
+
+Every function here has the name and argument order of the C entry point it
+wraps (include/pe.h).  Tensors are passed as raw device pointers; streams as
+the raw CUDA stream handle.  There is no fallback: if libpe.so is missing or a
+call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpe.so")
+
+PE_F32, PE_BF16 = 0, 1
+STATUS = {
+    0: "PE_OK", 1: "PE_ERR_INVALID_ARG", 2: "PE_ERR_SHAPE", 3: "PE_ERR_DTYPE",
+    4: "PE_ERR_ALIGN", 5: "PE_ERR_NO_WEIGHT", 6: "PE_ERR_CUDA", 7: "PE_ERR_UNSUPPORTED",
+    8: "PE_ERR_DEVICE_TIMEOUT",
+}
+PE_INLINE_ITEMS = 16
+PE_MAX_PATCH = 32
+
+# Every symbol include/pe.h declares.
+EXPORTS = (
+    "pe_create", "pe_set_weight", "pe_set_norm", "pe_forward_patches", "pe_forward_frames",
+    "pe_forward_frames_grouped", "pe_patchify", "pe_num_patches", "pe_last_error",
+    "pe_status_string", "pe_destroy", "pe_device",
+)
+
+
+class PEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+        super().__init__(f"{fn} failed: {self.status} ({status_string(code)})")
+
+
+_lib = None
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libpe.so (build it first with vlm_vision_patch_b200.build)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libpe.so not found at {p}: build it with "
+                           "`python -m vlm_vision_patch_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(p)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    f32p = ctypes.POINTER(ctypes.c_float)
+    sig = {
+        "pe_create": ([i32, i32, i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "pe_set_weight": ([vp, vp, i32, vp, i32, vp], i32),
+        "pe_set_norm": ([vp, f32p, f32p], i32),
+        "pe_forward_patches": ([vp, vp, i32, i64, vp, i32, vp], i32),
+        "pe_forward_frames": ([vp, vp, i32, i32, i32, i32, i32p, i32, vp, i32, vp], i32),
+        "pe_forward_frames_grouped": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
+        "pe_patchify": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
+        "pe_num_patches": ([i32p, i32], i64),
+        "pe_last_error": ([vp], i32),
+        "pe_status_string": ([i32], ctypes.c_char_p),
+        "pe_destroy": ([vp], None),
+        "pe_device": ([vp], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise PEError(fn, code)
+
+
+def _i32arr(vals: Sequence[int]):
+    return (ctypes.c_int32 * len(vals))(*[int(v) for v in vals])
+
+
+def _f32arr(vals: Sequence[float]):
+    return (ctypes.c_float * len(vals))(*[float(v) for v in vals])
+
+
+def _ptrs(ptrs: Sequence[int]):
+    return (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(int(p)) for p in ptrs])
+
+
+# ----------------------------------------------------------- raw entry points
+
+def status_string(code: int) -> str:
+    return load().pe_status_string(int(code)).decode()
+
+
+def pe_create(E: int, C: int, tp: int, p: int, has_bias: bool) -> int:
+    h = ctypes.c_void_p()
+    _check("pe_create", load().pe_create(E, C, tp, p, int(bool(has_bias)), ctypes.byref(h)))
+    return h.value
+
+
+def pe_destroy(h: int) -> None:
+    load().pe_destroy(h)
+
+
+def pe_device(h: int) -> int:
+    return int(load().pe_device(h))
+
+
+def pe_set_weight(h: int, w_ptr: int, w_dt: int, bias_ptr: Optional[int], b_dt: int, stream: int) -> None:
+    _check("pe_set_weight", load().pe_set_weight(h, w_ptr, w_dt, bias_ptr, b_dt, stream))
+
+
+def pe_set_norm(h: int, mean: Sequence[float], std: Sequence[float]) -> None:
+    _check("pe_set_norm", load().pe_set_norm(h, _f32arr(mean), _f32arr(std)))
+
+
+def pe_forward_patches(h: int, x_ptr: int, x_dt: int, N: int, out_ptr: int, out_dt: int, stream: int) -> None:
+    _check("pe_forward_patches", load().pe_forward_patches(h, x_ptr, x_dt, N, out_ptr, out_dt, stream))
+
+
+def pe_forward_frames(h: int, f_ptr: int, f_dt: int, T: int, H: int, W: int, grid_thw: Sequence[int],
+                      merge: int, out_ptr: int, out_dt: int, stream: int) -> None:
+    _check("pe_forward_frames", load().pe_forward_frames(h, f_ptr, f_dt, T, H, W, _i32arr(grid_thw), merge,
+                                                          out_ptr, out_dt, stream))
+
+
+def pe_forward_frames_grouped(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence[int]],
+                              grid_thw: Sequence[Sequence[int]], merge: int, out_ptr: int, out_dt: int,
+                              stream: int) -> None:
+    n = len(f_ptrs)
+    _check("pe_forward_frames_grouped", load().pe_forward_frames_grouped(
+        h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
+        _i32arr([v for g in grid_thw for v in g]), merge, out_ptr, out_dt, stream))
+
+
+def pe_patchify(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence[int]],
+                grid_thw: Sequence[Sequence[int]], merge: int, rows_ptr: int, rows_dt: int,
+                stream: int) -> None:
+    n = len(f_ptrs)
+    _check("pe_patchify", load().pe_patchify(
+        h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
+        _i32arr([v for g in grid_thw for v in g]), merge, rows_ptr, rows_dt, stream))
+
+
+def pe_num_patches(grid_thw: Sequence[Sequence[int]]) -> int:
+    flat = [v for g in grid_thw for v in g]
+    return int(load().pe_num_patches(_i32arr(flat) if flat else None, len(grid_thw)))
+
+
+def pe_last_error(h: int) -> int:
+    return int(load().pe_last_error(h))

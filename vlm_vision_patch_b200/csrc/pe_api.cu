@@ -1,0 +1,477 @@
+// C ABI of the vision PatchEmbed library (see include/pe.h for the contract of
+// every entry point).  Host side: argument validation, weight packing, TMA
+// tensor-map encoding, tile-shape choice and kernel launches.  Nothing here
+// computes on the host; every step of the forward path runs in the kernels of
+// pe_kernels.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/pe.h"
+#include "pe_kernels.cuh"
+
+using namespace pe;
+
+struct pe_handle {
+    int dev = -1;
+    int E = 0, C = 0, tp = 0, p = 0, K = 0, Kpad = 0;
+    bool has_bias = false;
+    bool weight_set = false;
+    uint16_t *wpack = nullptr;  // dev [E, Kpad] bf16
+    float *bias = nullptr;      // dev [E] fp32 (has_bias)
+    int *err = nullptr;         // dev error word
+    float mean[4] = {0, 0, 0, 0};
+    float stdv[4] = {1, 1, 1, 1};
+    CUtensorMap tmap_w[3];      // box rows 64, 128, 256
+    int num_sms = 0;
+    int smem_optin = 0;
+    // item table for grouped calls beyond PE_INLINE_ITEMS
+    ItemDesc *items_dev = nullptr;
+    ItemDesc *items_pinned = nullptr;
+    int items_cap = 0;
+    cudaEvent_t items_evt = nullptr;
+    bool items_evt_pending = false;
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous, row stride `ld` elements),
+// box [box_rows, 64], 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t ld,
+                    uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(int d) { return d == PE_F32 || d == PE_BF16; }
+
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+int bn_override() {
+    const char *s = std::getenv("PE_BN");
+    if (!s) return 0;
+    const int v = std::atoi(s);
+    return (v == 64 || v == 128 || v == 256) ? v : 0;
+}
+
+// Tile width: frames tiles pay the gather once per tile whatever BN is, so use
+// the widest BN unless the problem is too small to fill the GPU in one wave;
+// TMA-fed patch tiles are cheap to refill, so prefer enough tiles for all SMs.
+int choose_bn(int64_t N, int E, int num_sms, bool gather_fed) {
+    if (const int o = bn_override()) return o;
+    const int64_t mt = (N + kBM - 1) / kBM;
+    auto tiles = [&](int bn) { return mt * ((E + bn - 1) / bn); };
+    if (tiles(256) >= num_sms) return 256;
+    if (gather_fed) {
+        // Less than one wave even at BN=256: every CTA runs one tile, so the
+        // narrowest BN that still fits one wave finishes first.
+        if (tiles(64) <= num_sms) return 64;
+        if (tiles(128) <= num_sms) return 128;
+        return 256;
+    }
+    if (tiles(128) >= num_sms) return 128;
+    return 64;
+}
+
+template <int AMODE, int PT, bool F32IN>
+cudaError_t launch_fwd(const pe_handle *h, const FwdParams &P, const CUtensorMap &tx, size_t smem,
+                       int grid, cudaStream_t st) {
+    auto kern = pe_fwd_kernel<AMODE, PT, F32IN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int bi = P.bn == 64 ? 0 : (P.bn == 128 ? 1 : 2);
+    kern<<<grid, kThreads, smem, st>>>(h->tmap_w[bi], tx, P);
+    return cudaGetLastError();
+}
+
+void fill_common(const pe_handle *h, FwdParams &P) {
+    std::memset(&P, 0, sizeof(P));
+    P.E = h->E;
+    P.C = h->C;
+    P.TP = h->tp;
+    P.P = h->p;
+    P.K = h->K;
+    P.Kpad = h->Kpad;
+    for (int c = 0; c < 4; ++c) {
+        P.mean[c] = h->mean[c];
+        P.stdv[c] = h->stdv[c];
+        P.nstdv[c] = -h->stdv[c];
+        P.rstd[c] = 1.0f / h->stdv[c];  // IEEE division on the host: correctly rounded
+    }
+    P.bias = h->has_bias ? h->bias : nullptr;
+    P.err = h->err;
+}
+
+// Ring depths and per-tile stage counts; returns the dynamic shared memory size.
+size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
+    P.num_ksteps = (P.K + 15) / 16;
+    P.n_b_stages = (P.num_ksteps + 3) / 4;
+    if (amode == kAModeFrames) {
+        P.a_stage_bytes = 2048 * P.P;  // 8 segments of p pixels, 128 rows
+        P.n_a_stages = (P.C * P.TP * P.P + 7) / 8;
+    } else {
+        P.a_stage_bytes = kBM * kBK * 2;
+        P.n_a_stages = P.n_b_stages;
+    }
+    const size_t b_bytes = (size_t)kMaxBN * kBK * 2;
+    auto total = [&](int nb, int na) {
+        return 1024 + (size_t)nb * b_bytes + (size_t)na * P.a_stage_bytes + (size_t)(2 * nb + 2 * na + 5) * 8 + 16;
+    };
+    int nb = 4, na = (amode == kAModeFrames) ? 3 : 4;
+    while (total(nb, na) > (size_t)h->smem_optin) {
+        if (na > 2) --na;
+        else if (nb > 2) --nb;
+        else break;
+    }
+    P.nb = nb;
+    P.na = na;
+    return total(nb, na);
+}
+
+pe_status finish(cudaError_t e) { return e == cudaSuccess ? PE_OK : PE_ERR_CUDA; }
+
+// Validate one frames item and fill its descriptor.  Returns PE_OK or an error.
+pe_status make_item(const pe_handle *h, const void *frames, int T, int H, int W, const int32_t *g,
+                    int merge, int64_t row0, ItemDesc &d) {
+    if (!frames || !g) return PE_ERR_INVALID_ARG;
+    if (!aligned16(frames)) return PE_ERR_ALIGN;
+    if (T < 1 || H < 1 || W < 1 || g[0] < 1 || g[1] < 1 || g[2] < 1) return PE_ERR_SHAPE;
+    if ((int64_t)H != (int64_t)g[1] * h->p || (int64_t)W != (int64_t)g[2] * h->p) return PE_ERR_SHAPE;
+    if ((T + h->tp - 1) / h->tp != g[0]) return PE_ERR_SHAPE;
+    if (merge == 2 && ((g[1] & 1) || (g[2] & 1))) return PE_ERR_SHAPE;
+    if ((int64_t)T * h->C * H * W >= (int64_t)1 << 40) return PE_ERR_UNSUPPORTED;
+    if ((int64_t)h->C * H * W > INT32_MAX) return PE_ERR_UNSUPPORTED;
+    d.frames = frames;
+    d.row0 = row0;
+    d.T = T;
+    d.H = H;
+    d.W = W;
+    d.gt = g[0];
+    d.gh = g[1];
+    d.gw = g[2];
+    return PE_OK;
+}
+
+// Shared front half of the frames entry points: validation + item table.
+pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt, const int32_t *THW,
+                       const int32_t *grid, int merge, const void *out, FwdParams &P, cudaStream_t st) {
+    if (!h || n < 1 || !frames || !THW || !grid || !out) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(f_dt)) return PE_ERR_DTYPE;
+    if (merge != 1 && merge != 2) return PE_ERR_INVALID_ARG;
+    if ((h->p & 1) || h->p > PE_MAX_PATCH) return PE_ERR_UNSUPPORTED;
+    if (!aligned16(out)) return PE_ERR_ALIGN;
+    fill_common(h, P);
+    P.merge = merge;
+    P.n_items = n;
+    std::vector<ItemDesc> items((size_t)n);
+    int64_t row0 = 0;
+    for (int i = 0; i < n; ++i) {
+        const pe_status s = make_item(h, frames[i], THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid + 3 * i,
+                                      merge, row0, items[(size_t)i]);
+        if (s != PE_OK) return s;
+        row0 += (int64_t)grid[3 * i] * grid[3 * i + 1] * grid[3 * i + 2];
+    }
+    P.N = row0;
+    if (n <= PE_INLINE_ITEMS) {
+        for (int i = 0; i < n; ++i) P.items[i] = items[(size_t)i];
+        P.items_dev = nullptr;
+        return PE_OK;
+    }
+    // Upload the table into the handle's workspace (pinned staging, stream order).
+    if (h->items_evt_pending) {
+        if (cudaEventSynchronize(h->items_evt) != cudaSuccess) return PE_ERR_CUDA;
+        h->items_evt_pending = false;
+    }
+    if (n > h->items_cap) {
+        if (h->items_dev) cudaFree(h->items_dev);
+        if (h->items_pinned) cudaFreeHost(h->items_pinned);
+        h->items_dev = nullptr;
+        h->items_pinned = nullptr;
+        h->items_cap = 0;
+        const int cap = std::max(n, 64);
+        if (cudaMalloc(&h->items_dev, sizeof(ItemDesc) * cap) != cudaSuccess) return PE_ERR_CUDA;
+        if (cudaMallocHost(&h->items_pinned, sizeof(ItemDesc) * cap) != cudaSuccess) return PE_ERR_CUDA;
+        h->items_cap = cap;
+    }
+    std::memcpy(h->items_pinned, items.data(), sizeof(ItemDesc) * (size_t)n);
+    if (cudaMemcpyAsync(h->items_dev, h->items_pinned, sizeof(ItemDesc) * (size_t)n, cudaMemcpyHostToDevice,
+                        st) != cudaSuccess)
+        return PE_ERR_CUDA;
+    if (cudaEventRecord(h->items_evt, st) != cudaSuccess) return PE_ERR_CUDA;
+    h->items_evt_pending = true;
+    P.items_dev = h->items_dev;
+    return PE_OK;
+}
+
+pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st) {
+    P.out = out;
+    P.out_f32 = out_dt == PE_F32;
+    if (P.N == 0) return PE_OK;
+    P.bn = choose_bn(P.N, P.E, h->num_sms, true);
+    P.n_tiles_n = (P.E + P.bn - 1) / P.bn;
+    const int64_t mt = (P.N + kBM - 1) / kBM;
+    if (mt * P.n_tiles_n > INT32_MAX) return PE_ERR_UNSUPPORTED;
+    P.num_tiles = (int)(mt * P.n_tiles_n);
+    const size_t smem = plan_pipeline(h, P, kAModeFrames);
+    const int grid = std::min(P.num_tiles, h->num_sms);
+    CUtensorMap dummy;
+    std::memset(&dummy, 0, sizeof(dummy));
+    const bool f32 = f_dt == PE_F32;
+    cudaError_t e;
+    if (h->p == 14)
+        e = f32 ? launch_fwd<kAModeFrames, 14, true>(h, P, dummy, smem, grid, st)
+                : launch_fwd<kAModeFrames, 14, false>(h, P, dummy, smem, grid, st);
+    else if (h->p == 16)
+        e = f32 ? launch_fwd<kAModeFrames, 16, true>(h, P, dummy, smem, grid, st)
+                : launch_fwd<kAModeFrames, 16, false>(h, P, dummy, smem, grid, st);
+    else
+        e = f32 ? launch_fwd<kAModeFrames, 0, true>(h, P, dummy, smem, grid, st)
+                : launch_fwd<kAModeFrames, 0, false>(h, P, dummy, smem, grid, st);
+    return finish(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pe_status_string(pe_status s) {
+    switch (s) {
+        case PE_OK: return "ok";
+        case PE_ERR_INVALID_ARG: return "invalid argument";
+        case PE_ERR_SHAPE: return "inconsistent shape";
+        case PE_ERR_DTYPE: return "unsupported dtype";
+        case PE_ERR_ALIGN: return "device pointer not 16-byte aligned";
+        case PE_ERR_NO_WEIGHT: return "weight not set";
+        case PE_ERR_CUDA: return "CUDA error";
+        case PE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PE_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    }
+    return "unknown status";
+}
+
+int64_t pe_num_patches(const int32_t *grid_thw, int n) {
+    if (n == 0) return 0;
+    if (!grid_thw || n < 0) return -1;
+    int64_t s = 0;
+    for (int i = 0; i < n; ++i) {
+        const int32_t *g = grid_thw + 3 * i;
+        if (g[0] < 1 || g[1] < 1 || g[2] < 1) return -1;
+        s += (int64_t)g[0] * g[1] * g[2];
+    }
+    return s;
+}
+
+int pe_device(const pe_handle *h) { return h ? h->dev : -1; }
+
+pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) {
+    if (!out) return PE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (E < 16 || E > 65535 || (E % 8) != 0 || C < 1 || C > 4 || tp < 1 || tp > 4 || p < 1)
+        return PE_ERR_INVALID_ARG;
+    const int64_t K = (int64_t)C * tp * p * p;
+    if (K > 8192) return PE_ERR_UNSUPPORTED;
+    pe_handle *h = new (std::nothrow) pe_handle();
+    if (!h) return PE_ERR_CUDA;
+    if (cudaGetDevice(&h->dev) != cudaSuccess) { delete h; return PE_ERR_CUDA; }
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, h->dev);
+    if (major != 10 || minor != 0) { delete h; return PE_ERR_UNSUPPORTED; }
+    cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->dev);
+    cudaDeviceGetAttribute(&h->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev);
+    h->E = E;
+    h->C = C;
+    h->tp = tp;
+    h->p = p;
+    h->K = (int)K;
+    h->Kpad = (int)((K + 63) / 64 * 64);
+    h->has_bias = has_bias != 0;
+    bool ok = cudaMalloc(&h->wpack, sizeof(uint16_t) * (size_t)E * h->Kpad) == cudaSuccess &&
+              cudaMalloc(&h->err, sizeof(int)) == cudaSuccess &&
+              cudaMemset(h->err, 0, sizeof(int)) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->items_evt, cudaEventDisableTiming) == cudaSuccess;
+    if (ok && h->has_bias) ok = cudaMalloc(&h->bias, sizeof(float) * E) == cudaSuccess;
+    if (ok) {
+        const uint32_t boxes[3] = {64, 128, 256};
+        for (int i = 0; i < 3 && ok; ++i)
+            ok = make_tmap_bf16(&h->tmap_w[i], h->wpack, (uint64_t)E, (uint64_t)h->Kpad, (uint64_t)h->Kpad,
+                                boxes[i]);
+    }
+    if (!ok) { pe_destroy(h); return PE_ERR_CUDA; }
+    *out = h;
+    return PE_OK;
+}
+
+void pe_destroy(pe_handle *h) {
+    if (!h) return;
+    DeviceGuard g(h->dev);
+    cudaDeviceSynchronize();
+    if (h->wpack) cudaFree(h->wpack);
+    if (h->bias) cudaFree(h->bias);
+    if (h->err) cudaFree(h->err);
+    if (h->items_dev) cudaFree(h->items_dev);
+    if (h->items_pinned) cudaFreeHost(h->items_pinned);
+    if (h->items_evt) cudaEventDestroy(h->items_evt);
+    delete h;
+}
+
+pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *bias, pe_dtype b_dt,
+                        pe_stream_t stream) {
+    if (!h || !w) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(w_dt) || (bias && !valid_dtype(b_dt))) return PE_ERR_DTYPE;
+    if ((bias != nullptr) != h->has_bias) return PE_ERR_INVALID_ARG;
+    if (!aligned16(w) || (bias && !aligned16(bias))) return PE_ERR_ALIGN;
+    DeviceGuard g(h->dev);
+    const int64_t total = (int64_t)h->E * h->Kpad;
+    const int threads = 256;
+    const int blocks = (int)std::min<int64_t>((total + threads - 1) / threads, (int64_t)h->num_sms * 8);
+    pe_pack_weight_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
+        w, w_dt == PE_F32, bias, b_dt == PE_F32, h->wpack, h->bias, h->E, h->K, h->Kpad);
+    if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    h->weight_set = true;
+    return PE_OK;
+}
+
+pe_status pe_set_norm(pe_handle *h, const float *mean, const float *std) {
+    if (!h || !mean || !std) return PE_ERR_INVALID_ARG;
+    for (int c = 0; c < h->C; ++c) {
+        if (!(std[c] > 0.f) || !(std[c] < 3.0e38f) || !(mean[c] == mean[c]) ||
+            !(mean[c] < 3.0e38f && mean[c] > -3.0e38f))
+            return PE_ERR_INVALID_ARG;
+    }
+    for (int c = 0; c < h->C; ++c) {
+        h->mean[c] = mean[c];
+        h->stdv[c] = std[c];
+    }
+    return PE_OK;
+}
+
+pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, void *out,
+                             pe_dtype out_dt, pe_stream_t stream) {
+    if (!h || N < 0) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(x_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
+    if (!h->weight_set) return PE_ERR_NO_WEIGHT;
+    if (N == 0) return PE_OK;
+    if (!x || !out) return PE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return PE_ERR_ALIGN;
+    DeviceGuard g(h->dev);
+    FwdParams P;
+    fill_common(h, P);
+    P.N = N;
+    P.x = x;
+    P.x_f32 = x_dt == PE_F32;
+    P.out = out;
+    P.out_f32 = out_dt == PE_F32;
+    P.merge = 1;
+    const bool tma = (x_dt == PE_BF16) && (h->K % 8 == 0);
+    P.x_vec = (x_dt == PE_BF16) ? (h->K % 8 == 0) : (h->K % 4 == 0);
+    P.bn = choose_bn(N, h->E, h->num_sms, false);
+    P.n_tiles_n = (h->E + P.bn - 1) / P.bn;
+    const int64_t mt = (N + kBM - 1) / kBM;
+    if (mt * P.n_tiles_n > INT32_MAX) return PE_ERR_UNSUPPORTED;
+    P.num_tiles = (int)(mt * P.n_tiles_n);
+    const size_t smem = plan_pipeline(h, P, tma ? kAModeTma : kAModePatchThreads);
+    const int grid = std::min(P.num_tiles, h->num_sms);
+    cudaStream_t st = (cudaStream_t)stream;
+    CUtensorMap tx;
+    std::memset(&tx, 0, sizeof(tx));
+    if (tma) {
+        if (!make_tmap_bf16(&tx, x, (uint64_t)N, (uint64_t)h->K, (uint64_t)h->K, kBM)) return PE_ERR_CUDA;
+        return finish(launch_fwd<kAModeTma, 0, false>(h, P, tx, smem, grid, st));
+    }
+    return finish(launch_fwd<kAModePatchThreads, 0, false>(h, P, tx, smem, grid, st));
+}
+
+pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                    const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
+                                    pe_dtype out_dt, pe_stream_t stream) {
+    if (!h) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(out_dt)) return PE_ERR_DTYPE;
+    if (!h->weight_set) return PE_ERR_NO_WEIGHT;
+    DeviceGuard g(h->dev);
+    FwdParams P;
+    const pe_status s = setup_frames(h, n, frames, f_dt, THW, grid_thw, merge, out, P, (cudaStream_t)stream);
+    if (s != PE_OK) return s;
+    return run_frames(h, P, f_dt, out, out_dt, (cudaStream_t)stream);
+}
+
+pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H, int W,
+                            const int32_t grid_thw[3], int merge, void *out, pe_dtype out_dt,
+                            pe_stream_t stream) {
+    const int32_t thw[3] = {T, H, W};
+    const void *fr[1] = {frames};
+    return pe_forward_frames_grouped(h, 1, fr, f_dt, thw, grid_thw, merge, out, out_dt, stream);
+}
+
+pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt, const int32_t *THW,
+                      const int32_t *grid_thw, int merge, void *rows, pe_dtype rows_dt, pe_stream_t stream) {
+    if (!h) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(rows_dt)) return PE_ERR_DTYPE;
+    DeviceGuard g(h->dev);
+    FwdParams P;
+    cudaStream_t st = (cudaStream_t)stream;
+    const pe_status s = setup_frames(h, n, frames, f_dt, THW, grid_thw, merge, rows, P, st);
+    if (s != PE_OK) return s;
+    if (P.N == 0) return PE_OK;
+    const int64_t total = P.N * (h->K / 2);
+    const int threads = 256;
+    const int blocks = (int)std::min<int64_t>((total + threads - 1) / threads, (int64_t)h->num_sms * 16);
+    if (f_dt == PE_F32)
+        pe_patchify_kernel<true><<<blocks, threads, 0, st>>>(P, rows, rows_dt == PE_F32);
+    else
+        pe_patchify_kernel<false><<<blocks, threads, 0, st>>>(P, rows, rows_dt == PE_F32);
+    return finish(cudaGetLastError());
+}
+
+pe_status pe_last_error(pe_handle *h) {
+    if (!h) return PE_ERR_INVALID_ARG;
+    DeviceGuard g(h->dev);
+    int v = 0;
+    if (cudaMemcpy(&v, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PE_ERR_CUDA;
+    if (v != 0 && cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return PE_ERR_CUDA;
+    return v == 0 ? PE_OK : (pe_status)v;
+}
+
+}  // extern "C"

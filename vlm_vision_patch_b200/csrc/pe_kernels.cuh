@@ -1,0 +1,609 @@
+// sm_100a kernels of the vision PatchEmbed.
+//
+// The PatchEmbed is a Conv3d whose kernel equals its stride, i.e. one dense
+// contraction out[N, E] = A[N, K] * W[E, K]^T (+ bias) with K = C*tp*p*p
+// (Qwen2.5VL-Vision Encode-PatchEmbed: "the conv is a dot product of the
+// flattened input and weight"; mytransformer README §4.1: F.linear(x,
+// w.reshape(1280, 1176))).  One persistent kernel runs the whole path:
+//
+//   warp 0      TMA producer: weight tiles (and A tiles of bf16 patch rows)
+//   warp 1      MMA issuer (one thread) + TMEM owner
+//   warps 4-7   epilogue: TMEM -> registers, + bias, cast, 16-byte stores
+//   warps 8-15  A producers for the thread-fed modes: fp32/unaligned patch rows
+//               (converted to bf16), or the fused frames gather that builds
+//               each patch row from raw [T, C, H, W] frames, normalises it and
+//               places it in merge order, straight into shared memory.
+//
+// Tiles are 128 rows x BN (64/128/256) columns; the fp32 accumulator lives in
+// tensor memory, double buffered (2 x 256 columns) so the epilogue of tile i
+// overlaps the MMAs of tile i+1.  Every pipeline wait is bounded.
+#pragma once
+
+#include "pe_device.cuh"
+#include "../../include/pe.h"
+
+namespace pe {
+
+constexpr int kThreads = 512;
+constexpr int kBM = 128;           // rows per tile (MMA M)
+constexpr int kMaxBN = 256;        // largest MMA N
+constexpr int kBK = 64;            // weight K per TMA stage (one 128-byte swizzle row)
+constexpr int kProdThreads = 256;  // warps 8..15
+constexpr int kProdWarps = 8;
+constexpr int kEpiWarp0 = 4;
+
+enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2 };
+
+struct ItemDesc {
+    const void *frames;  // [T, C, H, W]
+    int64_t row0;        // first output row of the item
+    int32_t T, H, W;
+    int32_t gt, gh, gw;
+};
+
+struct FwdParams {
+    int32_t E, C, TP, P, K, Kpad;
+    int32_t bn, n_tiles_n, num_tiles, num_ksteps;
+    int32_t n_b_stages, n_a_stages;   // per tile
+    int32_t nb, na;                   // ring depths
+    int32_t a_stage_bytes;
+    int32_t merge, n_items;
+    int64_t N;
+    const ItemDesc *items_dev;        // table in device memory when n_items > PE_INLINE_ITEMS
+    ItemDesc items[PE_INLINE_ITEMS];
+    float mean[4], stdv[4], nstdv[4], rstd[4];
+    const void *x;                    // patches input
+    int32_t x_f32;                    // patches dtype is fp32
+    int32_t x_vec;                    // patch rows allow 16-byte vector loads
+    void *out;
+    int32_t out_f32;
+    const float *bias;                // fp32 [E] or nullptr
+    int *err;                         // device error word
+};
+
+// ------------------------------------------------------------ row decoding
+
+__device__ __forceinline__ const ItemDesc &item_at(const FwdParams &P, int i) {
+    return P.n_items <= PE_INLINE_ITEMS ? P.items[i] : P.items_dev[i];
+}
+
+// Output row R -> the patch it embeds.  Items are concatenated in list order;
+// inside an item rows follow the spatial-merge order for merge = 2 (2x2 windows
+// consecutive, windows row-major over (t, h/2, w/2), (dh, dw) row-major inside)
+// or raster order (t, h, w) for merge = 1.
+struct RowSrc {
+    const char *base;   // byte address of pixel (frame tau0, c = 0, y = g_h*p, x = g_w*p)
+    int32_t W;          // elements per image row
+    int32_t HW;         // elements per channel plane
+    int32_t CHW;        // elements per frame
+    int32_t tmax;       // last usable temporal offset: min(t, tmax) frames past tau0
+};
+
+__device__ __forceinline__ RowSrc locate_row(const FwdParams &P, int64_t R, int esize) {
+    int lo = 0, hi = P.n_items - 1;
+    while (lo < hi) {  // last item with row0 <= R
+        const int mid = (lo + hi + 1) >> 1;
+        if (item_at(P, mid).row0 <= R) lo = mid; else hi = mid - 1;
+    }
+    const ItemDesc &it = item_at(P, lo);
+    const int64_t rho = R - it.row0;
+    int64_t g_t, g_h, g_w;
+    if (P.merge == 2) {
+        const int64_t win = rho >> 2;
+        const int d = (int)(rho & 3);
+        const int64_t wpr = it.gw >> 1, wpt = (int64_t)(it.gh >> 1) * wpr;
+        g_t = win / wpt;
+        const int64_t rem = win - g_t * wpt;
+        const int64_t wy = rem / wpr;
+        g_h = 2 * wy + (d >> 1);
+        g_w = 2 * (rem - wy * wpr) + (d & 1);
+    } else {
+        g_w = rho % it.gw;
+        const int64_t tmp = rho / it.gw;
+        g_h = tmp % it.gh;
+        g_t = tmp / it.gh;
+    }
+    int64_t tau0 = g_t * P.TP;
+    if (tau0 > it.T - 1) tau0 = it.T - 1;
+    RowSrc s;
+    s.W = it.W;
+    s.HW = it.H * it.W;
+    s.CHW = P.C * s.HW;
+    s.tmax = (int32_t)(it.T - 1 - tau0);
+    const int64_t el = (tau0 * P.C * it.H + g_h * P.P) * (int64_t)it.W + g_w * P.P;
+    s.base = reinterpret_cast<const char *>(it.frames) + el * esize;
+    return s;
+}
+
+// (x - mean) / std in fp32 with IEEE rounding of the subtract and of the
+// quotient, for two pixels at once; returns the two results rounded to bf16.
+// The quotient is computed as q0 = d * rcp(std), then one fused
+// multiply-add correction q = q0 + (d - q0 * std) * rcp(std), Markstein's
+// final step for a correctly rounded quotient (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. R&D 1990),
+// given rcp(std) correctly rounded.  Verified bit-exact against IEEE division on
+// every bf16 input by the patchify tests.
+__device__ __forceinline__ uint32_t norm_pair(float x0, float x1, float mean, float stdv,
+                                              float nstdv, float rstd) {
+    uint64_t X, M, D, R, NS, Q0, Er, Q;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(x0), "f"(x1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(M) : "f"(mean));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(R) : "f"(rstd));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(NS) : "f"(nstdv));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(X), "l"(M));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q0) : "l"(D), "l"(R));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Er) : "l"(Q0), "l"(NS), "l"(D));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Q) : "l"(Er), "l"(R), "l"(Q0));
+    float q0, q1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(q0), "=f"(q1) : "l"(Q));
+    (void)stdv;
+    return pack_bf16x2(q0, q1);
+}
+
+// One 2-pixel word of a frame row, as two fp32.
+template <bool F32IN>
+__device__ __forceinline__ void load_pair(const char *p, float &a, float &b) {
+    if constexpr (F32IN) {
+        float2 v;
+        asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+        a = v.x;
+        b = v.y;
+    } else {
+        uint32_t w;
+        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w) : "l"(p));
+        a = bf16lo_to_f32(w);
+        b = bf16hi_to_f32(w);
+    }
+}
+
+// Item u of a segment (one 2-pixel word of one tile row) -> (tile row, word).
+// For merge = 2 the order walks patch-row halves of the windows so that
+// consecutive u read consecutive words of one image row.
+__device__ __forceinline__ void unit_to_row_word(int u, int ws, int merge, int &r, int &jw) {
+    jw = u % ws;
+    const int t1 = u / ws;
+    if (merge == 2) {
+        const int dw = t1 & 1, t2 = t1 >> 1;
+        const int q = t2 & 31, dh = t2 >> 5;
+        r = 4 * q + 2 * dh + dw;
+    } else {
+        r = t1;
+    }
+}
+
+// ------------------------------------------------------------- producers
+
+// Frames producer: every A stage holds 8 whole segments (c, t, i) of p pixels,
+// i.e. 8p consecutive k of the view(-1, C, tp, p, p) order, in the no-swizzle
+// K-major layout: element (r, k) at (k / 8) * 2048 + r * 16 + (k % 8) * 2.
+template <int PT, bool F32IN>
+__device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ring,
+                                               uint64_t *full_a, uint64_t *empty_a,
+                                               volatile int *abort, int pt, int lane) {
+    const int p = PT ? PT : P.P;
+    const int ws = p >> 1;
+    const int units = kBM * ws;
+    constexpr int MAXIT = PT ? (PT + 3) / 4 : (PE_MAX_PATCH + 3) / 4;
+    constexpr int esize = F32IN ? 4 : 2;
+    const int nseg = P.C * P.TP * p;
+
+    int rr[MAXIT], kw[MAXIT];
+    bool uok[MAXIT];
+#pragma unroll
+    for (int v = 0; v < MAXIT; ++v) {
+        const int u = pt + kProdThreads * v;
+        uok[v] = u < units;
+        int r = 0, jw = 0;
+        if (uok[v]) unit_to_row_word(u, ws, P.merge, r, jw);
+        rr[v] = r;
+        kw[v] = 2 * jw;
+    }
+
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
+        const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * kBM;
+        const char *src[MAXIT];
+        int32_t sW[MAXIT], sHW[MAXIT], sCHW[MAXIT], sTm[MAXIT];
+        bool rok[MAXIT];
+#pragma unroll
+        for (int v = 0; v < MAXIT; ++v) {
+            rok[v] = uok[v] && (m0 + rr[v] < P.N);
+            if (rok[v]) {
+                const RowSrc s = locate_row(P, m0 + rr[v], esize);
+                src[v] = s.base + (int64_t)kw[v] * esize;
+                sW[v] = s.W;
+                sHW[v] = s.HW;
+                sCHW[v] = s.CHW;
+                sTm[v] = s.tmax;
+            } else {
+                src[v] = nullptr;
+                sW[v] = sHW[v] = sCHW[v] = sTm[v] = 0;
+            }
+        }
+        int c = 0, t = 0, i = 0;  // segment counters, seg = (c * TP + t) * p + i
+        for (int s = 0; s < P.n_a_stages; ++s) {
+            if (!mbar_wait(smem_addr(&empty_a[stage]), phase ^ 1, abort)) return;
+            uint8_t *As = a_ring + (size_t)stage * P.a_stage_bytes;
+            float va[8][MAXIT], vb[8][MAXIT];
+            int cq[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const bool live = (8 * s + q) < nseg;
+                cq[q] = live ? c : -1;
+#pragma unroll
+                for (int v = 0; v < MAXIT; ++v) {
+                    va[q][v] = 0.f;
+                    vb[q][v] = 0.f;
+                    if (live && rok[v]) {
+                        const int tt = t < sTm[v] ? t : sTm[v];
+                        const int64_t off = (int64_t)tt * sCHW[v] + c * sHW[v] + i * sW[v];
+                        load_pair<F32IN>(src[v] + off * esize, va[q][v], vb[q][v]);
+                    }
+                }
+                if (++i == p) {
+                    i = 0;
+                    if (++t == P.TP) { t = 0; ++c; }
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int ch = cq[q];
+                float mu = 0.f, sd = 1.f, nsd = -1.f, rs = 1.f;
+                if (ch >= 0) { mu = P.mean[ch]; sd = P.stdv[ch]; nsd = P.nstdv[ch]; rs = P.rstd[ch]; }
+#pragma unroll
+                for (int v = 0; v < MAXIT; ++v) {
+                    if (!rok[v]) continue;
+                    const uint32_t w = ch >= 0 ? norm_pair(va[q][v], vb[q][v], mu, sd, nsd, rs) : 0u;
+                    const int k = q * p + kw[v];
+                    const uint32_t off = (uint32_t)(k >> 3) * 2048u + (uint32_t)rr[v] * 16u +
+                                         (uint32_t)(k & 7) * 2u;
+                    *reinterpret_cast<uint32_t *>(As + off) = w;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&full_a[stage]));
+            if (++stage == P.na) { stage = 0; phase ^= 1; }
+        }
+    }
+}
+
+// Patch-row producer for rows the TMA cannot fetch directly (fp32 rows, or bf16
+// rows whose stride is not a multiple of 16 bytes): 64 k per stage, converted
+// to bf16 (RNE) into the no-swizzle K-major layout.
+__device__ __forceinline__ void produce_patches(const FwdParams &P, uint8_t *a_ring,
+                                                uint64_t *full_a, uint64_t *empty_a,
+                                                volatile int *abort, int pt, int lane) {
+    const int K = P.K;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
+        const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * kBM;
+        for (int s = 0; s < P.n_a_stages; ++s) {
+            if (!mbar_wait(smem_addr(&empty_a[stage]), phase ^ 1, abort)) return;
+            uint8_t *As = a_ring + (size_t)stage * P.a_stage_bytes;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int u = pt + kProdThreads * v;  // 0..1023
+                const int r = u >> 3, kg = u & 7;
+                const int64_t R = m0 + r;
+                const int k0 = s * kBK + kg * 8;
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+                if (R < P.N) {
+                    if (P.x_f32) {
+                        const float *row = reinterpret_cast<const float *>(P.x) + R * K;
+                        float f[8];
+                        if (P.x_vec && k0 + 8 <= K) {
+                            const float4 a = __ldg(reinterpret_cast<const float4 *>(row + k0));
+                            const float4 b = __ldg(reinterpret_cast<const float4 *>(row + k0 + 4));
+                            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+                            f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] = (k0 + e < K) ? __ldg(row + k0 + e) : 0.f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+                    } else {
+                        const uint16_t *row = reinterpret_cast<const uint16_t *>(P.x) + R * K;
+                        if (P.x_vec && k0 + 8 <= K) {
+                            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(row + k0));
+                            w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+                        } else {
+                            uint16_t h[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) h[e] = (k0 + e < K) ? __ldg(row + k0 + e) : (uint16_t)0;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) w[e] = (uint32_t)h[2 * e] | ((uint32_t)h[2 * e + 1] << 16);
+                        }
+                    }
+                }
+                *reinterpret_cast<uint4 *>(As + kg * 2048 + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&full_a[stage]));
+            if (++stage == P.na) { stage = 0; phase ^= 1; }
+        }
+    }
+}
+
+// ------------------------------------------------------------- the kernel
+
+template <int AMODE, int PT, bool F32IN>
+__global__ void __launch_bounds__(kThreads, 1)
+    pe_fwd_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                  const __grid_constant__ FwdParams P) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int b_stage_bytes = kMaxBN * kBK * 2;
+    uint8_t *b_ring = smem;
+    uint8_t *a_ring = b_ring + (size_t)P.nb * b_stage_bytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(a_ring + (size_t)P.na * P.a_stage_bytes);
+    uint64_t *full_b = bars;
+    uint64_t *empty_b = full_b + P.nb;
+    uint64_t *full_a = empty_b + P.nb;
+    uint64_t *empty_a = full_a + P.na;
+    uint64_t *tfull = empty_a + P.na;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *mma_done = tempty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P.nb; ++s) {
+            mbar_init(smem_addr(&full_b[s]), 1);
+            mbar_init(smem_addr(&empty_b[s]), 1);
+        }
+        for (int s = 0; s < P.na; ++s) {
+            mbar_init(smem_addr(&full_a[s]), AMODE == kAModeTma ? 1 : kProdWarps);
+            mbar_init(smem_addr(&empty_a[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&tfull[s]), 1);
+            mbar_init(smem_addr(&tempty[s]), 4);
+        }
+        mbar_init(smem_addr(mma_done), 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_w);
+        if (AMODE == kAModeTma) prefetch_tmap(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_last();
+            const uint64_t pol_x = l2_policy_evict_first();
+            const uint32_t b_bytes = (uint32_t)P.bn * kBK * 2;
+            int bs = 0, as = 0;
+            uint32_t bph = 0, aph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < P.num_tiles && ok; tile += gridDim.x) {
+                const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
+                for (int kb = 0; kb < P.n_b_stages && ok; ++kb) {
+                    if (AMODE == kAModeTma) {
+                        if (!mbar_wait(smem_addr(&empty_a[as]), aph ^ 1, abort)) { ok = false; break; }
+                        mbar_arrive_expect_tx(smem_addr(&full_a[as]), kBM * kBK * 2);
+                        tma_load_2d(smem_addr(a_ring + (size_t)as * P.a_stage_bytes), &tmap_x,
+                                    smem_addr(&full_a[as]), kb * kBK, m_blk * kBM, pol_x);
+                        if (++as == P.na) { as = 0; aph ^= 1; }
+                    }
+                    if (!mbar_wait(smem_addr(&empty_b[bs]), bph ^ 1, abort)) { ok = false; break; }
+                    mbar_arrive_expect_tx(smem_addr(&full_b[bs]), b_bytes);
+                    tma_load_2d(smem_addr(b_ring + (size_t)bs * b_stage_bytes), &tmap_w,
+                                smem_addr(&full_b[bs]), kb * kBK, n_blk * P.bn, pol_w);
+                    if (++bs == P.nb) { bs = 0; bph ^= 1; }
+                }
+            }
+            // Drain: let the last loads of every ring slot land before exiting.
+            for (int s = 0; s < P.nb; ++s) {
+                const int slot = (bs + s) % P.nb;  // oldest first
+                const uint32_t par = (slot < bs) ? bph : (bph ^ 1);
+                mbar_wait(smem_addr(&full_b[slot]), par, abort);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(kBM, P.bn);
+            const int ks_a = (AMODE == kAModeFrames) ? (P.P >> 1) : (kBK / 16);
+            int bs = 0, as = 0, acc = 0;
+            uint32_t bph = 0, aph = 0, accph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < P.num_tiles && ok; tile += gridDim.x) {
+                if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)acc * kMaxBN;
+                int ka = 0, kbi = 0;  // k-step inside the current A / B stage
+                for (int ks = 0; ks < P.num_ksteps; ++ks) {
+                    if (kbi == 0) {
+                        if (!mbar_wait(smem_addr(&full_b[bs]), bph, abort)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    if (ka == 0) {
+                        if (!mbar_wait(smem_addr(&full_a[as]), aph, abort)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    const uint32_t a_base = smem_addr(a_ring + (size_t)as * P.a_stage_bytes);
+                    const uint32_t b_base = smem_addr(b_ring + (size_t)bs * b_stage_bytes);
+                    uint64_t adesc;
+                    if (AMODE == kAModeTma)
+                        adesc = smem_desc(a_base + ka * 32, 16, 1024, kLayoutSw128);
+                    else
+                        adesc = smem_desc(a_base + ka * 4096, 2048, 128, kLayoutInterleave);
+                    const uint64_t bdesc = smem_desc(b_base + kbi * 32, 16, 1024, kLayoutSw128);
+                    mma_bf16(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+                    const bool last = (ks == P.num_ksteps - 1);
+                    if (++kbi == kBK / 16 || last) {
+                        mma_commit(smem_addr(&empty_b[bs]));
+                        kbi = 0;
+                        if (++bs == P.nb) { bs = 0; bph ^= 1; }
+                    }
+                    if (++ka == ks_a || last) {
+                        mma_commit(smem_addr(&empty_a[as]));
+                        ka = 0;
+                        if (++as == P.na) { as = 0; aph ^= 1; }
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_addr(&tfull[acc]));
+                if (++acc == 2) { acc = 0; accph ^= 1; }
+            }
+            mma_commit(smem_addr(mma_done));
+            mbar_wait(smem_addr(mma_done), 0, abort);
+        }
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        // ---------------- epilogue
+        const int wq = warp & 3;  // TMEM lane quarter this warp may access
+        int acc = 0;
+        uint32_t accph = 0;
+        for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
+            const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
+            if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)m_blk * kBM + wq * 32 + lane;
+            const bool row_ok = row < P.N;
+            for (int cc = 0; cc < P.bn / 32; ++cc) {
+                uint32_t v[32];
+                const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN + cc * 32);
+                tmem_ld_32x32b_x32(taddr, v);
+                tmem_ld_wait();
+                const int col0 = n_blk * P.bn + cc * 32;
+                if (!row_ok || col0 >= P.E) continue;
+                float f[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+                if (P.bias) {
+                    if (col0 + 32 <= P.E) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 b = __ldg(reinterpret_cast<const float4 *>(P.bias + col0 + e));
+                            f[e] += b.x; f[e + 1] += b.y; f[e + 2] += b.z; f[e + 3] += b.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
+                    }
+                }
+                if (P.out_f32) {
+                    float *o = reinterpret_cast<float *>(P.out) + row * P.E + col0;
+                    if (col0 + 32 <= P.E) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4 *>(o + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (col0 + e < P.E) o[e] = f[e];
+                    }
+                } else {
+                    uint32_t h[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) h[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+                    uint16_t *o = reinterpret_cast<uint16_t *>(P.out) + row * P.E + col0;
+                    if (col0 + 32 <= P.E) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<uint4 *>(o + 2 * e) = make_uint4(h[e], h[e + 1], h[e + 2], h[e + 3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (col0 + 2 * e < P.E) *reinterpret_cast<uint32_t *>(o + 2 * e) = h[e];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tempty[acc]));
+            if (++acc == 2) { acc = 0; accph ^= 1; }
+        }
+    } else if (warp >= 8) {
+        // ---------------- A producers
+        if constexpr (AMODE == kAModeFrames)
+            produce_frames<PT, F32IN>(P, a_ring, full_a, empty_a, abort, threadIdx.x - 256, lane);
+        else if constexpr (AMODE == kAModePatchThreads)
+            produce_patches(P, a_ring, full_a, empty_a, abort, threadIdx.x - 256, lane);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+    if (threadIdx.x == 0 && *abort) atomicExch(P.err, (int)PE_ERR_DEVICE_TIMEOUT);
+}
+
+// ------------------------------------------------------------- helpers
+
+// Ŵ[e, k] = bf16_rne(W[e, k]) for k < K, 0 for K <= k < Kpad; bias widened to fp32.
+__global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias, int b_f32,
+                                      uint16_t *wpack, float *bias32, int E, int K, int Kpad) {
+    const int64_t total = (int64_t)E * Kpad;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = idx / Kpad;
+        const int k = (int)(idx - e * Kpad);
+        uint16_t v = 0;
+        if (k < K) {
+            if (w_f32) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(reinterpret_cast<const float *>(w)[e * K + k]);
+                v = *reinterpret_cast<const uint16_t *>(&b);
+            } else {
+                v = reinterpret_cast<const uint16_t *>(w)[e * K + k];
+            }
+        }
+        wpack[idx] = v;
+        if (k == 0 && bias && bias32)
+            bias32[e] = b_f32 ? reinterpret_cast<const float *>(bias)[e]
+                              : __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(bias)[e] << 16);
+    }
+}
+
+// rows[R, k] for every output row R: the frames producer's gather and
+// normalisation written to memory (bf16 or fp32 values; bf16-exact either way).
+template <bool F32IN>
+__global__ void pe_patchify_kernel(const __grid_constant__ FwdParams P, void *rows, int rows_f32) {
+    constexpr int esize = F32IN ? 4 : 2;
+    const int p = P.P, ws = p >> 1;
+    const int words = P.K >> 1;
+    const int64_t total = P.N * words;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t R = idx / words;
+        const int wk = (int)(idx - R * words);
+        const int seg = wk / ws, jw = wk - seg * ws;
+        const int i = seg % p, t = (seg / p) % P.TP, c = seg / (p * P.TP);
+        const RowSrc s = locate_row(P, R, esize);
+        const int tt = t < s.tmax ? t : s.tmax;
+        const int64_t off = (int64_t)tt * s.CHW + (int64_t)c * s.HW + (int64_t)i * s.W + 2 * jw;
+        float a, b;
+        load_pair<F32IN>(s.base + off * esize, a, b);
+        const uint32_t w = norm_pair(a, b, P.mean[c], P.stdv[c], P.nstdv[c], P.rstd[c]);
+        const int64_t k = 2 * (int64_t)wk;
+        if (rows_f32) {
+            float *o = reinterpret_cast<float *>(rows) + R * P.K + k;
+            o[0] = bf16lo_to_f32(w);
+            o[1] = bf16hi_to_f32(w);
+        } else {
+            *reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(rows) + R * P.K + k) = w;
+        }
+    }
+}
+
+}  // namespace pe
