@@ -103,7 +103,8 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
 /*
  * pe_set_norm -- per-channel pixel normalisation used by the frames calls:
  * x_hat = bf16_rne( fp32( fp32(x - mean[c]) / std[c] ) ), IEEE fp32 subtract
- * and divide.  mean, std: host [C] fp32; std[c] must be finite and > 0.
+ * and divide, bit-exact for every finite pixel value x (non-finite pixels give
+ * NaN).  mean, std: host [C] fp32; mean[c] finite, std[c] finite and > 0.
  * Default after pe_create: mean 0, std 1 (x_hat = bf16_rne(x)).
  * Errors: PE_ERR_INVALID_ARG.
  */

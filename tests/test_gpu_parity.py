@@ -31,6 +31,15 @@ def _bits32(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").float().numpy().view(np.uint32)
 
 
+def assert_bits_equal(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    bad = got != ref
+    if bad.any():
+        idx = np.argwhere(bad)[:6]
+        det = [(tuple(int(x) for x in i), hex(int(got[tuple(i)])), hex(int(ref[tuple(i)]))) for i in idx]
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} differ; first (index, got, ref): {det}")
+
+
 # --------------------------------------------------------------- patches form
 
 @pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
@@ -66,7 +75,8 @@ def test_patches_one_hot_recovers_weight():
     out = pe.forward_patches(x, out_dtype=torch.float32)
     ref, _ = oracle.conv3d_patches(torch.eye(K), w, b, C, tp, p)
     torch.cuda.synchronize()
-    assert np.array_equal(out.cpu().double().numpy(), ref)
+    # one product, then the fp32 bias add: the exact sum rounded once to fp32
+    assert_bits_equal(out.cpu().numpy().view(np.uint32), ref.astype(np.float32).view(np.uint32), "one-hot")
     zero = pe.forward_patches(torch.zeros(5, K, dtype=torch.bfloat16, device=DEV), out_dtype=torch.float32)
     assert torch.equal(zero.cpu(), b.float().expand(5, E))
 
@@ -252,14 +262,16 @@ def test_patchify_bit_exact(T, gh, gw, merge, p, tp, fdt):
     rows = pe.patchify([frames.to(DEV)], [(gt, gh, gw)], merge, rows_dtype=torch.float32)
     ref = oracle.patchify(frames, (gt, gh, gw), merge, workloads.CLIP_MEAN, workloads.CLIP_STD, C, tp, p)
     torch.cuda.synchronize()
-    assert np.array_equal(_bits32(rows), ref.view(np.uint32))
+    assert_bits_equal(_bits32(rows), ref.view(np.uint32), "patchify fp32 rows")
     rows16 = pe.patchify([frames.to(DEV)], [(gt, gh, gw)], merge, rows_dtype=torch.bfloat16)
-    assert np.array_equal(_bits32(rows16), ref.view(np.uint32))
+    assert_bits_equal(_bits32(rows16), ref.view(np.uint32), "patchify bf16 rows")
 
 
 @pytest.mark.parametrize("mean,std", [(workloads.CLIP_MEAN, workloads.CLIP_STD),
                                       ((0.5, -0.25, 3.0), (0.5, 0.1, 7.0)),
-                                      ((0.0, 0.0, 0.0), (1.0, 1.0, 1.0))])
+                                      ((0.0, 0.0, 0.0), (1.0, 1.0, 1.0)),
+                                      ((0.0, -0.0, 1e-30), (0.3, 1.0, 5e-40)),
+                                      ((123.675, 116.28, 103.53), (58.395, 57.12, 57.375))])
 def test_normalization_exhaustive_bf16(mean, std):
     """Every finite bf16 value in every channel: the kernel's fp32 (x-mean)/std
     then bf16 rounding equals the oracle's IEEE divide bit for bit."""
@@ -278,7 +290,7 @@ def test_normalization_exhaustive_bf16(mean, std):
     rows = pe.patchify([frames.to(DEV)], [(1, H // 2, W // 2)], 2, rows_dtype=torch.float32)
     ref = oracle.patchify(frames, (1, H // 2, W // 2), 2, mean, std, 3, 1, 2)
     torch.cuda.synchronize()
-    assert np.array_equal(_bits32(rows), ref.view(np.uint32))
+    assert_bits_equal(_bits32(rows), ref.view(np.uint32), f"normalisation mean={mean} std={std}")
 
 
 # --------------------------------------------------------------- error paths

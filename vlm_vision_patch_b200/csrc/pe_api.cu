@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -135,10 +136,22 @@ void fill_common(const pe_handle *h, FwdParams &P) {
     P.K = h->K;
     P.Kpad = h->Kpad;
     for (int c = 0; c < 4; ++c) {
-        P.mean[c] = h->mean[c];
-        P.stdv[c] = h->stdv[c];
-        P.nstdv[c] = -h->stdv[c];
-        P.rstd[c] = 1.0f / h->stdv[c];  // IEEE division on the host: correctly rounded
+        const float mu = h->mean[c], sd = h->stdv[c];
+        uint32_t mu_bits;
+        std::memcpy(&mu_bits, &mu, 4);
+        P.mean[c] = mu;
+        P.stdv[c] = sd;
+        int e = 0;
+        const float s = 2.0f * std::frexp(sd, &e);   // sd = s * 2^(e-1), s in [1, 2)
+        P.nstd_s[c] = -s;
+        P.rcp_s[c] = 1.0f / s;                        // IEEE division on the host: correctly rounded
+        P.scale[c] = std::ldexp(1.0f, 1 - e);         // 1 / sd = (1 / s) * 2^(1-e)
+        if (mu_bits == 0u && sd == 1.0f)
+            P.norm_mode[c] = kNormIdentity;
+        else if (std::fabs(mu) >= 0x1p-70f && sd >= 0x1p-32f && sd <= 0x1p32f)
+            P.norm_mode[c] = kNormScaled;
+        else
+            P.norm_mode[c] = kNormDivide;
     }
     P.bias = h->has_bias ? h->bias : nullptr;
     P.err = h->err;

@@ -51,7 +51,9 @@ struct FwdParams {
     int64_t N;
     const ItemDesc *items_dev;        // table in device memory when n_items > PE_INLINE_ITEMS
     ItemDesc items[PE_INLINE_ITEMS];
-    float mean[4], stdv[4], nstdv[4], rstd[4];
+    float mean[4], stdv[4];          // per-channel normalisation (see NormMode)
+    float nstd_s[4], rcp_s[4], scale[4];
+    int32_t norm_mode[4];
     const void *x;                    // patches input
     int32_t x_f32;                    // patches dtype is fp32
     int32_t x_vec;                    // patch rows allow 16-byte vector loads
@@ -115,46 +117,88 @@ __device__ __forceinline__ RowSrc locate_row(const FwdParams &P, int64_t R, int 
     return s;
 }
 
-// (x - mean) / std in fp32 with IEEE rounding of the subtract and of the
-// quotient, for two pixels at once; returns the two results rounded to bf16.
-// The quotient is computed as q0 = d * rcp(std), then one fused
-// multiply-add correction q = q0 + (d - q0 * std) * rcp(std), Markstein's
-// final step for a correctly rounded quotient (P. Markstein, "Computation of
-// elementary functions on the IBM RISC System/6000 processor", IBM J. R&D 1990),
-// given rcp(std) correctly rounded.  Verified bit-exact against IEEE division on
-// every bf16 input by the patchify tests.
-__device__ __forceinline__ uint32_t norm_pair(float x0, float x1, float mean, float stdv,
-                                              float nstdv, float rstd) {
-    uint64_t X, M, D, R, NS, Q0, Er, Q;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(x0), "f"(x1));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(M) : "f"(mean));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(R) : "f"(rstd));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(NS) : "f"(nstdv));
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(X), "l"(M));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q0) : "l"(D), "l"(R));
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Er) : "l"(Q0), "l"(NS), "l"(D));
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Q) : "l"(Er), "l"(R), "l"(Q0));
-    float q0, q1;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(q0), "=f"(q1) : "l"(Q));
-    (void)stdv;
-    return pack_bf16x2(q0, q1);
+// Per-channel pixel normalisation x_hat = bf16_rne(fp32(fp32(x - mean) / std)),
+// bit-identical to an IEEE fp32 subtract and divide for every finite input.
+// The host picks one mode per channel:
+//   kNormIdentity  mean == +0 and std == 1: x_hat = bf16_rne(x), a plain copy
+//                  for bf16 frames.
+//   kNormScaled    |mean| >= 2^-70 and 2^-32 <= std <= 2^32: std = s * 2^-k with
+//                  s in [1, 2).  q0 = d * rcp(s), one fused multiply-add
+//                  correction q = q0 + (d - q0 * s) * rcp(s) -- Markstein's
+//                  final step, which returns the correctly rounded quotient when
+//                  rcp(s) is correctly rounded and nothing over/underflows
+//                  (P. Markstein, IBM J. Res. Dev. 34(1), 1990) -- then the
+//                  exact scaling q * 2^k.  With s in [1, 2) the first product
+//                  cannot overflow, and |mean| >= 2^-70 keeps d = x - mean
+//                  either 0 or above 2^-93, so the residual never underflows;
+//                  an overflowing quotient still rounds to +-inf in the final
+//                  scaling.  Checked exhaustively against IEEE division.
+//   kNormDivide    anything else: the IEEE divide itself, per element.
+enum NormMode : int { kNormIdentity = 0, kNormScaled = 1, kNormDivide = 2 };
+
+struct NormConst {
+    float mean, stdv, nstd_s, rcp_s, scale;
+    int mode;
+};
+
+__device__ __forceinline__ NormConst norm_const(const FwdParams &P, int c) {
+    NormConst n;
+    n.mean = P.mean[c];
+    n.stdv = P.stdv[c];
+    n.nstd_s = P.nstd_s[c];
+    n.rcp_s = P.rcp_s[c];
+    n.scale = P.scale[c];
+    n.mode = P.norm_mode[c];
+    return n;
 }
 
-// One 2-pixel word of a frame row, as two fp32.
-template <bool F32IN>
-__device__ __forceinline__ void load_pair(const char *p, float &a, float &b) {
-    if constexpr (F32IN) {
-        float2 v;
-        asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
-        a = v.x;
-        b = v.y;
-    } else {
-        uint32_t w;
-        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w) : "l"(p));
-        a = bf16lo_to_f32(w);
-        b = bf16hi_to_f32(w);
+// Two pixels (lo, hi) -> their normalised values packed as bf16 x 2.
+__device__ __forceinline__ uint32_t norm_pair_f32(float x0, float x1, const NormConst &n) {
+    if (n.mode == kNormScaled) {
+        uint64_t X, M, R, NS, SC, D, Q0, Er, Q;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(x0), "f"(x1));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(M) : "f"(n.mean));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(R) : "f"(n.rcp_s));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(NS) : "f"(n.nstd_s));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(SC) : "f"(n.scale));
+        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(X), "l"(M));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q0) : "l"(D), "l"(R));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Er) : "l"(Q0), "l"(NS), "l"(D));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Q) : "l"(Er), "l"(R), "l"(Q0));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q) : "l"(Q), "l"(SC));
+        float q0, q1;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(q0), "=f"(q1) : "l"(Q));
+        return pack_bf16x2(q0, q1);
     }
+    if (n.mode == kNormDivide)
+        return pack_bf16x2(__fdiv_rn(__fsub_rn(x0, n.mean), n.stdv), __fdiv_rn(__fsub_rn(x1, n.mean), n.stdv));
+    return pack_bf16x2(x0, x1);
 }
+
+// Same for a raw bf16 x 2 word; the identity mode is then the word itself.
+__device__ __forceinline__ uint32_t norm_pair_bf16(uint32_t w, const NormConst &n) {
+    if (n.mode == kNormIdentity) return w;
+    return norm_pair_f32(bf16lo_to_f32(w), bf16hi_to_f32(w), n);
+}
+
+// One 2-pixel word of a frame row: the raw bf16 x 2 word, or two fp32.
+template <bool F32IN> struct PixPair;
+template <> struct PixPair<false> {
+    uint32_t w;
+    __device__ __forceinline__ void load(const char *p) {
+        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w) : "l"(p));
+    }
+    __device__ __forceinline__ void zero() { w = 0u; }
+    __device__ __forceinline__ uint32_t norm(const NormConst &n) const { return norm_pair_bf16(w, n); }
+};
+template <> struct PixPair<true> {
+    float a, b;
+    __device__ __forceinline__ void load(const char *p) {
+        asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "l"(p));
+    }
+    __device__ __forceinline__ void zero() { a = b = 0.f; }
+    __device__ __forceinline__ uint32_t norm(const NormConst &n) const { return norm_pair_f32(a, b, n); }
+};
 
 // Item u of a segment (one 2-pixel word of one tile row) -> (tile row, word).
 // For merge = 2 the order walks patch-row halves of the windows so that
@@ -225,7 +269,7 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ri
         for (int s = 0; s < P.n_a_stages; ++s) {
             if (!mbar_wait(smem_addr(&empty_a[stage]), phase ^ 1, abort)) return;
             uint8_t *As = a_ring + (size_t)stage * P.a_stage_bytes;
-            float va[8][MAXIT], vb[8][MAXIT];
+            PixPair<F32IN> px[8][MAXIT];
             int cq[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -233,12 +277,11 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ri
                 cq[q] = live ? c : -1;
 #pragma unroll
                 for (int v = 0; v < MAXIT; ++v) {
-                    va[q][v] = 0.f;
-                    vb[q][v] = 0.f;
+                    px[q][v].zero();
                     if (live && rok[v]) {
                         const int tt = t < sTm[v] ? t : sTm[v];
                         const int64_t off = (int64_t)tt * sCHW[v] + c * sHW[v] + i * sW[v];
-                        load_pair<F32IN>(src[v] + off * esize, va[q][v], vb[q][v]);
+                        px[q][v].load(src[v] + off * esize);
                     }
                 }
                 if (++i == p) {
@@ -249,12 +292,11 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ri
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int ch = cq[q];
-                float mu = 0.f, sd = 1.f, nsd = -1.f, rs = 1.f;
-                if (ch >= 0) { mu = P.mean[ch]; sd = P.stdv[ch]; nsd = P.nstdv[ch]; rs = P.rstd[ch]; }
+                const NormConst nc = norm_const(P, ch < 0 ? 0 : ch);
 #pragma unroll
                 for (int v = 0; v < MAXIT; ++v) {
                     if (!rok[v]) continue;
-                    const uint32_t w = ch >= 0 ? norm_pair(va[q][v], vb[q][v], mu, sd, nsd, rs) : 0u;
+                    const uint32_t w = ch >= 0 ? px[q][v].norm(nc) : 0u;
                     const int k = q * p + kw[v];
                     const uint32_t off = (uint32_t)(k >> 3) * 2048u + (uint32_t)rr[v] * 16u +
                                          (uint32_t)(k & 7) * 2u;
@@ -592,9 +634,9 @@ __global__ void pe_patchify_kernel(const __grid_constant__ FwdParams P, void *ro
         const RowSrc s = locate_row(P, R, esize);
         const int tt = t < s.tmax ? t : s.tmax;
         const int64_t off = (int64_t)tt * s.CHW + (int64_t)c * s.HW + (int64_t)i * s.W + 2 * jw;
-        float a, b;
-        load_pair<F32IN>(s.base + off * esize, a, b);
-        const uint32_t w = norm_pair(a, b, P.mean[c], P.stdv[c], P.nstdv[c], P.rstd[c]);
+        PixPair<F32IN> px;
+        px.load(s.base + off * esize);
+        const uint32_t w = px.norm(norm_const(P, c));
         const int64_t k = 2 * (int64_t)wk;
         if (rows_f32) {
             float *o = reinterpret_cast<float *>(rows) + R * P.K + k;
