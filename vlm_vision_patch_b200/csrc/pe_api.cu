@@ -24,12 +24,14 @@ struct pe_handle {
     int E = 0, C = 0, tp = 0, p = 0, K = 0, Kpad = 0;
     bool has_bias = false;
     bool weight_set = false;
-    uint16_t *wpack = nullptr;  // dev [E, Kpad] bf16
+    uint16_t *wpack = nullptr;  // dev [E, Kpad] bf16, view(-1, C, tp, p, p) k order
+    uint16_t *wpack_f = nullptr; // dev [E, Kpad] bf16, k order of the frames producer
     float *bias = nullptr;      // dev [E] fp32 (has_bias)
     int *err = nullptr;         // dev error word
     float mean[4] = {0, 0, 0, 0};
     float stdv[4] = {1, 1, 1, 1};
-    CUtensorMap tmap_w[3];      // box rows 64, 128, 256
+    CUtensorMap tmap_w[3];      // weight boxes of 32, 64, 128 rows (half a pair tile)
+    CUtensorMap tmap_wf[3];     // same for the frames-order weight
     int num_sms = 0;
     int smem_optin = 0;
     // item table for grouped calls beyond PE_INLINE_ITEMS
@@ -59,19 +61,32 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (cols contiguous, row stride `ld` elements),
-// box [box_rows, 64], 128-byte swizzle, out-of-bounds elements read as zero.
-bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t ld,
-                    uint32_t box_rows) {
+// 2-D tensor [rows, cols] (cols contiguous, row stride `ld` elements) of bf16 or
+// fp32, box [box_rows, box_cols]; out-of-bounds elements read as zero and are
+// not written by stores.
+bool make_tmap(CUtensorMap *m, const void *base, bool f32, uint64_t rows, uint64_t cols, uint64_t ld,
+               uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const uint64_t es = f32 ? 4 : 2;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {ld * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint64_t strides[1] = {ld * es};
+    cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t ld,
+                    uint32_t box_rows) {
+    return make_tmap(m, base, false, rows, cols, ld, box_rows, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Output [N, E]: 32 x 32 boxes, swizzled to match the epilogue's staging layout.
+bool make_out_tmap(CUtensorMap *m, void *out, bool f32, int64_t N, int E) {
+    return make_tmap(m, out, f32, (uint64_t)N, (uint64_t)E, (uint64_t)E, 32, 32,
+                     f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -100,31 +115,43 @@ int bn_override() {
 // Tile width: frames tiles pay the gather once per tile whatever BN is, so use
 // the widest BN unless the problem is too small to fill the GPU in one wave;
 // TMA-fed patch tiles are cheap to refill, so prefer enough tiles for all SMs.
-int choose_bn(int64_t N, int E, int num_sms, bool gather_fed) {
+int choose_bn(int64_t N, int E, int num_pairs, bool gather_fed) {
     if (const int o = bn_override()) return o;
-    const int64_t mt = (N + kBM - 1) / kBM;
+    const int64_t mt = (N + 2 * kBM - 1) / (2 * kBM);
     auto tiles = [&](int bn) { return mt * ((E + bn - 1) / bn); };
-    if (tiles(256) >= num_sms) return 256;
+    if (tiles(256) >= num_pairs) return 256;
     if (gather_fed) {
-        // Less than one wave even at BN=256: every CTA runs one tile, so the
+        // Less than one wave even at BN=256: every pair runs one tile, so the
         // narrowest BN that still fits one wave finishes first.
-        if (tiles(64) <= num_sms) return 64;
-        if (tiles(128) <= num_sms) return 128;
+        if (tiles(64) <= num_pairs) return 64;
+        if (tiles(128) <= num_pairs) return 128;
         return 256;
     }
-    if (tiles(128) >= num_sms) return 128;
+    if (tiles(128) >= num_pairs) return 128;
     return 64;
 }
 
 template <int AMODE, int PT, bool F32IN>
-cudaError_t launch_fwd(const pe_handle *h, const FwdParams &P, const CUtensorMap &tx, size_t smem,
-                       int grid, cudaStream_t st) {
+cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensorMap &tx, const CUtensorMap &to,
+                       size_t smem, int grid, cudaStream_t st) {
     auto kern = pe_fwd_kernel<AMODE, PT, F32IN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int bi = P.bn == 64 ? 0 : (P.bn == 128 ? 1 : 2);
-    kern<<<grid, kThreads, smem, st>>>(h->tmap_w[bi], tx, P);
+    kern<<<grid, kThreads, smem, st>>>(tw, tx, to, P);
     return cudaGetLastError();
+}
+
+int bn_index(int bn) { return bn == 64 ? 0 : (bn == 128 ? 1 : 2); }
+
+// Pair tiles, grid (two CTAs per pair, at most one pair per two SMs).
+void plan_tiles(const pe_handle *h, FwdParams &P, int64_t N, bool gather_fed, int &grid, bool &ok) {
+    const int num_pairs = h->num_sms / 2;
+    P.bn = choose_bn(N, P.E, num_pairs, gather_fed);
+    P.n_tiles_n = (P.E + P.bn - 1) / P.bn;
+    const int64_t mt = (N + 2 * kBM - 1) / (2 * kBM);
+    ok = mt * P.n_tiles_n <= INT32_MAX;
+    P.num_tiles = ok ? (int)(mt * P.n_tiles_n) : 0;
+    grid = 2 * std::min(P.num_tiles, num_pairs);
 }
 
 void fill_common(const pe_handle *h, FwdParams &P) {
@@ -168,18 +195,23 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
         P.a_stage_bytes = kBM * kBK * 2;
         P.n_a_stages = P.n_b_stages;
     }
-    const size_t b_bytes = (size_t)kMaxBN * kBK * 2;
+    const size_t epi_bytes = (size_t)8 * 32 * 32 * (P.out_f32 ? 4 : 2);
+    auto rings = [&](int nb, int na) { return (size_t)nb * kBStageBytes + (size_t)na * P.a_stage_bytes; };
     auto total = [&](int nb, int na) {
-        return 1024 + (size_t)nb * b_bytes + (size_t)na * P.a_stage_bytes + (size_t)(2 * nb + 2 * na + 5) * 8 + 16;
+        const size_t r = (rings(nb, na) + 1023) / 1024 * 1024;
+        return 1024 + r + epi_bytes + (size_t)(2 * nb + 2 * na + 5) * 8 + 16;
     };
-    int nb = 4, na = (amode == kAModeFrames) ? 3 : 4;
+    int nb = 6, na = (amode == kAModeFrames) ? 4 : 6;
     while (total(nb, na) > (size_t)h->smem_optin) {
-        if (na > 2) --na;
+        if (na > 3) --na;
+        else if (nb > 3) --nb;
+        else if (na > 2) --na;
         else if (nb > 2) --nb;
         else break;
     }
     P.nb = nb;
     P.na = na;
+    P.epi_offset = (int)((rings(nb, na) + 1023) / 1024 * 1024);
     return total(nb, na);
 }
 
@@ -259,29 +291,28 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
 }
 
 pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st) {
-    P.out = out;
     P.out_f32 = out_dt == PE_F32;
     if (P.N == 0) return PE_OK;
-    P.bn = choose_bn(P.N, P.E, h->num_sms, true);
-    P.n_tiles_n = (P.E + P.bn - 1) / P.bn;
-    const int64_t mt = (P.N + kBM - 1) / kBM;
-    if (mt * P.n_tiles_n > INT32_MAX) return PE_ERR_UNSUPPORTED;
-    P.num_tiles = (int)(mt * P.n_tiles_n);
+    int grid = 0;
+    bool ok = true;
+    plan_tiles(h, P, P.N, true, grid, ok);
+    if (!ok) return PE_ERR_UNSUPPORTED;
     const size_t smem = plan_pipeline(h, P, kAModeFrames);
-    const int grid = std::min(P.num_tiles, h->num_sms);
-    CUtensorMap dummy;
+    CUtensorMap dummy, to;
     std::memset(&dummy, 0, sizeof(dummy));
+    if (!make_out_tmap(&to, out, P.out_f32, P.N, P.E)) return PE_ERR_CUDA;
+    const CUtensorMap &tw = h->tmap_wf[bn_index(P.bn)];
     const bool f32 = f_dt == PE_F32;
     cudaError_t e;
     if (h->p == 14)
-        e = f32 ? launch_fwd<kAModeFrames, 14, true>(h, P, dummy, smem, grid, st)
-                : launch_fwd<kAModeFrames, 14, false>(h, P, dummy, smem, grid, st);
+        e = f32 ? launch_fwd<kAModeFrames, 14, true>(tw, P, dummy, to, smem, grid, st)
+                : launch_fwd<kAModeFrames, 14, false>(tw, P, dummy, to, smem, grid, st);
     else if (h->p == 16)
-        e = f32 ? launch_fwd<kAModeFrames, 16, true>(h, P, dummy, smem, grid, st)
-                : launch_fwd<kAModeFrames, 16, false>(h, P, dummy, smem, grid, st);
+        e = f32 ? launch_fwd<kAModeFrames, 16, true>(tw, P, dummy, to, smem, grid, st)
+                : launch_fwd<kAModeFrames, 16, false>(tw, P, dummy, to, smem, grid, st);
     else
-        e = f32 ? launch_fwd<kAModeFrames, 0, true>(h, P, dummy, smem, grid, st)
-                : launch_fwd<kAModeFrames, 0, false>(h, P, dummy, smem, grid, st);
+        e = f32 ? launch_fwd<kAModeFrames, 0, true>(tw, P, dummy, to, smem, grid, st)
+                : launch_fwd<kAModeFrames, 0, false>(tw, P, dummy, to, smem, grid, st);
     return finish(e);
 }
 
@@ -342,14 +373,17 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
     h->Kpad = (int)((K + 63) / 64 * 64);
     h->has_bias = has_bias != 0;
     bool ok = cudaMalloc(&h->wpack, sizeof(uint16_t) * (size_t)E * h->Kpad) == cudaSuccess &&
+              cudaMalloc(&h->wpack_f, sizeof(uint16_t) * (size_t)E * h->Kpad) == cudaSuccess &&
               cudaMalloc(&h->err, sizeof(int)) == cudaSuccess &&
               cudaMemset(h->err, 0, sizeof(int)) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->items_evt, cudaEventDisableTiming) == cudaSuccess;
     if (ok && h->has_bias) ok = cudaMalloc(&h->bias, sizeof(float) * E) == cudaSuccess;
     if (ok) {
-        const uint32_t boxes[3] = {64, 128, 256};
+        const uint32_t boxes[3] = {32, 64, 128};   // half of BN = 64, 128, 256
         for (int i = 0; i < 3 && ok; ++i)
             ok = make_tmap_bf16(&h->tmap_w[i], h->wpack, (uint64_t)E, (uint64_t)h->Kpad, (uint64_t)h->Kpad,
+                                boxes[i]) &&
+                 make_tmap_bf16(&h->tmap_wf[i], h->wpack_f, (uint64_t)E, (uint64_t)h->Kpad, (uint64_t)h->Kpad,
                                 boxes[i]);
     }
     if (!ok) { pe_destroy(h); return PE_ERR_CUDA; }
@@ -362,6 +396,7 @@ void pe_destroy(pe_handle *h) {
     DeviceGuard g(h->dev);
     cudaDeviceSynchronize();
     if (h->wpack) cudaFree(h->wpack);
+    if (h->wpack_f) cudaFree(h->wpack_f);
     if (h->bias) cudaFree(h->bias);
     if (h->err) cudaFree(h->err);
     if (h->items_dev) cudaFree(h->items_dev);
@@ -381,7 +416,10 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
     const int threads = 256;
     const int blocks = (int)std::min<int64_t>((total + threads - 1) / threads, (int64_t)h->num_sms * 8);
     pe_pack_weight_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
-        w, w_dt == PE_F32, bias, b_dt == PE_F32, h->wpack, h->bias, h->E, h->K, h->Kpad);
+        w, w_dt == PE_F32, bias, b_dt == PE_F32, h->wpack, h->bias, h->E, h->C, h->tp, h->p, h->Kpad, 0);
+    if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    pe_pack_weight_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
+        w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_f, nullptr, h->E, h->C, h->tp, h->p, h->Kpad, 1);
     if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
     h->weight_set = true;
     return PE_OK;
@@ -415,26 +453,25 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
     P.N = N;
     P.x = x;
     P.x_f32 = x_dt == PE_F32;
-    P.out = out;
     P.out_f32 = out_dt == PE_F32;
     P.merge = 1;
     const bool tma = (x_dt == PE_BF16) && (h->K % 8 == 0);
     P.x_vec = (x_dt == PE_BF16) ? (h->K % 8 == 0) : (h->K % 4 == 0);
-    P.bn = choose_bn(N, h->E, h->num_sms, false);
-    P.n_tiles_n = (h->E + P.bn - 1) / P.bn;
-    const int64_t mt = (N + kBM - 1) / kBM;
-    if (mt * P.n_tiles_n > INT32_MAX) return PE_ERR_UNSUPPORTED;
-    P.num_tiles = (int)(mt * P.n_tiles_n);
+    int grid = 0;
+    bool ok = true;
+    plan_tiles(h, P, N, !tma, grid, ok);
+    if (!ok) return PE_ERR_UNSUPPORTED;
     const size_t smem = plan_pipeline(h, P, tma ? kAModeTma : kAModePatchThreads);
-    const int grid = std::min(P.num_tiles, h->num_sms);
     cudaStream_t st = (cudaStream_t)stream;
-    CUtensorMap tx;
+    CUtensorMap tx, to;
     std::memset(&tx, 0, sizeof(tx));
+    if (!make_out_tmap(&to, out, P.out_f32, N, h->E)) return PE_ERR_CUDA;
+    const CUtensorMap &tw = h->tmap_w[bn_index(P.bn)];
     if (tma) {
         if (!make_tmap_bf16(&tx, x, (uint64_t)N, (uint64_t)h->K, (uint64_t)h->K, kBM)) return PE_ERR_CUDA;
-        return finish(launch_fwd<kAModeTma, 0, false>(h, P, tx, smem, grid, st));
+        return finish(launch_fwd<kAModeTma, 0, false>(tw, P, tx, to, smem, grid, st));
     }
-    return finish(launch_fwd<kAModePatchThreads, 0, false>(h, P, tx, smem, grid, st));
+    return finish(launch_fwd<kAModePatchThreads, 0, false>(tw, P, tx, to, smem, grid, st));
 }
 
 pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,

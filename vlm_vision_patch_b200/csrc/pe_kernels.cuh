@@ -2,21 +2,25 @@
 //
 // The PatchEmbed is a Conv3d whose kernel equals its stride, i.e. one dense
 // contraction out[N, E] = A[N, K] * W[E, K]^T (+ bias) with K = C*tp*p*p
-// (Qwen2.5VL-Vision Encode-PatchEmbed: "the conv is a dot product of the
-// flattened input and weight"; mytransformer README §4.1: F.linear(x,
-// w.reshape(1280, 1176))).  One persistent kernel runs the whole path:
+// (Qwen2.5VL-Vision Encode-PatchEmbed: the conv is a dot product of the
+// flattened input and weight; mytransformer README §4.1: F.linear(x,
+// w.reshape(1280, 1176))).  One persistent kernel runs the whole path on CTA
+// pairs (thread-block clusters of 2) that share each 256 x BN output tile
+// through the pair form of the 5th-generation MMA (tcgen05 cta_group::2):
+// every CTA stages its own 128 rows of A and BN/2 rows of the weight, the
+// leader CTA issues the MMAs, and each CTA accumulates its 128 rows x BN fp32
+// in its own tensor memory.
 //
 //   warp 0      TMA producer: weight tiles (and A tiles of bf16 patch rows)
-//   warp 1      MMA issuer (one thread) + TMEM owner
-//   warps 4-7   epilogue: TMEM -> registers, + bias, cast, 16-byte stores
-//   warps 8-15  A producers for the thread-fed modes: fp32/unaligned patch rows
-//               (converted to bf16), or the fused frames gather that builds
+//   warp 1      TMEM owner; in the leader CTA one thread issues the MMAs
+//   warps 4-7   epilogue: TMEM -> registers, + bias, cast, TMA stores
+//   warps 8-15  A producers for the thread-fed modes: fp32 / unaligned patch
+//               rows converted to bf16, or the fused frames gather that builds
 //               each patch row from raw [T, C, H, W] frames, normalises it and
 //               places it in merge order, straight into shared memory.
 //
-// Tiles are 128 rows x BN (64/128/256) columns; the fp32 accumulator lives in
-// tensor memory, double buffered (2 x 256 columns) so the epilogue of tile i
-// overlaps the MMAs of tile i+1.  Every pipeline wait is bounded.
+// The accumulator is double buffered (2 x 256 TMEM columns) so the epilogue of
+// one tile overlaps the MMAs of the next.  Every pipeline wait is bounded.
 #pragma once
 
 #include "pe_device.cuh"
@@ -25,12 +29,13 @@
 namespace pe {
 
 constexpr int kThreads = 512;
-constexpr int kBM = 128;           // rows per tile (MMA M)
-constexpr int kMaxBN = 256;        // largest MMA N
+constexpr int kBM = 128;           // rows per CTA (pair tile: 256 rows)
+constexpr int kMaxBN = 256;        // largest pair-MMA N
 constexpr int kBK = 64;            // weight K per TMA stage (one 128-byte swizzle row)
 constexpr int kProdThreads = 256;  // warps 8..15
 constexpr int kProdWarps = 8;
 constexpr int kEpiWarp0 = 4;
+constexpr int kBStageBytes = (kMaxBN / 2) * kBK * 2;   // 16 KB: this CTA's half of the weight tile
 
 enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2 };
 
@@ -43,21 +48,21 @@ struct ItemDesc {
 
 struct FwdParams {
     int32_t E, C, TP, P, K, Kpad;
-    int32_t bn, n_tiles_n, num_tiles, num_ksteps;
-    int32_t n_b_stages, n_a_stages;   // per tile
-    int32_t nb, na;                   // ring depths
+    int32_t bn, n_tiles_n, num_tiles, num_ksteps;   // num_tiles counts pair tiles
+    int32_t n_b_stages, n_a_stages;                 // per tile
+    int32_t nb, na;                                 // ring depths
     int32_t a_stage_bytes;
+    int32_t epi_offset;                             // staging area offset past the rings
     int32_t merge, n_items;
     int64_t N;
     const ItemDesc *items_dev;        // table in device memory when n_items > PE_INLINE_ITEMS
     ItemDesc items[PE_INLINE_ITEMS];
-    float mean[4], stdv[4];          // per-channel normalisation (see NormMode)
+    float mean[4], stdv[4];           // per-channel normalisation (see NormMode)
     float nstd_s[4], rcp_s[4], scale[4];
     int32_t norm_mode[4];
     const void *x;                    // patches input
     int32_t x_f32;                    // patches dtype is fp32
     int32_t x_vec;                    // patch rows allow 16-byte vector loads
-    void *out;
     int32_t out_f32;
     const float *bias;                // fp32 [E] or nullptr
     int *err;                         // device error word
@@ -67,6 +72,15 @@ struct FwdParams {
 
 __device__ __forceinline__ const ItemDesc &item_at(const FwdParams &P, int i) {
     return P.n_items <= PE_INLINE_ITEMS ? P.items[i] : P.items_dev[i];
+}
+
+__device__ __forceinline__ int find_item(const FwdParams &P, int64_t R) {
+    int lo = 0, hi = P.n_items - 1;
+    while (lo < hi) {  // last item with row0 <= R
+        const int mid = (lo + hi + 1) >> 1;
+        if (item_at(P, mid).row0 <= R) lo = mid; else hi = mid - 1;
+    }
+    return lo;
 }
 
 // Output row R -> the patch it embeds.  Items are concatenated in list order;
@@ -82,12 +96,7 @@ struct RowSrc {
 };
 
 __device__ __forceinline__ RowSrc locate_row(const FwdParams &P, int64_t R, int esize) {
-    int lo = 0, hi = P.n_items - 1;
-    while (lo < hi) {  // last item with row0 <= R
-        const int mid = (lo + hi + 1) >> 1;
-        if (item_at(P, mid).row0 <= R) lo = mid; else hi = mid - 1;
-    }
-    const ItemDesc &it = item_at(P, lo);
+    const ItemDesc &it = item_at(P, find_item(P, R));
     const int64_t rho = R - it.row0;
     int64_t g_t, g_h, g_w;
     if (P.merge == 2) {
@@ -116,6 +125,8 @@ __device__ __forceinline__ RowSrc locate_row(const FwdParams &P, int64_t R, int 
     s.base = reinterpret_cast<const char *>(it.frames) + el * esize;
     return s;
 }
+
+// ------------------------------------------------------------ normalisation
 
 // Per-channel pixel normalisation x_hat = bf16_rne(fp32(fp32(x - mean) / std)),
 // bit-identical to an IEEE fp32 subtract and divide for every finite input.
@@ -200,7 +211,9 @@ template <> struct PixPair<true> {
     __device__ __forceinline__ uint32_t norm(const NormConst &n) const { return norm_pair_f32(a, b, n); }
 };
 
-// Item u of a segment (one 2-pixel word of one tile row) -> (tile row, word).
+// ------------------------------------------------------------- producers
+
+// Unit u of a segment (one 2-pixel word of one tile row) -> (tile row, word).
 // For merge = 2 the order walks patch-row halves of the windows so that
 // consecutive u read consecutive words of one image row.
 __device__ __forceinline__ void unit_to_row_word(int u, int ws, int merge, int &r, int &jw) {
@@ -215,44 +228,86 @@ __device__ __forceinline__ void unit_to_row_word(int u, int ws, int merge, int &
     }
 }
 
-// ------------------------------------------------------------- producers
+// Shared state of the A producers of one CTA.
+struct ProdCtx {
+    uint8_t *a_ring;
+    uint64_t *empty_a;          // this CTA's empty barriers
+    uint32_t full_a_leader;     // shared::cluster address of the leader's full_a[0]
+    volatile int *abort;
+    int pt, lane;
+    uint32_t rank;
+};
 
-// Frames producer: every A stage holds 8 whole segments (c, t, i) of p pixels,
-// i.e. 8p consecutive k of the view(-1, C, tp, p, p) order, in the no-swizzle
-// K-major layout: element (r, k) at (k / 8) * 2048 + r * 16 + (k % 8) * 2.
+// The stage's generic-proxy writes become visible to the MMA, then one arrival
+// per warp on the leader's full barrier.
+__device__ __forceinline__ void producer_release(const ProdCtx &X, int stage) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (X.lane == 0) mbar_arrive_cluster(X.full_a_leader + 8u * (uint32_t)stage);
+}
+
+// Frames producer.  The frames path runs in the K order k' = ((c*p + i)*tp + t)*p + j
+// (the weight is packed in the same order), so that one A stage holds 8 whole
+// segments (c, i, t) of p pixels: 4 (c, i) pairs x both temporal slices when
+// tp = 2.  Layout: no-swizzle K-major, element (r, k') at
+// (k' / 8) * 2048 + r * 16 + (k' % 8) * 2 of the stage.
 template <int PT, bool F32IN>
-__device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ring,
-                                               uint64_t *full_a, uint64_t *empty_a,
-                                               volatile int *abort, int pt, int lane) {
+__device__ __forceinline__ void produce_frames(const FwdParams &P, const ProdCtx &X) {
     const int p = PT ? PT : P.P;
     const int ws = p >> 1;
     const int units = kBM * ws;
     constexpr int MAXIT = PT ? (PT + 3) / 4 : (PE_MAX_PATCH + 3) / 4;
     constexpr int esize = F32IN ? 4 : 2;
-    const int nseg = P.C * P.TP * p;
+    const int TP = P.TP;
+    const int nseg = P.C * TP * p;
+    const int nci = P.C * p;            // (c, i) pairs
 
     int rr[MAXIT], kw[MAXIT];
     bool uok[MAXIT];
 #pragma unroll
     for (int v = 0; v < MAXIT; ++v) {
-        const int u = pt + kProdThreads * v;
+        const int u = X.pt + kProdThreads * v;
         uok[v] = u < units;
         int r = 0, jw = 0;
         if (uok[v]) unit_to_row_word(u, ws, P.merge, r, jw);
         rr[v] = r;
         kw[v] = 2 * jw;
     }
+    // shared-memory byte offset of (row, k' = q*p + kw) inside a stage
+    auto soff = [&](int q, int v) -> uint32_t {
+        const int k = q * p + kw[v];
+        return (uint32_t)(k >> 3) * 2048u + (uint32_t)rr[v] * 16u + (uint32_t)(k & 7) * 2u;
+    };
 
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
-        const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * kBM;
+    for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+        const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * (2 * kBM) + X.rank * kBM;
+        if (m0 >= P.N) {
+            // Nothing of this CTA's half exists: release the stages untouched
+            // (their rows are never stored).
+            for (int s = 0; s < P.n_a_stages; ++s) {
+                if (!mbar_wait(smem_addr(&X.empty_a[stage]), phase ^ 1, X.abort)) return;
+                producer_release(X, stage);
+                if (++stage == P.na) { stage = 0; phase ^= 1; }
+            }
+            continue;
+        }
+        const int64_t mlast = (m0 + kBM - 1 < P.N) ? m0 + kBM - 1 : P.N - 1;
+        const int it0 = find_item(P, m0);
+        const bool fast = (TP == 2) && (it0 == find_item(P, mlast));
+        const ItemDesc &itd = item_at(P, it0);
+        const bool dup = fast && itd.T == 1;     // both temporal slices are the same frame
+        const int uW = itd.W, uHW = itd.H * itd.W;
+
         const char *src[MAXIT];
         int32_t sW[MAXIT], sHW[MAXIT], sCHW[MAXIT], sTm[MAXIT];
         bool rok[MAXIT];
 #pragma unroll
         for (int v = 0; v < MAXIT; ++v) {
             rok[v] = uok[v] && (m0 + rr[v] < P.N);
+            src[v] = nullptr;
+            sW[v] = sHW[v] = sCHW[v] = sTm[v] = 0;
             if (rok[v]) {
                 const RowSrc s = locate_row(P, m0 + rr[v], esize);
                 src[v] = s.base + (int64_t)kw[v] * esize;
@@ -260,52 +315,81 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ri
                 sHW[v] = s.HW;
                 sCHW[v] = s.CHW;
                 sTm[v] = s.tmax;
-            } else {
-                src[v] = nullptr;
-                sW[v] = sHW[v] = sCHW[v] = sTm[v] = 0;
             }
         }
-        int c = 0, t = 0, i = 0;  // segment counters, seg = (c * TP + t) * p + i
+        int c = 0, i = 0;   // (c, i) of the stage's first segment pair (fast path)
         for (int s = 0; s < P.n_a_stages; ++s) {
-            if (!mbar_wait(smem_addr(&empty_a[stage]), phase ^ 1, abort)) return;
-            uint8_t *As = a_ring + (size_t)stage * P.a_stage_bytes;
-            PixPair<F32IN> px[8][MAXIT];
-            int cq[8];
+            if (!mbar_wait(smem_addr(&X.empty_a[stage]), phase ^ 1, X.abort)) return;
+            uint8_t *As = X.a_ring + (size_t)stage * P.a_stage_bytes;
+            if (fast) {
+                // 4 (c, i) pairs, t = 0 and t = 1 each: segment q = 2 * qq + t
+                PixPair<F32IN> px[4][2][MAXIT];
+                int cq[4];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const bool live = (8 * s + q) < nseg;
-                cq[q] = live ? c : -1;
+                for (int qq = 0; qq < 4; ++qq) {
+                    const bool live = (4 * s + qq) < nci;
+                    cq[qq] = live ? c : -1;
+                    const int64_t uoff = ((int64_t)c * uHW + (int64_t)i * uW) * esize;
 #pragma unroll
-                for (int v = 0; v < MAXIT; ++v) {
-                    px[q][v].zero();
-                    if (live && rok[v]) {
-                        const int tt = t < sTm[v] ? t : sTm[v];
-                        const int64_t off = (int64_t)tt * sCHW[v] + c * sHW[v] + i * sW[v];
-                        px[q][v].load(src[v] + off * esize);
+                    for (int v = 0; v < MAXIT; ++v) {
+                        px[qq][0][v].zero();
+                        px[qq][1][v].zero();
+                        if (live && rok[v]) {
+                            px[qq][0][v].load(src[v] + uoff);
+                            if (!dup) {
+                                const int64_t t1 = (sTm[v] > 0 ? (int64_t)sCHW[v] : 0) * esize;
+                                px[qq][1][v].load(src[v] + uoff + t1);
+                            }
+                        }
+                    }
+                    if (++i == p) { i = 0; ++c; }
+                }
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int ch = cq[qq];
+                    const NormConst nc = norm_const(P, ch < 0 ? 0 : ch);
+#pragma unroll
+                    for (int v = 0; v < MAXIT; ++v) {
+                        if (!rok[v]) continue;
+                        const uint32_t w0 = ch >= 0 ? px[qq][0][v].norm(nc) : 0u;
+                        const uint32_t w1 = dup ? w0 : (ch >= 0 ? px[qq][1][v].norm(nc) : 0u);
+                        *reinterpret_cast<uint32_t *>(As + soff(2 * qq, v)) = w0;
+                        *reinterpret_cast<uint32_t *>(As + soff(2 * qq + 1, v)) = w1;
                     }
                 }
-                if (++i == p) {
-                    i = 0;
-                    if (++t == P.TP) { t = 0; ++c; }
+            } else {
+                PixPair<F32IN> px[8][MAXIT];
+                int cq[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int seg = 8 * s + q;
+                    const bool live = seg < nseg;
+                    const int t = seg % TP, ci = seg / TP;
+                    const int cc = ci / p, ii = ci - cc * p;
+                    cq[q] = live ? cc : -1;
+#pragma unroll
+                    for (int v = 0; v < MAXIT; ++v) {
+                        px[q][v].zero();
+                        if (live && rok[v]) {
+                            const int tt = t < sTm[v] ? t : sTm[v];
+                            const int64_t off = (int64_t)tt * sCHW[v] + (int64_t)cc * sHW[v] + (int64_t)ii * sW[v];
+                            px[q][v].load(src[v] + off * esize);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int ch = cq[q];
+                    const NormConst nc = norm_const(P, ch < 0 ? 0 : ch);
+#pragma unroll
+                    for (int v = 0; v < MAXIT; ++v) {
+                        if (!rok[v]) continue;
+                        const uint32_t w = ch >= 0 ? px[q][v].norm(nc) : 0u;
+                        *reinterpret_cast<uint32_t *>(As + soff(q, v)) = w;
+                    }
                 }
             }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int ch = cq[q];
-                const NormConst nc = norm_const(P, ch < 0 ? 0 : ch);
-#pragma unroll
-                for (int v = 0; v < MAXIT; ++v) {
-                    if (!rok[v]) continue;
-                    const uint32_t w = ch >= 0 ? px[q][v].norm(nc) : 0u;
-                    const int k = q * p + kw[v];
-                    const uint32_t off = (uint32_t)(k >> 3) * 2048u + (uint32_t)rr[v] * 16u +
-                                         (uint32_t)(k & 7) * 2u;
-                    *reinterpret_cast<uint32_t *>(As + off) = w;
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&full_a[stage]));
+            producer_release(X, stage);
             if (++stage == P.na) { stage = 0; phase ^= 1; }
         }
     }
@@ -314,20 +398,18 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, uint8_t *a_ri
 // Patch-row producer for rows the TMA cannot fetch directly (fp32 rows, or bf16
 // rows whose stride is not a multiple of 16 bytes): 64 k per stage, converted
 // to bf16 (RNE) into the no-swizzle K-major layout.
-__device__ __forceinline__ void produce_patches(const FwdParams &P, uint8_t *a_ring,
-                                                uint64_t *full_a, uint64_t *empty_a,
-                                                volatile int *abort, int pt, int lane) {
+__device__ __forceinline__ void produce_patches(const FwdParams &P, const ProdCtx &X) {
     const int K = P.K;
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
-        const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * kBM;
+    for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+        const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * (2 * kBM) + X.rank * kBM;
         for (int s = 0; s < P.n_a_stages; ++s) {
-            if (!mbar_wait(smem_addr(&empty_a[stage]), phase ^ 1, abort)) return;
-            uint8_t *As = a_ring + (size_t)stage * P.a_stage_bytes;
+            if (!mbar_wait(smem_addr(&X.empty_a[stage]), phase ^ 1, X.abort)) return;
+            uint8_t *As = X.a_ring + (size_t)stage * P.a_stage_bytes;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-                const int u = pt + kProdThreads * v;  // 0..1023
+                const int u = X.pt + kProdThreads * v;  // 0..1023
                 const int r = u >> 3, kg = u & 7;
                 const int64_t R = m0 + r;
                 const int k0 = s * kBK + kg * 8;
@@ -363,9 +445,7 @@ __device__ __forceinline__ void produce_patches(const FwdParams &P, uint8_t *a_r
                 }
                 *reinterpret_cast<uint4 *>(As + kg * 2048 + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&full_a[stage]));
+            producer_release(X, stage);
             if (++stage == P.na) { stage = 0; phase ^= 1; }
         }
     }
@@ -374,15 +454,16 @@ __device__ __forceinline__ void produce_patches(const FwdParams &P, uint8_t *a_r
 // ------------------------------------------------------------- the kernel
 
 template <int AMODE, int PT, bool F32IN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pe_fwd_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                  const __grid_constant__ FwdParams P) {
+                  const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ FwdParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const int b_stage_bytes = kMaxBN * kBK * 2;
     uint8_t *b_ring = smem;
-    uint8_t *a_ring = b_ring + (size_t)P.nb * b_stage_bytes;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(a_ring + (size_t)P.na * P.a_stage_bytes);
+    uint8_t *a_ring = b_ring + (size_t)P.nb * kBStageBytes;
+    uint8_t *epi = smem + P.epi_offset;
+    const int epi_buf_bytes = 32 * 32 * (P.out_f32 ? 4 : 2);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(epi + 8 * epi_buf_bytes);
     uint64_t *full_b = bars;
     uint64_t *empty_b = full_b + P.nb;
     uint64_t *full_a = empty_b + P.nb;
@@ -394,6 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    constexpr uint16_t kPair = 0x3;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P.nb; ++s) {
@@ -401,12 +485,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_addr(&empty_b[s]), 1);
         }
         for (int s = 0; s < P.na; ++s) {
-            mbar_init(smem_addr(&full_a[s]), AMODE == kAModeTma ? 1 : kProdWarps);
+            mbar_init(smem_addr(&full_a[s]), AMODE == kAModeTma ? 1 : 2 * kProdWarps);
             mbar_init(smem_addr(&empty_a[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&tfull[s]), 1);
-            mbar_init(smem_addr(&tempty[s]), 4);
+            mbar_init(smem_addr(&tempty[s]), 8);
         }
         mbar_init(smem_addr(mma_done), 1);
         *abort = 0;
@@ -414,59 +498,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_out);
         if (AMODE == kAModeTma) prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_holder), 512);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_addr(tmem_holder), 512);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- TMA producer (both CTAs; bytes complete on the leader's barriers)
         if (lane == 0) {
             const uint64_t pol_w = l2_policy_evict_last();
             const uint64_t pol_x = l2_policy_evict_first();
-            const uint32_t b_bytes = (uint32_t)P.bn * kBK * 2;
+            const uint32_t b_bytes = (uint32_t)(P.bn / 2) * kBK * 2;
+            const uint32_t a_bytes = kBM * kBK * 2;
+            const uint32_t fb0 = mapa_shared(smem_addr(&full_b[0]), 0);
+            const uint32_t fa0 = mapa_shared(smem_addr(&full_a[0]), 0);
             int bs = 0, as = 0;
             uint32_t bph = 0, aph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < P.num_tiles && ok; tile += gridDim.x) {
+            for (int tile = blockIdx.x >> 1; tile < P.num_tiles && ok; tile += gridDim.x >> 1) {
                 const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
                 for (int kb = 0; kb < P.n_b_stages && ok; ++kb) {
                     if (AMODE == kAModeTma) {
                         if (!mbar_wait(smem_addr(&empty_a[as]), aph ^ 1, abort)) { ok = false; break; }
-                        mbar_arrive_expect_tx(smem_addr(&full_a[as]), kBM * kBK * 2);
-                        tma_load_2d(smem_addr(a_ring + (size_t)as * P.a_stage_bytes), &tmap_x,
-                                    smem_addr(&full_a[as]), kb * kBK, m_blk * kBM, pol_x);
+                        if (leader) mbar_arrive_expect_tx(smem_addr(&full_a[as]), 2 * a_bytes);
+                        tma_load_2d_pair(smem_addr(a_ring + (size_t)as * P.a_stage_bytes), &tmap_x, fa0 + 8u * as,
+                                         kb * kBK, m_blk * (2 * kBM) + (int)rank * kBM, pol_x);
                         if (++as == P.na) { as = 0; aph ^= 1; }
                     }
                     if (!mbar_wait(smem_addr(&empty_b[bs]), bph ^ 1, abort)) { ok = false; break; }
-                    mbar_arrive_expect_tx(smem_addr(&full_b[bs]), b_bytes);
-                    tma_load_2d(smem_addr(b_ring + (size_t)bs * b_stage_bytes), &tmap_w,
-                                smem_addr(&full_b[bs]), kb * kBK, n_blk * P.bn, pol_w);
+                    if (leader) mbar_arrive_expect_tx(smem_addr(&full_b[bs]), 2 * b_bytes);
+                    tma_load_2d_pair(smem_addr(b_ring + (size_t)bs * kBStageBytes), &tmap_w, fb0 + 8u * bs,
+                                     kb * kBK, n_blk * P.bn + (int)rank * (P.bn / 2), pol_w);
                     if (++bs == P.nb) { bs = 0; bph ^= 1; }
                 }
             }
-            // Drain: let the last loads of every ring slot land before exiting.
+            // Drain: the MMA signals every consumed stage back on our empty
+            // barriers; waiting for the last signal of each slot means every
+            // load this CTA issued has landed and been read.
             for (int s = 0; s < P.nb; ++s) {
-                const int slot = (bs + s) % P.nb;  // oldest first
-                const uint32_t par = (slot < bs) ? bph : (bph ^ 1);
-                mbar_wait(smem_addr(&full_b[slot]), par, abort);
+                const int slot = (bs + s) % P.nb;
+                mbar_wait(smem_addr(&empty_b[slot]), (slot < bs) ? bph : (bph ^ 1), abort);
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(kBM, P.bn);
+        // ---------------- MMA issuer (leader CTA only)
+        if (leader && lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
             const int ks_a = (AMODE == kAModeFrames) ? (P.P >> 1) : (kBK / 16);
             int bs = 0, as = 0, acc = 0;
             uint32_t bph = 0, aph = 0, accph = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < P.num_tiles && ok; tile += gridDim.x) {
+            for (int tile = blockIdx.x >> 1; tile < P.num_tiles && ok; tile += gridDim.x >> 1) {
                 if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * kMaxBN;
@@ -481,128 +570,144 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                     }
                     const uint32_t a_base = smem_addr(a_ring + (size_t)as * P.a_stage_bytes);
-                    const uint32_t b_base = smem_addr(b_ring + (size_t)bs * b_stage_bytes);
+                    const uint32_t b_base = smem_addr(b_ring + (size_t)bs * kBStageBytes);
                     uint64_t adesc;
                     if (AMODE == kAModeTma)
                         adesc = smem_desc(a_base + ka * 32, 16, 1024, kLayoutSw128);
                     else
                         adesc = smem_desc(a_base + ka * 4096, 2048, 128, kLayoutInterleave);
                     const uint64_t bdesc = smem_desc(b_base + kbi * 32, 16, 1024, kLayoutSw128);
-                    mma_bf16(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+                    mma_bf16_pair(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
                     const bool last = (ks == P.num_ksteps - 1);
                     if (++kbi == kBK / 16 || last) {
-                        mma_commit(smem_addr(&empty_b[bs]));
+                        mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
                         kbi = 0;
                         if (++bs == P.nb) { bs = 0; bph ^= 1; }
                     }
                     if (++ka == ks_a || last) {
-                        mma_commit(smem_addr(&empty_a[as]));
+                        mma_commit_pair(smem_addr(&empty_a[as]), kPair);
                         ka = 0;
                         if (++as == P.na) { as = 0; aph ^= 1; }
                     }
                 }
                 if (!ok) break;
-                mma_commit(smem_addr(&tfull[acc]));
+                mma_commit_pair(smem_addr(&tfull[acc]), kPair);
                 if (++acc == 2) { acc = 0; accph ^= 1; }
             }
-            mma_commit(smem_addr(mma_done));
+            mma_commit_pair(smem_addr(mma_done), 0x1);
             mbar_wait(smem_addr(mma_done), 0, abort);
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
-        // ---------------- epilogue
+        // ---------------- epilogue (both CTAs)
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
-        int acc = 0;
+        const uint32_t tempty0 = mapa_shared(smem_addr(&tempty[0]), 0);
+        uint8_t *stage_buf = epi + (size_t)wq * 2 * epi_buf_bytes;
+        int acc = 0, nbuf = 0;
         uint32_t accph = 0;
-        for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
+        for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
             const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
             if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
             tc_fence_after();
-            const int64_t row = (int64_t)m_blk * kBM + wq * 32 + lane;
-            const bool row_ok = row < P.N;
+            const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
             for (int cc = 0; cc < P.bn / 32; ++cc) {
                 uint32_t v[32];
                 const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN + cc * 32);
                 tmem_ld_32x32b_x32(taddr, v);
                 tmem_ld_wait();
                 const int col0 = n_blk * P.bn + cc * 32;
-                if (!row_ok || col0 >= P.E) continue;
+                if (row0 >= P.N || col0 >= P.E) continue;   // whole box outside: nothing to store
                 float f[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
                 if (P.bias) {
-                    if (col0 + 32 <= P.E) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4) {
-                            const float4 b = __ldg(reinterpret_cast<const float4 *>(P.bias + col0 + e));
-                            f[e] += b.x; f[e + 1] += b.y; f[e + 2] += b.z; f[e + 3] += b.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
                 }
+                // this warp's staging buffer must be free of the store issued two chunks ago
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+                uint8_t *buf = stage_buf + (size_t)nbuf * epi_buf_bytes;
                 if (P.out_f32) {
-                    float *o = reinterpret_cast<float *>(P.out) + row * P.E + col0;
-                    if (col0 + 32 <= P.E) {
+                    // 128-byte rows, 128-byte swizzle: chunk c of row r at (c ^ (r & 7))
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4 *>(o + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (col0 + e < P.E) o[e] = f[e];
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<float4 *>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_float4(f[4 * c], f[4 * c + 1], f[4 * c + 2], f[4 * c + 3]);
                 } else {
-                    uint32_t h[16];
+                    // 64-byte rows, 64-byte swizzle: chunk c of row r at (c ^ ((r >> 1) & 3))
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) h[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
-                    uint16_t *o = reinterpret_cast<uint16_t *>(P.out) + row * P.E + col0;
-                    if (col0 + 32 <= P.E) {
-#pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            *reinterpret_cast<uint4 *>(o + 2 * e) = make_uint4(h[e], h[e + 1], h[e + 2], h[e + 3]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (col0 + 2 * e < P.E) *reinterpret_cast<uint32_t *>(o + 2 * e) = h[e];
-                    }
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(pack_bf16x2(f[8 * c], f[8 * c + 1]), pack_bf16x2(f[8 * c + 2], f[8 * c + 3]),
+                                       pack_bf16x2(f[8 * c + 4], f[8 * c + 5]),
+                                       pack_bf16x2(f[8 * c + 6], f[8 * c + 7]));
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_out, smem_addr(buf), col0, (int32_t)row0);
+                    bulk_commit();
+                }
+                nbuf ^= 1;
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&tempty[acc]));
+            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
             if (++acc == 2) { acc = 0; accph ^= 1; }
         }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     } else if (warp >= 8) {
-        // ---------------- A producers
+        // ---------------- A producers (both CTAs)
+        ProdCtx X;
+        X.a_ring = a_ring;
+        X.empty_a = empty_a;
+        X.full_a_leader = mapa_shared(smem_addr(&full_a[0]), 0);
+        X.abort = abort;
+        X.pt = threadIdx.x - 256;
+        X.lane = lane;
+        X.rank = rank;
         if constexpr (AMODE == kAModeFrames)
-            produce_frames<PT, F32IN>(P, a_ring, full_a, empty_a, abort, threadIdx.x - 256, lane);
+            produce_frames<PT, F32IN>(P, X);
         else if constexpr (AMODE == kAModePatchThreads)
-            produce_patches(P, a_ring, full_a, empty_a, abort, threadIdx.x - 256, lane);
+            produce_patches(P, X);
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        tmem_dealloc_pair(tmem_base, 512);
     }
     if (threadIdx.x == 0 && *abort) atomicExch(P.err, (int)PE_ERR_DEVICE_TIMEOUT);
 }
 
 // ------------------------------------------------------------- helpers
 
-// Ŵ[e, k] = bf16_rne(W[e, k]) for k < K, 0 for K <= k < Kpad; bias widened to fp32.
+// Weight packing.  Ŵ[e, k] = bf16_rne(W[e, k]) for k < K and 0 for K <= k < Kpad,
+// stored either in the view(-1, C, tp, p, p) order k = ((c*tp + t)*p + i)*p + j
+// (patches path) or, with `frames_order`, in the order
+// k' = ((c*p + i)*tp + t)*p + j the frames producer fills its stages in.
+// The bias is widened exactly to fp32.
 __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias, int b_f32,
-                                      uint16_t *wpack, float *bias32, int E, int K, int Kpad) {
+                                      uint16_t *wpack, float *bias32, int E, int C, int TP, int P,
+                                      int Kpad, int frames_order) {
+    const int K = C * TP * P * P;
     const int64_t total = (int64_t)E * Kpad;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t e = idx / Kpad;
-        const int k = (int)(idx - e * Kpad);
+        const int kd = (int)(idx - e * Kpad);
         uint16_t v = 0;
-        if (k < K) {
+        if (kd < K) {
+            int k = kd;
+            if (frames_order) {
+                const int j = kd % P, t = (kd / P) % TP, ci = kd / (P * TP);
+                const int c = ci / P, i = ci % P;
+                k = ((c * TP + t) * P + i) * P + j;
+            }
             if (w_f32) {
                 const __nv_bfloat16 b = __float2bfloat16_rn(reinterpret_cast<const float *>(w)[e * K + k]);
                 v = *reinterpret_cast<const uint16_t *>(&b);
@@ -611,14 +716,15 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
             }
         }
         wpack[idx] = v;
-        if (k == 0 && bias && bias32)
+        if (kd == 0 && bias && bias32)
             bias32[e] = b_f32 ? reinterpret_cast<const float *>(bias)[e]
                               : __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(bias)[e] << 16);
     }
 }
 
-// rows[R, k] for every output row R: the frames producer's gather and
-// normalisation written to memory (bf16 or fp32 values; bf16-exact either way).
+// rows[R, k] for every output row R, in the view(-1, C, tp, p, p) order: the
+// frames producer's gather and normalisation written to memory (bf16 or fp32
+// values; bf16-exact either way).
 template <bool F32IN>
 __global__ void pe_patchify_kernel(const __grid_constant__ FwdParams P, void *rows, int rows_f32) {
     constexpr int esize = F32IN ? 4 : 2;

@@ -172,6 +172,14 @@ def long_video_64x896() -> Workload:
                     mean=CLIP_MEAN, std=CLIP_STD)
 
 
+def patches_bf16_131072() -> Workload:
+    """pixel_values [131072, 1176] bf16 ~N(0,1) (the long-video row count) against
+    the bf16 N(0,0.02) weight: the TMA-fed patches form at full size."""
+    x = normal((131072, 1176), 13, dtype=torch.bfloat16)
+    return Workload("patches_bf16_131072", 1280, 3, 2, 14, _w_bf16(1280, 3, 2, 14, 4), None,
+                    torch.bfloat16, merge=1, patches=x)
+
+
 ALL = {
     "patches_fp32_1024": patches_fp32_1024,
     "image_224x896": image_224x896,
@@ -179,4 +187,5 @@ ALL = {
     "image_448_e1152": image_448_e1152,
     "grouped_16_images": grouped_16_images,
     "long_video_64x896": long_video_64x896,
+    "patches_bf16_131072": patches_bf16_131072,
 }
