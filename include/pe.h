@@ -159,6 +159,34 @@ pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *fram
                                     const int32_t *THW, const int32_t *grid_thw, int merge,
                                     void *out, pe_dtype out_dt, pe_stream_t stream);
 
+/* Largest item count pe_forward_frames_grouped_noalloc accepts. */
+#define PE_NOALLOC_MAX_ITEMS 1024
+
+/*
+ * pe_forward_frames_grouped_noalloc -- pe_forward_frames_grouped for callers
+ * that must not allocate memory while they run: serving loops that hand every
+ * byte of device memory to their own pool up front and forbid cudaMalloc
+ * (and its implicit device synchronisation) on the request path.  The plain
+ * grouped call allocates, on its first group of more than PE_INLINE_ITEMS
+ * items, a device table and a pinned host staging buffer in the handle; this
+ * variant instead uses a fixed table of PE_NOALLOC_MAX_ITEMS item descriptors
+ * (40 bytes each) in the library's static device memory, which every device
+ * that loads the library holds until the process exits.  It never calls
+ * cudaMalloc, cudaMallocHost or cudaFree.  The pages have no counterpart: this
+ * is an allocation-free calling convention of this library only.
+ *
+ * Arguments, layouts and results are those of pe_forward_frames_grouped.
+ * n > PE_NOALLOC_MAX_ITEMS returns PE_ERR_UNSUPPORTED before anything runs.
+ * The first call on a device (with more than PE_INLINE_ITEMS items) looks up
+ * the table's device address; make that first call before any stream capture.
+ * All calls share the one table and it keeps the last call's contents, so calls
+ * that can overlap on the GPU (different streams) race; calls on one stream
+ * are ordered and safe.
+ */
+pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                            const int32_t *THW, const int32_t *grid_thw, int merge,
+                                            void *out, pe_dtype out_dt, pe_stream_t stream);
+
 /*
  * pe_patchify -- test hook: the fused producer's gather and normalisation
  * written out to memory instead of feeding the tensor cores.

@@ -22,11 +22,12 @@ STATUS = {
 }
 PE_INLINE_ITEMS = 16
 PE_MAX_PATCH = 32
+PE_NOALLOC_MAX_ITEMS = 1024
 
 # Every symbol include/pe.h declares.
 EXPORTS = (
     "pe_create", "pe_set_weight", "pe_set_norm", "pe_forward_patches", "pe_forward_frames",
-    "pe_forward_frames_grouped", "pe_patchify", "pe_num_patches", "pe_last_error",
+    "pe_forward_frames_grouped", "pe_forward_frames_grouped_noalloc", "pe_patchify", "pe_num_patches", "pe_last_error",
     "pe_status_string", "pe_destroy", "pe_device",
 )
 
@@ -61,6 +62,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_forward_patches": ([vp, vp, i32, i64, vp, i32, vp], i32),
         "pe_forward_frames": ([vp, vp, i32, i32, i32, i32, i32p, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
+        "pe_forward_frames_grouped_noalloc": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
         "pe_patchify": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
         "pe_num_patches": ([i32p, i32], i64),
         "pe_last_error": ([vp], i32),
@@ -137,6 +139,15 @@ def pe_forward_frames_grouped(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Seq
                               stream: int) -> None:
     n = len(f_ptrs)
     _check("pe_forward_frames_grouped", load().pe_forward_frames_grouped(
+        h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
+        _i32arr([v for g in grid_thw for v in g]), merge, out_ptr, out_dt, stream))
+
+
+def pe_forward_frames_grouped_noalloc(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence[int]],
+                                      grid_thw: Sequence[Sequence[int]], merge: int, out_ptr: int, out_dt: int,
+                                      stream: int) -> None:
+    n = len(f_ptrs)
+    _check("pe_forward_frames_grouped_noalloc", load().pe_forward_frames_grouped_noalloc(
         h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
         _i32arr([v for g in grid_thw for v in g]), merge, out_ptr, out_dt, stream))
 

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -513,6 +514,86 @@ pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f
     else
         pe_patchify_kernel<false><<<blocks, threads, 0, st>>>(P, rows, rows_dt == PE_F32);
     return finish(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// pe_forward_frames_grouped_noalloc: the grouped call with its item table in
+// this fixed, file-scope device array instead of the handle's workspace.  The
+// array lives in every device that loads the library, for the life of the
+// process.  Host code must not hand the symbol itself to a kernel (on the host
+// it only names a stand-in); its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) ItemDesc g_noalloc_items[PE_NOALLOC_MAX_ITEMS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+ItemDesc *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_items on the current device (set up on first use).
+cudaError_t noalloc_table(int dev, ItemDesc **out) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_items);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = static_cast<ItemDesc *>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                            const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
+                                            pe_dtype out_dt, pe_stream_t stream) {
+    if (!h || n < 1 || !frames || !THW || !grid_thw || !out) return PE_ERR_INVALID_ARG;
+    if (n > PE_NOALLOC_MAX_ITEMS) return PE_ERR_UNSUPPORTED;
+    if (!valid_dtype(f_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
+    if (merge != 1 && merge != 2) return PE_ERR_INVALID_ARG;
+    if (!h->weight_set) return PE_ERR_NO_WEIGHT;
+    if ((h->p & 1) || h->p > PE_MAX_PATCH) return PE_ERR_UNSUPPORTED;
+    if (!aligned16(out)) return PE_ERR_ALIGN;
+    DeviceGuard g(h->dev);
+    cudaStream_t st = (cudaStream_t)stream;
+    FwdParams P;
+    fill_common(h, P);
+    P.merge = merge;
+    P.n_items = n;
+    // Validate every item before anything is copied or launched.
+    int64_t row0 = 0;
+    for (int i = 0; i < n; ++i) {
+        ItemDesc d;
+        const pe_status s = make_item(h, frames[i], THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid_thw + 3 * i,
+                                      merge, row0, d);
+        if (s != PE_OK) return s;
+        if (n <= PE_INLINE_ITEMS) P.items[i] = d;
+        row0 += (int64_t)grid_thw[3 * i] * grid_thw[3 * i + 1] * grid_thw[3 * i + 2];
+    }
+    P.N = row0;
+    if (n > PE_INLINE_ITEMS) {
+        ItemDesc *table = nullptr;
+        if (noalloc_table(h->dev, &table) != cudaSuccess) return PE_ERR_CUDA;
+        // Upload in stack-sized chunks; a pageable-source copy returns once the
+        // chunk has been staged, so the stack buffer can be reused at once.
+        ItemDesc chunk[64];
+        int64_t r0 = 0;
+        for (int base = 0; base < n; base += 64) {
+            const int m = std::min(64, n - base);
+            for (int j = 0; j < m; ++j) {
+                const int i = base + j;
+                make_item(h, frames[i], THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid_thw + 3 * i, merge, r0,
+                          chunk[j]);
+                r0 += (int64_t)grid_thw[3 * i] * grid_thw[3 * i + 1] * grid_thw[3 * i + 2];
+            }
+            if (cudaMemcpyAsync(table + base, chunk, sizeof(ItemDesc) * (size_t)m, cudaMemcpyHostToDevice, st) !=
+                cudaSuccess)
+                return PE_ERR_CUDA;
+        }
+        P.items_dev = table;
+    }
+    return run_frames(h, P, f_dt, out, out_dt, st);
 }
 
 pe_status pe_last_error(pe_handle *h) {
