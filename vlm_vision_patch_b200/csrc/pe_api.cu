@@ -203,15 +203,21 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
         return 1024 + r + epi_bytes + (size_t)(2 * nb + 2 * na + 5) * 8 + 16;
     };
     int nb = 6, na = (amode == kAModeFrames) ? 4 : 6;
-    while (total(nb, na) > (size_t)h->smem_optin) {
-        if (na > 3) --na;
-        else if (nb > 3) --nb;
-        else if (na > 2) --na;
-        else if (nb > 2) --nb;
-        else break;
+    if (amode == kAModeFrames) {
+        while (total(nb, na) > (size_t)h->smem_optin) {
+            if (na > 3) --na;
+            else if (nb > 3) --nb;
+            else if (na > 2) --na;
+            else if (nb > 2) --nb;
+            else break;
+        }
+    } else {
+        // A and weight stages share ring slots: equal depths
+        while (total(nb, na) > (size_t)h->smem_optin && nb > 2) { --nb; --na; }
     }
     P.nb = nb;
     P.na = na;
+    P.n_iss = std::min(amode == kAModeTma ? 6 : 3, std::min(nb, na));
     P.epi_offset = (int)((rings(nb, na) + 1023) / 1024 * 1024);
     return total(nb, na);
 }

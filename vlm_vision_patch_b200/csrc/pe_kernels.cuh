@@ -51,6 +51,7 @@ struct FwdParams {
     int32_t bn, n_tiles_n, num_tiles, num_ksteps;   // num_tiles counts pair tiles
     int32_t n_b_stages, n_a_stages;                 // per tile
     int32_t nb, na;                                 // ring depths
+    int32_t n_iss;                                  // TMA issuer warps, <= min(nb, na)
     int32_t a_stage_bytes;
     int32_t epi_offset;                             // staging area offset past the rings
     int32_t merge, n_items;
@@ -244,6 +245,135 @@ __device__ __forceinline__ void producer_release(const ProdCtx &X, int stage) {
     fence_proxy_async_smem();
     __syncwarp();
     if (X.lane == 0) mbar_arrive_cluster(X.full_a_leader + 8u * (uint32_t)stage);
+}
+
+// Pipelined frames producer for bf16 frames with tp = 2 and a compile-time p.
+// Every thread owns MAXIT (tile row, word) units.  For each stage it issues
+// 4-byte asynchronous copies of its raw pixel words straight into their final
+// positions of the A stage (one copy per unit and (c, i) pair when the row's
+// item is a single frame, since both temporal slices are that frame; two
+// otherwise), runs kDepth stages ahead, and then normalises its own words of
+// the oldest stage in place -- writing the duplicated slice at the same time --
+// before releasing the stage to the MMA.  No register holds data in flight.
+template <int PT>
+__device__ __forceinline__ void produce_frames_async(const FwdParams &P, const ProdCtx &X) {
+    constexpr int p = PT;
+    constexpr int ws = p / 2;
+    constexpr int units = kBM * ws;
+    constexpr int MAXIT = (PT + 3) / 4;
+    constexpr int kDepth = 2;
+    const int nci = P.C * p;             // (c, i) pairs; 4 per stage
+    const int nst = P.n_a_stages;
+
+    int rr[MAXIT], kw[MAXIT];
+    bool uok[MAXIT];
+#pragma unroll
+    for (int v = 0; v < MAXIT; ++v) {
+        const int u = X.pt + kProdThreads * v;
+        uok[v] = u < units;
+        int r = 0, jw = 0;
+        if (uok[v]) unit_to_row_word(u, ws, P.merge, r, jw);
+        rr[v] = r;
+        kw[v] = 2 * jw;
+    }
+    auto soff = [&](int q, int v) -> uint32_t {
+        const int k = q * p + kw[v];
+        return (uint32_t)(k >> 3) * 2048u + (uint32_t)rr[v] * 16u + (uint32_t)(k & 7) * 2u;
+    };
+    const uint32_t ring = smem_addr(X.a_ring);
+    const int tile0 = blockIdx.x >> 1, tstride = gridDim.x >> 1;
+    const int n_my_tiles = (P.num_tiles > tile0) ? (P.num_tiles - tile0 + tstride - 1) / tstride : 0;
+    const int total = n_my_tiles * nst;   // stages this CTA produces
+
+    // Row sources of the tile whose stages are being issued.
+    const char *src[MAXIT];
+    int32_t sW[MAXIT], sHW[MAXIT], sCHW[MAXIT];
+    uint32_t iss_rok = 0, iss_dup = 0;     // per-unit bits
+    uint32_t nrm_rok = 0, nrm_dup = 0;
+    auto tile_m0 = [&](int local_tile) -> int64_t {
+        const int tile = tile0 + local_tile * tstride;
+        return (int64_t)(tile / P.n_tiles_n) * (2 * kBM) + X.rank * kBM;
+    };
+    auto tile_bits = [&](int local_tile, bool fill_src, uint32_t &rok, uint32_t &dup) {
+        const int64_t m0 = tile_m0(local_tile);
+        rok = dup = 0;
+#pragma unroll
+        for (int v = 0; v < MAXIT; ++v) {
+            if (!(uok[v] && m0 + rr[v] < P.N)) continue;
+            const RowSrc s = locate_row(P, m0 + rr[v], 2);
+            rok |= 1u << v;
+            if (s.tmax == 0) dup |= 1u << v;
+            if (fill_src) {
+                src[v] = s.base + (int64_t)kw[v] * 2;
+                sW[v] = s.W;
+                sHW[v] = s.HW;
+                sCHW[v] = s.CHW;
+            }
+        }
+    };
+    auto issue = [&](int g) {   // issue the copies of global stage g (one commit group)
+        const int lt = g / nst, s = g - lt * nst;
+        if (s == 0) tile_bits(lt, true, iss_rok, iss_dup);
+        const int slot = g % P.na;
+        if (!mbar_wait(smem_addr(&X.empty_a[slot]), ((g / P.na) & 1) ^ 1, X.abort)) return false;
+        const uint32_t As = ring + (uint32_t)slot * (uint32_t)P.a_stage_bytes;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const int ci = 4 * s + qq;
+            if (ci >= nci) break;
+            const int c = ci / p, i = ci - c * p;
+#pragma unroll
+            for (int v = 0; v < MAXIT; ++v) {
+                if (!(iss_rok >> v & 1u)) continue;
+                const char *a = src[v] + ((int64_t)c * sHW[v] + (int64_t)i * sW[v]) * 2;
+                cp_async_4(As + soff(2 * qq, v), a);
+                if (!(iss_dup >> v & 1u)) cp_async_4(As + soff(2 * qq + 1, v), a + (int64_t)sCHW[v] * 2);
+            }
+        }
+        cp_async_commit();
+        return true;
+    };
+
+    bool ok = true;
+    for (int g = 0; g < kDepth && ok; ++g) {     // always kDepth groups ahead
+        if (g < total) ok = issue(g);
+        else cp_async_commit();
+    }
+    for (int g = 0; g < total && ok; ++g) {
+        if (g + kDepth < total) ok = issue(g + kDepth);
+        else cp_async_commit();                       // keep one group per stage
+        if (!ok) break;
+        cp_async_wait<kDepth>();                       // this thread's copies of stage g landed
+        const int lt = g / nst, s = g - lt * nst;
+        if (s == 0) tile_bits(lt, false, nrm_rok, nrm_dup);
+        const int slot = g % P.na;
+        const uint32_t As = ring + (uint32_t)slot * (uint32_t)P.a_stage_bytes;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const int ci = 4 * s + qq;
+            const bool live = ci < nci;
+            const int c = live ? ci / p : 0;
+            const NormConst nc = norm_const(P, c);
+#pragma unroll
+            for (int v = 0; v < MAXIT; ++v) {
+                if (!(nrm_rok >> v & 1u)) continue;
+                const uint32_t a0 = As + soff(2 * qq, v), a1 = As + soff(2 * qq + 1, v);
+                if (!live) {
+                    sts32(a0, 0u);
+                    sts32(a1, 0u);
+                } else if (nrm_dup >> v & 1u) {
+                    const uint32_t w = norm_pair_bf16(lds32(a0), nc);
+                    sts32(a0, w);
+                    sts32(a1, w);
+                } else if (nc.mode != kNormIdentity) {
+                    sts32(a0, norm_pair_bf16(lds32(a0), nc));
+                    sts32(a1, norm_pair_bf16(lds32(a1), nc));
+                }
+            }
+        }
+        producer_release(X, slot);
+    }
+    cp_async_wait<0>();
 }
 
 // Frames producer.  The frames path runs in the K order k' = ((c*p + i)*tp + t)*p + j
@@ -451,6 +581,133 @@ __device__ __forceinline__ void produce_patches(const FwdParams &P, const ProdCt
     }
 }
 
+// ------------------------------------------------------------- MMA issue
+
+// The single MMA-issuing thread must keep pace with the tensor core (one pair
+// MMA of 256 x 256 x 16 every 128 cycles), so the loop is unrolled over a
+// super-stage of lcm(KSA, 4) k-steps: waits, commits and descriptor offsets
+// sit at compile-time positions, descriptors advance by constant adds, and
+// nothing divides.  A stages hold KSA k-steps, weight stages 4.
+//   SEP_A_COMMIT  A stages have their own empty barriers (frames path);
+//                 otherwise A and weight stages coincide and share one.
+//   SEP_A_WAIT    A stages have their own full barriers (thread-produced A);
+//                 otherwise the A TMA bytes land on the weight stage's barrier.
+__host__ __device__ constexpr int lcm4(int a) { return (a % 4 == 0) ? a : (a % 2 == 0 ? 2 * a : 4 * a); }
+
+__device__ __forceinline__ uint64_t desc_with_lo(uint64_t d, uint32_t lo) {
+    return (d & 0xFFFFFFFF00000000ull) | lo;
+}
+
+template <int KSA, bool SEP_A_COMMIT, bool SEP_A_WAIT>
+__device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring, uint64_t *full_a,
+                                          uint64_t *empty_a, uint64_t *full_b, uint64_t *empty_b, uint64_t *tfull,
+                                          uint64_t *tempty, uint64_t *mma_done, uint32_t tmem_base,
+                                          volatile int *abort) {
+    constexpr int KSB = kBK / 16;
+    constexpr int L = lcm4(KSA);
+    constexpr uint16_t kPair = 0x3;
+    const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
+    // Descriptor templates (address field of slot 0); a k-step inside a stage
+    // adds 32 bytes (128-byte swizzle) or 4096 bytes (no-swizzle, 2 core-matrix columns).
+    const uint64_t a0 = (SEP_A_COMMIT) ? smem_desc(smem_addr(a_ring), 2048, 128, kLayoutInterleave)
+                        : (SEP_A_WAIT) ? smem_desc(smem_addr(a_ring), 2048, 128, kLayoutInterleave)
+                                       : smem_desc(smem_addr(a_ring), 16, 1024, kLayoutSw128);
+    const uint64_t b0 = smem_desc(smem_addr(b_ring), 16, 1024, kLayoutSw128);
+    constexpr uint32_t kAStep = (SEP_A_WAIT) ? (4096u >> 4) : (32u >> 4);
+    const uint32_t a_slot_step = (uint32_t)P.a_stage_bytes >> 4;
+    constexpr uint32_t kBSlotStep = (uint32_t)kBStageBytes >> 4;
+    const uint32_t a_lo0 = (uint32_t)a0, b_lo0 = (uint32_t)b0;
+    const int nk = P.num_ksteps;
+
+    int bs = 0, as = 0, acc = 0;
+    uint32_t bph = 0, aph = 0, accph = 0;
+    uint32_t a_lo = a_lo0, b_lo = b_lo0;
+    for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+        if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) return;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)acc * kMaxBN;
+        for (int ks0 = 0; ks0 < nk; ks0 += L) {
+#pragma unroll
+            for (int j = 0; j < L; ++j) {
+                const int ks = ks0 + j;
+                if (ks < nk) {
+                    if (j % KSB == 0) {
+                        if (!mbar_wait(smem_addr(&full_b[bs]), bph, abort)) return;
+                        b_lo = b_lo0 + (uint32_t)bs * kBSlotStep;
+                        if (!SEP_A_WAIT) a_lo = a_lo0 + (uint32_t)bs * a_slot_step;
+                    }
+                    if (SEP_A_WAIT && j % KSA == 0) {
+                        if (!mbar_wait(smem_addr(&full_a[as]), aph, abort)) return;
+                        a_lo = a_lo0 + (uint32_t)(SEP_A_COMMIT ? as : bs) * a_slot_step;
+                    }
+                    tc_fence_after();
+                    mma_bf16_pair(d_tmem, desc_with_lo(a0, a_lo + (uint32_t)(j % KSA) * kAStep),
+                                  desc_with_lo(b0, b_lo + (uint32_t)(j % KSB) * 2u), idesc, ks > 0 ? 1u : 0u);
+                    const bool last = ks == nk - 1;
+                    if (j % KSB == KSB - 1 || last) {
+                        mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
+                        if (++bs == P.nb) { bs = 0; bph ^= 1; }
+                    }
+                    if (SEP_A_COMMIT && (j % KSA == KSA - 1 || last)) {
+                        mma_commit_pair(smem_addr(&empty_a[as]), kPair);
+                        if (++as == P.na) { as = 0; aph ^= 1; }
+                    }
+                    if (SEP_A_WAIT && !SEP_A_COMMIT && (j % KSA == KSA - 1 || last)) {
+                        if (++as == P.na) { as = 0; aph ^= 1; }
+                    }
+                }
+            }
+        }
+        mma_commit_pair(smem_addr(&tfull[acc]), kPair);
+        if (++acc == 2) { acc = 0; accph ^= 1; }
+    }
+    mma_commit_pair(smem_addr(mma_done), 0x1);
+    mbar_wait(smem_addr(mma_done), 0, abort);
+}
+
+// Runtime-p frames path (p not 14 or 16): the same protocol, not unrolled.
+__device__ __noinline__ void mma_issue_generic(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring,
+                                               uint64_t *full_a, uint64_t *empty_a, uint64_t *full_b,
+                                               uint64_t *empty_b, uint64_t *tfull, uint64_t *tempty,
+                                               uint64_t *mma_done, uint32_t tmem_base, volatile int *abort) {
+    constexpr uint16_t kPair = 0x3;
+    const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
+    const int ks_a = P.P >> 1;
+    int bs = 0, as = 0, acc = 0;
+    uint32_t bph = 0, aph = 0, accph = 0;
+    for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+        if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) return;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)acc * kMaxBN;
+        int ka = 0, kbi = 0;
+        for (int ks = 0; ks < P.num_ksteps; ++ks) {
+            if (kbi == 0 && !mbar_wait(smem_addr(&full_b[bs]), bph, abort)) return;
+            if (ka == 0 && !mbar_wait(smem_addr(&full_a[as]), aph, abort)) return;
+            tc_fence_after();
+            const uint64_t adesc =
+                smem_desc(smem_addr(a_ring + (size_t)as * P.a_stage_bytes) + ka * 4096, 2048, 128, kLayoutInterleave);
+            const uint64_t bdesc = smem_desc(smem_addr(b_ring + (size_t)bs * kBStageBytes) + kbi * 32, 16, 1024,
+                                             kLayoutSw128);
+            mma_bf16_pair(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+            const bool last = (ks == P.num_ksteps - 1);
+            if (++kbi == kBK / 16 || last) {
+                mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
+                kbi = 0;
+                if (++bs == P.nb) { bs = 0; bph ^= 1; }
+            }
+            if (++ka == ks_a || last) {
+                mma_commit_pair(smem_addr(&empty_a[as]), kPair);
+                ka = 0;
+                if (++as == P.na) { as = 0; aph ^= 1; }
+            }
+        }
+        mma_commit_pair(smem_addr(&tfull[acc]), kPair);
+        if (++acc == 2) { acc = 0; accph ^= 1; }
+    }
+    mma_commit_pair(smem_addr(mma_done), 0x1);
+    mbar_wait(smem_addr(mma_done), 0, abort);
+}
+
 // ------------------------------------------------------------- the kernel
 
 template <int AMODE, int PT, bool F32IN>
@@ -477,7 +734,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    constexpr uint16_t kPair = 0x3;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P.nb; ++s) {
@@ -510,92 +766,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    if (warp == 0) {
-        // ---------------- TMA producer (both CTAs; bytes complete on the leader's barriers)
-        if (lane == 0) {
+    // Issuer warps: 0, 2, 3 and, when no warp produces A, 8, 9, 10.  At most
+    // P.n_iss of them issue, and P.n_iss never exceeds a ring depth: an issuer
+    // then can never lap a slot, so its parity waits cannot alias.
+    const int iss = (warp == 0) ? 0 : (warp == 2 || warp == 3) ? warp - 1
+                  : (AMODE == kAModeTma && warp >= 8 && warp < 11) ? warp - 5 : -1;
+    const int n_iss = P.n_iss;
+    if (iss >= 0) {
+        // ---------------- TMA issuers (both CTAs; bytes complete on the leader's barriers).
+        // Stage g of this CTA's sequence is issued by issuer g % n_iss: one
+        // thread's bulk copies are serviced one after another, so several
+        // issuing warps keep several copies in flight.
+        if (lane == 0 && iss < n_iss) {
             const uint64_t pol_w = l2_policy_evict_last();
             const uint64_t pol_x = l2_policy_evict_first();
             const uint32_t b_bytes = (uint32_t)(P.bn / 2) * kBK * 2;
             const uint32_t a_bytes = kBM * kBK * 2;
             const uint32_t fb0 = mapa_shared(smem_addr(&full_b[0]), 0);
-            const uint32_t fa0 = mapa_shared(smem_addr(&full_a[0]), 0);
-            int bs = 0, as = 0;
-            uint32_t bph = 0, aph = 0;
+            int g = 0;
             bool ok = true;
             for (int tile = blockIdx.x >> 1; tile < P.num_tiles && ok; tile += gridDim.x >> 1) {
                 const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
-                for (int kb = 0; kb < P.n_b_stages && ok; ++kb) {
-                    if (AMODE == kAModeTma) {
-                        if (!mbar_wait(smem_addr(&empty_a[as]), aph ^ 1, abort)) { ok = false; break; }
-                        if (leader) mbar_arrive_expect_tx(smem_addr(&full_a[as]), 2 * a_bytes);
-                        tma_load_2d_pair(smem_addr(a_ring + (size_t)as * P.a_stage_bytes), &tmap_x, fa0 + 8u * as,
+                for (int kb = 0; kb < P.n_b_stages && ok; ++kb, ++g) {
+                    if (g % n_iss != iss) continue;
+                    // In the TMA-fed path A and weight share ring slot and barriers.
+                    const int bs = g % P.nb;
+                    if (!mbar_wait(smem_addr(&empty_b[bs]), ((g / P.nb) & 1) ^ 1, abort)) { ok = false; break; }
+                    if (leader)
+                        mbar_arrive_expect_tx(smem_addr(&full_b[bs]),
+                                              2 * (b_bytes + (AMODE == kAModeTma ? a_bytes : 0u)));
+                    if (AMODE == kAModeTma)
+                        tma_load_2d_pair(smem_addr(a_ring + (size_t)bs * P.a_stage_bytes), &tmap_x, fb0 + 8u * bs,
                                          kb * kBK, m_blk * (2 * kBM) + (int)rank * kBM, pol_x);
-                        if (++as == P.na) { as = 0; aph ^= 1; }
-                    }
-                    if (!mbar_wait(smem_addr(&empty_b[bs]), bph ^ 1, abort)) { ok = false; break; }
-                    if (leader) mbar_arrive_expect_tx(smem_addr(&full_b[bs]), 2 * b_bytes);
                     tma_load_2d_pair(smem_addr(b_ring + (size_t)bs * kBStageBytes), &tmap_w, fb0 + 8u * bs,
                                      kb * kBK, n_blk * P.bn + (int)rank * (P.bn / 2), pol_w);
-                    if (++bs == P.nb) { bs = 0; bph ^= 1; }
                 }
-            }
-            // Drain: the MMA signals every consumed stage back on our empty
-            // barriers; waiting for the last signal of each slot means every
-            // load this CTA issued has landed and been read.
-            for (int s = 0; s < P.nb; ++s) {
-                const int slot = (bs + s) % P.nb;
-                mbar_wait(smem_addr(&empty_b[slot]), (slot < bs) ? bph : (bph ^ 1), abort);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (leader CTA only)
         if (leader && lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
-            const int ks_a = (AMODE == kAModeFrames) ? (P.P >> 1) : (kBK / 16);
-            int bs = 0, as = 0, acc = 0;
-            uint32_t bph = 0, aph = 0, accph = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x >> 1; tile < P.num_tiles && ok; tile += gridDim.x >> 1) {
-                if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)acc * kMaxBN;
-                int ka = 0, kbi = 0;  // k-step inside the current A / B stage
-                for (int ks = 0; ks < P.num_ksteps; ++ks) {
-                    if (kbi == 0) {
-                        if (!mbar_wait(smem_addr(&full_b[bs]), bph, abort)) { ok = false; break; }
-                        tc_fence_after();
-                    }
-                    if (ka == 0) {
-                        if (!mbar_wait(smem_addr(&full_a[as]), aph, abort)) { ok = false; break; }
-                        tc_fence_after();
-                    }
-                    const uint32_t a_base = smem_addr(a_ring + (size_t)as * P.a_stage_bytes);
-                    const uint32_t b_base = smem_addr(b_ring + (size_t)bs * kBStageBytes);
-                    uint64_t adesc;
-                    if (AMODE == kAModeTma)
-                        adesc = smem_desc(a_base + ka * 32, 16, 1024, kLayoutSw128);
-                    else
-                        adesc = smem_desc(a_base + ka * 4096, 2048, 128, kLayoutInterleave);
-                    const uint64_t bdesc = smem_desc(b_base + kbi * 32, 16, 1024, kLayoutSw128);
-                    mma_bf16_pair(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
-                    const bool last = (ks == P.num_ksteps - 1);
-                    if (++kbi == kBK / 16 || last) {
-                        mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
-                        kbi = 0;
-                        if (++bs == P.nb) { bs = 0; bph ^= 1; }
-                    }
-                    if (++ka == ks_a || last) {
-                        mma_commit_pair(smem_addr(&empty_a[as]), kPair);
-                        ka = 0;
-                        if (++as == P.na) { as = 0; aph ^= 1; }
-                    }
-                }
-                if (!ok) break;
-                mma_commit_pair(smem_addr(&tfull[acc]), kPair);
-                if (++acc == 2) { acc = 0; accph ^= 1; }
-            }
-            mma_commit_pair(smem_addr(mma_done), 0x1);
-            mbar_wait(smem_addr(mma_done), 0, abort);
+            constexpr int KSA = (AMODE == kAModeFrames) ? (PT ? PT / 2 : 0) : 4;
+            if constexpr (KSA > 0)
+                mma_issue<KSA, AMODE == kAModeFrames, AMODE != kAModeTma>(P, a_ring, b_ring, full_a, empty_a, full_b,
+                                                                          empty_b, tfull, tempty, mma_done, tmem_base,
+                                                                          abort);
+            else
+                mma_issue_generic(P, a_ring, b_ring, full_a, empty_a, full_b, empty_b, tfull, tempty, mma_done,
+                                  tmem_base, abort);
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         // ---------------- epilogue (both CTAs)
@@ -658,18 +876,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
-    } else if (warp >= 8) {
+    } else if (warp >= 8 && AMODE != kAModeTma) {
         // ---------------- A producers (both CTAs)
         ProdCtx X;
         X.a_ring = a_ring;
-        X.empty_a = empty_a;
+        X.empty_a = (AMODE == kAModePatchThreads) ? empty_b : empty_a;   // stages coincide
         X.full_a_leader = mapa_shared(smem_addr(&full_a[0]), 0);
         X.abort = abort;
         X.pt = threadIdx.x - 256;
         X.lane = lane;
         X.rank = rank;
-        if constexpr (AMODE == kAModeFrames)
+        if constexpr (AMODE == kAModeFrames && PT != 0 && !F32IN) {
+            if (P.TP == 2) produce_frames_async<PT>(P, X);
+            else produce_frames<PT, F32IN>(P, X);
+        } else if constexpr (AMODE == kAModeFrames) {
             produce_frames<PT, F32IN>(P, X);
+        }
         else if constexpr (AMODE == kAModePatchThreads)
             produce_patches(P, X);
     }
