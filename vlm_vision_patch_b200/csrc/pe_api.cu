@@ -132,13 +132,13 @@ int choose_bn(int64_t N, int E, int num_pairs, bool gather_fed) {
     return 64;
 }
 
-template <int AMODE, int PT, bool F32IN>
+template <int AMODE, int PT, bool F32IN, int NORM = 2, bool DUPALL = false>
 cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensorMap &tx, const CUtensorMap &to,
                        size_t smem, int grid, cudaStream_t st) {
-    auto kern = pe_fwd_kernel<AMODE, PT, F32IN>;
+    auto kern = pe_fwd_kernel<AMODE, PT, F32IN, NORM, DUPALL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, st>>>(tw, tx, to, P);
+    kern<<<grid, threads_for(AMODE), smem, st>>>(tw, tx, to, P);
     return cudaGetLastError();
 }
 
@@ -196,7 +196,7 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
         P.a_stage_bytes = kBM * kBK * 2;
         P.n_a_stages = P.n_b_stages;
     }
-    const size_t epi_bytes = (size_t)8 * 32 * 32 * (P.out_f32 ? 4 : 2);
+    const size_t epi_bytes = (size_t)4 * 8192;   // staging ring of the 4 epilogue warps
     auto rings = [&](int nb, int na) { return (size_t)nb * kBStageBytes + (size_t)na * P.a_stage_bytes; };
     auto total = [&](int nb, int na) {
         const size_t r = (rings(nb, na) + 1023) / 1024 * 1024;
@@ -205,7 +205,8 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
     int nb = 6, na = (amode == kAModeFrames) ? 4 : 6;
     if (amode == kAModeFrames) {
         while (total(nb, na) > (size_t)h->smem_optin) {
-            if (na > 3) --na;
+            if (nb > 5) --nb;
+            else if (na > 3) --na;
             else if (nb > 3) --nb;
             else if (na > 2) --na;
             else if (nb > 2) --nb;
@@ -217,7 +218,7 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
     }
     P.nb = nb;
     P.na = na;
-    P.n_iss = std::min(amode == kAModeTma ? 6 : 3, std::min(nb, na));
+    P.n_iss = std::min(amode == kAModeTma ? 5 : 3, std::min(nb, na));
     P.epi_offset = (int)((rings(nb, na) + 1023) / 1024 * 1024);
     return total(nb, na);
 }
@@ -259,10 +260,12 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
     P.n_items = n;
     std::vector<ItemDesc> items((size_t)n);
     int64_t row0 = 0;
+    P.all_t1 = 1;
     for (int i = 0; i < n; ++i) {
         const pe_status s = make_item(h, frames[i], THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid + 3 * i,
                                       merge, row0, items[(size_t)i]);
         if (s != PE_OK) return s;
+        P.all_t1 = P.all_t1 && THW[3 * i] == 1;
         row0 += (int64_t)grid[3 * i] * grid[3 * i + 1] * grid[3 * i + 2];
     }
     P.N = row0;
@@ -310,13 +313,27 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
     if (!make_out_tmap(&to, out, P.out_f32, P.N, P.E)) return PE_ERR_CUDA;
     const CUtensorMap &tw = h->tmap_wf[bn_index(P.bn)];
     const bool f32 = f_dt == PE_F32;
+    // One normalisation mode for every channel lets the producer drop the
+    // per-word mode test (1: all scaled; 2: anything else, decided per word),
+    // and frames that are all single images (T = 1, tp = 2) need only one
+    // temporal slice per (c, i).
+    bool all_scaled = true;
+    for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
+    bool dupall = h->tp == 2;
+    dupall = dupall && P.all_t1;
     cudaError_t e;
-    if (h->p == 14)
-        e = f32 ? launch_fwd<kAModeFrames, 14, true>(tw, P, dummy, to, smem, grid, st)
-                : launch_fwd<kAModeFrames, 14, false>(tw, P, dummy, to, smem, grid, st);
+    if (!f32 && (h->p == 14 || h->p == 16)) {
+#define PE_LAUNCH_FRAMES(PP)                                                                                  \
+    (all_scaled ? (dupall ? launch_fwd<kAModeFrames, PP, false, 1, true>(tw, P, dummy, to, smem, grid, st)       \
+                          : launch_fwd<kAModeFrames, PP, false, 1, false>(tw, P, dummy, to, smem, grid, st))     \
+                : (dupall ? launch_fwd<kAModeFrames, PP, false, 2, true>(tw, P, dummy, to, smem, grid, st)       \
+                          : launch_fwd<kAModeFrames, PP, false, 2, false>(tw, P, dummy, to, smem, grid, st)))
+        e = (h->p == 14) ? PE_LAUNCH_FRAMES(14) : PE_LAUNCH_FRAMES(16);
+#undef PE_LAUNCH_FRAMES
+    } else if (h->p == 14)
+        e = launch_fwd<kAModeFrames, 14, true>(tw, P, dummy, to, smem, grid, st);
     else if (h->p == 16)
-        e = f32 ? launch_fwd<kAModeFrames, 16, true>(tw, P, dummy, to, smem, grid, st)
-                : launch_fwd<kAModeFrames, 16, false>(tw, P, dummy, to, smem, grid, st);
+        e = launch_fwd<kAModeFrames, 16, true>(tw, P, dummy, to, smem, grid, st);
     else
         e = f32 ? launch_fwd<kAModeFrames, 0, true>(tw, P, dummy, to, smem, grid, st)
                 : launch_fwd<kAModeFrames, 0, false>(tw, P, dummy, to, smem, grid, st);
@@ -569,7 +586,9 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
     P.n_items = n;
     // Validate every item before anything is copied or launched.
     int64_t row0 = 0;
+    P.all_t1 = 1;
     for (int i = 0; i < n; ++i) {
+        P.all_t1 = P.all_t1 && THW[3 * i] == 1;
         ItemDesc d;
         const pe_status s = make_item(h, frames[i], THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid_thw + 3 * i,
                                       merge, row0, d);

@@ -28,12 +28,14 @@
 
 namespace pe {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;       // 20 warps (A produced by threads)
+constexpr int kThreadsTma = 320;    // 10 warps (A fetched by TMA)
+__host__ __device__ constexpr int threads_for(int amode) { return amode == 0 ? kThreadsTma : kThreads; }
 constexpr int kBM = 128;           // rows per CTA (pair tile: 256 rows)
 constexpr int kMaxBN = 256;        // largest pair-MMA N
 constexpr int kBK = 64;            // weight K per TMA stage (one 128-byte swizzle row)
-constexpr int kProdThreads = 256;  // warps 8..15
-constexpr int kProdWarps = 8;
+constexpr int kProdThreads = 384;  // warps 8..19
+constexpr int kProdWarps = 12;
 constexpr int kEpiWarp0 = 4;
 constexpr int kBStageBytes = (kMaxBN / 2) * kBK * 2;   // 16 KB: this CTA's half of the weight tile
 
@@ -55,6 +57,7 @@ struct FwdParams {
     int32_t a_stage_bytes;
     int32_t epi_offset;                             // staging area offset past the rings
     int32_t merge, n_items;
+    int32_t all_t1;                   // every item is a single frame (host-side kernel choice)
     int64_t N;
     const ItemDesc *items_dev;        // table in device memory when n_items > PE_INLINE_ITEMS
     ItemDesc items[PE_INLINE_ITEMS];
@@ -247,21 +250,46 @@ __device__ __forceinline__ void producer_release(const ProdCtx &X, int stage) {
     if (X.lane == 0) mbar_arrive_cluster(X.full_a_leader + 8u * (uint32_t)stage);
 }
 
+// Normalisation of one raw bf16 x 2 word for a channel whose mode the kernel
+// knows at compile time: NORM 0 = identity (the word itself), 1 = the scaled
+// correctly rounded quotient, 2 = decided at run time per channel.
+template <int NORM>
+__device__ __forceinline__ uint32_t norm_word(uint32_t w, const NormConst &n) {
+    if constexpr (NORM == 0) {
+        return w;
+    } else if constexpr (NORM == 1) {
+        uint64_t X, M, R, NS, SC, D, Q0, Er, Q;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(bf16lo_to_f32(w)), "f"(bf16hi_to_f32(w)));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(M) : "f"(n.mean));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(R) : "f"(n.rcp_s));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(NS) : "f"(n.nstd_s));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(SC) : "f"(n.scale));
+        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(X), "l"(M));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q0) : "l"(D), "l"(R));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Er) : "l"(Q0), "l"(NS), "l"(D));
+        asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Q) : "l"(Er), "l"(R), "l"(Q0));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q) : "l"(Q), "l"(SC));
+        float q0, q1;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(q0), "=f"(q1) : "l"(Q));
+        return pack_bf16x2(q0, q1);
+    } else {
+        return norm_pair_bf16(w, n);
+    }
+}
+
 // Pipelined frames producer for bf16 frames with tp = 2 and a compile-time p.
-// Every thread owns MAXIT (tile row, word) units.  For each stage it issues
-// 4-byte asynchronous copies of its raw pixel words straight into their final
-// positions of the A stage (one copy per unit and (c, i) pair when the row's
-// item is a single frame, since both temporal slices are that frame; two
-// otherwise), runs kDepth stages ahead, and then normalises its own words of
-// the oldest stage in place -- writing the duplicated slice at the same time --
-// before releasing the stage to the MMA.  No register holds data in flight.
-template <int PT>
-__device__ __forceinline__ void produce_frames_async(const FwdParams &P, const ProdCtx &X) {
+// Each producer thread owns MAXIT (tile row, word) units.  The raw words of
+// stage g+1 are loaded (coalesced 32-bit loads into registers) before stage g
+// is normalised and stored, so one stage of loads is always in flight behind
+// the arithmetic.  A row whose item is a single frame loads its words once and
+// stores the normalised word to both temporal slices.
+template <int PT, int NORM, bool DUPALL>
+__device__ __forceinline__ void produce_frames_reg(const FwdParams &P, const ProdCtx &X) {
+    constexpr int NT = DUPALL ? 1 : 2;    // temporal slices held per (c, i)
     constexpr int p = PT;
     constexpr int ws = p / 2;
     constexpr int units = kBM * ws;
-    constexpr int MAXIT = (PT + 3) / 4;
-    constexpr int kDepth = 2;
+    constexpr int MAXIT = (units + kProdThreads - 1) / kProdThreads;
     const int nci = P.C * p;             // (c, i) pairs; 4 per stage
     const int nst = P.n_a_stages;
 
@@ -283,97 +311,95 @@ __device__ __forceinline__ void produce_frames_async(const FwdParams &P, const P
     const uint32_t ring = smem_addr(X.a_ring);
     const int tile0 = blockIdx.x >> 1, tstride = gridDim.x >> 1;
     const int n_my_tiles = (P.num_tiles > tile0) ? (P.num_tiles - tile0 + tstride - 1) / tstride : 0;
-    const int total = n_my_tiles * nst;   // stages this CTA produces
+    const int total = n_my_tiles * nst;
 
-    // Row sources of the tile whose stages are being issued.
+    // load side: row sources of the tile being loaded
     const char *src[MAXIT];
-    int32_t sW[MAXIT], sHW[MAXIT], sCHW[MAXIT];
-    uint32_t iss_rok = 0, iss_dup = 0;     // per-unit bits
-    uint32_t nrm_rok = 0, nrm_dup = 0;
-    auto tile_m0 = [&](int local_tile) -> int64_t {
-        const int tile = tile0 + local_tile * tstride;
-        return (int64_t)(tile / P.n_tiles_n) * (2 * kBM) + X.rank * kBM;
-    };
-    auto tile_bits = [&](int local_tile, bool fill_src, uint32_t &rok, uint32_t &dup) {
-        const int64_t m0 = tile_m0(local_tile);
-        rok = dup = 0;
+    int32_t sW[MAXIT], sHW[MAXIT], sT1[MAXIT];   // sT1: byte offset of the t = 1 slice (0: same frame)
+    int ld_lt = 0, ld_s = 0;
+    uint32_t rokb[2] = {0u, 0u}, dupb[2] = {0u, 0u};
+    uint32_t raw[2][4][NT][MAXIT];
+    // normalise side
+    int nm_s = 0;
+
+    auto load_stage = [&](const int b) {    // loads the next stage of the load side into buffer b
+        if (ld_s == 0) {
+            const int tile = tile0 + ld_lt * tstride;
+            const int64_t m0 = (int64_t)(tile / P.n_tiles_n) * (2 * kBM) + X.rank * kBM;
+            uint32_t rk = 0, dp = 0;
 #pragma unroll
-        for (int v = 0; v < MAXIT; ++v) {
-            if (!(uok[v] && m0 + rr[v] < P.N)) continue;
-            const RowSrc s = locate_row(P, m0 + rr[v], 2);
-            rok |= 1u << v;
-            if (s.tmax == 0) dup |= 1u << v;
-            if (fill_src) {
-                src[v] = s.base + (int64_t)kw[v] * 2;
-                sW[v] = s.W;
-                sHW[v] = s.HW;
-                sCHW[v] = s.CHW;
+            for (int v = 0; v < MAXIT; ++v) {
+                src[v] = nullptr;
+                sW[v] = sHW[v] = sT1[v] = 0;
+                if (!(uok[v] && m0 + rr[v] < P.N)) continue;
+                const RowSrc rs = locate_row(P, m0 + rr[v], 2);
+                src[v] = rs.base + (int64_t)kw[v] * 2;
+                sW[v] = rs.W * 2;
+                sHW[v] = rs.HW * 2;
+                sT1[v] = rs.tmax > 0 ? rs.CHW * 2 : 0;
+                rk |= 1u << v;
+                if (rs.tmax == 0) dp |= 1u << v;
+            }
+            rokb[b] = rk;
+            dupb[b] = dp;
+        } else {
+            rokb[b] = rokb[b ^ 1];
+            dupb[b] = dupb[b ^ 1];
+        }
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const int ci = 4 * ld_s + qq;
+            const int c = ci / p, i = ci - (ci / p) * p;
+#pragma unroll
+            for (int v = 0; v < MAXIT; ++v) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t) raw[b][qq][t][v] = 0u;
+                if (ci < nci && (rokb[b] >> v & 1u)) {
+                    const char *a = src[v] + (int64_t)c * sHW[v] + (int64_t)i * sW[v];
+                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][0][v]) : "l"(a));
+                    if constexpr (!DUPALL) {
+                        if (sT1[v] != 0)
+                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][NT - 1][v]) : "l"(a + sT1[v]));
+                    }
+                }
             }
         }
+        if (++ld_s == nst) { ld_s = 0; ++ld_lt; }
     };
-    auto issue = [&](int g) {   // issue the copies of global stage g (one commit group)
-        const int lt = g / nst, s = g - lt * nst;
-        if (s == 0) tile_bits(lt, true, iss_rok, iss_dup);
+    auto store_stage = [&](const int g, const int b) -> bool {   // normalise buffer b into stage g's slot
         const int slot = g % P.na;
         if (!mbar_wait(smem_addr(&X.empty_a[slot]), ((g / P.na) & 1) ^ 1, X.abort)) return false;
         const uint32_t As = ring + (uint32_t)slot * (uint32_t)P.a_stage_bytes;
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
-            const int ci = 4 * s + qq;
-            if (ci >= nci) break;
-            const int c = ci / p, i = ci - c * p;
-#pragma unroll
-            for (int v = 0; v < MAXIT; ++v) {
-                if (!(iss_rok >> v & 1u)) continue;
-                const char *a = src[v] + ((int64_t)c * sHW[v] + (int64_t)i * sW[v]) * 2;
-                cp_async_4(As + soff(2 * qq, v), a);
-                if (!(iss_dup >> v & 1u)) cp_async_4(As + soff(2 * qq + 1, v), a + (int64_t)sCHW[v] * 2);
-            }
-        }
-        cp_async_commit();
-        return true;
-    };
-
-    bool ok = true;
-    for (int g = 0; g < kDepth && ok; ++g) {     // always kDepth groups ahead
-        if (g < total) ok = issue(g);
-        else cp_async_commit();
-    }
-    for (int g = 0; g < total && ok; ++g) {
-        if (g + kDepth < total) ok = issue(g + kDepth);
-        else cp_async_commit();                       // keep one group per stage
-        if (!ok) break;
-        cp_async_wait<kDepth>();                       // this thread's copies of stage g landed
-        const int lt = g / nst, s = g - lt * nst;
-        if (s == 0) tile_bits(lt, false, nrm_rok, nrm_dup);
-        const int slot = g % P.na;
-        const uint32_t As = ring + (uint32_t)slot * (uint32_t)P.a_stage_bytes;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const int ci = 4 * s + qq;
+            const int ci = 4 * nm_s + qq;
             const bool live = ci < nci;
-            const int c = live ? ci / p : 0;
-            const NormConst nc = norm_const(P, c);
+            const NormConst nc = norm_const(P, live ? ci / p : 0);
 #pragma unroll
             for (int v = 0; v < MAXIT; ++v) {
-                if (!(nrm_rok >> v & 1u)) continue;
-                const uint32_t a0 = As + soff(2 * qq, v), a1 = As + soff(2 * qq + 1, v);
-                if (!live) {
-                    sts32(a0, 0u);
-                    sts32(a1, 0u);
-                } else if (nrm_dup >> v & 1u) {
-                    const uint32_t w = norm_pair_bf16(lds32(a0), nc);
-                    sts32(a0, w);
-                    sts32(a1, w);
-                } else if (nc.mode != kNormIdentity) {
-                    sts32(a0, norm_pair_bf16(lds32(a0), nc));
-                    sts32(a1, norm_pair_bf16(lds32(a1), nc));
+                if (!(rokb[b] >> v & 1u)) continue;
+                uint32_t w0 = 0u, w1 = 0u;
+                if (live) {
+                    w0 = norm_word<NORM>(raw[b][qq][0][v], nc);
+                    w1 = (DUPALL || (dupb[b] >> v & 1u)) ? w0 : norm_word<NORM>(raw[b][qq][NT - 1][v], nc);
                 }
+                sts32(As + soff(2 * qq, v), w0);
+                sts32(As + soff(2 * qq + 1, v), w1);
             }
         }
         producer_release(X, slot);
+        if (++nm_s == nst) nm_s = 0;
+        return true;
+    };
+
+    if (total > 0) load_stage(0);
+    for (int g = 0; g < total; g += 2) {
+        if (g + 1 < total) load_stage(1);
+        if (!store_stage(g, 0)) return;
+        if (g + 1 >= total) break;
+        if (g + 2 < total) load_stage(0);
+        if (!store_stage(g + 1, 1)) return;
     }
-    cp_async_wait<0>();
 }
 
 // Frames producer.  The frames path runs in the K order k' = ((c*p + i)*tp + t)*p + j
@@ -386,7 +412,7 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, const ProdCtx
     const int p = PT ? PT : P.P;
     const int ws = p >> 1;
     const int units = kBM * ws;
-    constexpr int MAXIT = PT ? (PT + 3) / 4 : (PE_MAX_PATCH + 3) / 4;
+    constexpr int MAXIT = (kBM * ((PT ? PT : PE_MAX_PATCH) / 2) + kProdThreads - 1) / kProdThreads;
     constexpr int esize = F32IN ? 4 : 2;
     const int TP = P.TP;
     const int nseg = P.C * TP * p;
@@ -538,8 +564,9 @@ __device__ __forceinline__ void produce_patches(const FwdParams &P, const ProdCt
             if (!mbar_wait(smem_addr(&X.empty_a[stage]), phase ^ 1, X.abort)) return;
             uint8_t *As = X.a_ring + (size_t)stage * P.a_stage_bytes;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const int u = X.pt + kProdThreads * v;  // 0..1023
+            for (int v = 0; v < (kBM * 8 + kProdThreads - 1) / kProdThreads; ++v) {
+                const int u = X.pt + kProdThreads * v;  // (row, 8-column group), 1024 of them
+                if (u >= kBM * 8) break;
                 const int r = u >> 3, kg = u & 7;
                 const int64_t R = m0 + r;
                 const int k0 = s * kBK + kg * 8;
@@ -710,8 +737,8 @@ __device__ __noinline__ void mma_issue_generic(const FwdParams &P, uint8_t *a_ri
 
 // ------------------------------------------------------------- the kernel
 
-template <int AMODE, int PT, bool F32IN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int AMODE, int PT, bool F32IN, int NORM, bool DUPALL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 1)
     pe_fwd_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                   const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ FwdParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -719,8 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *b_ring = smem;
     uint8_t *a_ring = b_ring + (size_t)P.nb * kBStageBytes;
     uint8_t *epi = smem + P.epi_offset;
-    const int epi_buf_bytes = 32 * 32 * (P.out_f32 ? 4 : 2);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(epi + 8 * epi_buf_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(epi + 4 * 8192);   // 8 KB staging per epilogue warp
     uint64_t *full_b = bars;
     uint64_t *empty_b = full_b + P.nb;
     uint64_t *full_a = empty_b + P.nb;
@@ -766,11 +792,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    // Issuer warps: 0, 2, 3 and, when no warp produces A, 8, 9, 10.  At most
+    // Issuer warps: 0, 2, 3 and, when no warp produces A, 8 and 9.  At most
     // P.n_iss of them issue, and P.n_iss never exceeds a ring depth: an issuer
     // then can never lap a slot, so its parity waits cannot alias.
     const int iss = (warp == 0) ? 0 : (warp == 2 || warp == 3) ? warp - 1
-                  : (AMODE == kAModeTma && warp >= 8 && warp < 11) ? warp - 5 : -1;
+                  : (AMODE == kAModeTma && warp >= 8 && warp < 10) ? warp - 5 : -1;
     const int n_iss = P.n_iss;
     if (iss >= 0) {
         // ---------------- TMA issuers (both CTAs; bytes complete on the leader's barriers).
@@ -817,57 +843,80 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         // ---------------- epilogue (both CTAs)
+        // Each warp drains its 32 TMEM lanes in 32-column chunks, loading chunk
+        // c+1 from TMEM while chunk c is converted, and hands each converted
+        // 32 x 32 box to a TMA store through a ring of staging buffers.
         const int wq = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t tempty0 = mapa_shared(smem_addr(&tempty[0]), 0);
-        uint8_t *stage_buf = epi + (size_t)wq * 2 * epi_buf_bytes;
+        const int nbufs = P.out_f32 ? 2 : 4;
+        uint8_t *stage_buf = epi + (size_t)wq * 8192;
+        const int nch = P.bn / 32;   // 2, 4 or 8
         int acc = 0, nbuf = 0;
         uint32_t accph = 0;
+        auto emit = [&](const uint32_t (&v)[32], int cc, int64_t row0, int n_blk) {
+            const int col0 = n_blk * P.bn + cc * 32;
+            if (row0 >= P.N || col0 >= P.E) return;   // whole box outside: nothing to store
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+            if (P.bias) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
+            }
+            // the buffer must be free of the store issued nbufs chunks ago
+            if (lane == 0) {
+                if (nbufs == 4) bulk_wait_read<3>(); else bulk_wait_read<1>();
+            }
+            __syncwarp();
+            uint8_t *buf = stage_buf + (size_t)nbuf * (P.out_f32 ? 4096 : 2048);
+            if (P.out_f32) {
+                // 128-byte rows, 128-byte swizzle: chunk c of row r at (c ^ (r & 7))
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                        make_float4(f[4 * c], f[4 * c + 1], f[4 * c + 2], f[4 * c + 3]);
+            } else {
+                // 64-byte rows, 64-byte swizzle: chunk c of row r at (c ^ ((r >> 1) & 3))
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                        make_uint4(pack_bf16x2(f[8 * c], f[8 * c + 1]), pack_bf16x2(f[8 * c + 2], f[8 * c + 3]),
+                                   pack_bf16x2(f[8 * c + 4], f[8 * c + 5]), pack_bf16x2(f[8 * c + 6], f[8 * c + 7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(&tmap_out, smem_addr(buf), col0, (int32_t)row0);
+                bulk_commit();
+            }
+            if (++nbuf == nbufs) nbuf = 0;
+        };
         for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
             const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
             if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
             tc_fence_after();
             const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
-            for (int cc = 0; cc < P.bn / 32; ++cc) {
-                uint32_t v[32];
-                const uint32_t taddr = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN + cc * 32);
-                tmem_ld_32x32b_x32(taddr, v);
-                tmem_ld_wait();
-                const int col0 = n_blk * P.bn + cc * 32;
-                if (row0 >= P.N || col0 >= P.E) continue;   // whole box outside: nothing to store
-                float f[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
-                if (P.bias) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
+            const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
+            if constexpr (AMODE == kAModeTma) {
+                // registers to spare: the next chunk's TMEM load overlaps this chunk's work
+                uint32_t va[32], vb[32];
+                tmem_ld_32x32b_x32(tbase, va);
+                for (int cc = 0; cc < nch; cc += 2) {
+                    tmem_ld_wait();
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 1) * 32, vb);
+                    emit(va, cc, row0, n_blk);
+                    tmem_ld_wait();
+                    if (cc + 2 < nch) tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 2) * 32, va);
+                    emit(vb, cc + 1, row0, n_blk);
                 }
-                // this warp's staging buffer must be free of the store issued two chunks ago
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-                uint8_t *buf = stage_buf + (size_t)nbuf * epi_buf_bytes;
-                if (P.out_f32) {
-                    // 128-byte rows, 128-byte swizzle: chunk c of row r at (c ^ (r & 7))
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<float4 *>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                            make_float4(f[4 * c], f[4 * c + 1], f[4 * c + 2], f[4 * c + 3]);
-                } else {
-                    // 64-byte rows, 64-byte swizzle: chunk c of row r at (c ^ ((r >> 1) & 3))
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
-                            make_uint4(pack_bf16x2(f[8 * c], f[8 * c + 1]), pack_bf16x2(f[8 * c + 2], f[8 * c + 3]),
-                                       pack_bf16x2(f[8 * c + 4], f[8 * c + 5]),
-                                       pack_bf16x2(f[8 * c + 6], f[8 * c + 7]));
+            } else {
+                uint32_t va[32];
+                for (int cc = 0; cc < nch; ++cc) {
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)cc * 32, va);
+                    tmem_ld_wait();
+                    emit(va, cc, row0, n_blk);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmap_out, smem_addr(buf), col0, (int32_t)row0);
-                    bulk_commit();
-                }
-                nbuf ^= 1;
             }
             tc_fence_before();
             __syncwarp();
@@ -887,7 +936,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         X.lane = lane;
         X.rank = rank;
         if constexpr (AMODE == kAModeFrames && PT != 0 && !F32IN) {
-            if (P.TP == 2) produce_frames_async<PT>(P, X);
+            if (P.TP == 2) produce_frames_reg<PT, NORM, DUPALL>(P, X);
             else produce_frames<PT, F32IN>(P, X);
         } else if constexpr (AMODE == kAModeFrames) {
             produce_frames<PT, F32IN>(P, X);
