@@ -30,10 +30,10 @@
  *   - Dense row-major layouts only.  Device pointers must be 16-byte aligned.
  *   - No C++ exception crosses this interface.  A CUDA error maps to
  *     PE_ERR_CUDA.
- *   - A handle may be used by concurrent forward calls on different streams,
- *     except that grouped calls with more than PE_INLINE_ITEMS items upload
- *     their item table into the handle's workspace and must therefore be
- *     serialised (same stream).  pe_set_weight / pe_set_norm must not run
+ *   - Forward calls that use a handle's workspace must be serialised on one
+ *     stream: grouped calls with more than PE_INLINE_ITEMS items (item table),
+ *     and frames calls large enough to take the staged path (see
+ *     pe_forward_frames).  pe_set_weight / pe_set_norm must not run
  *     concurrently with anything else on the same handle.
  */
 #ifndef PE_H_
@@ -136,9 +136,14 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
  *              README §3.2 PatchMerger and §4.1; Qwen2.5VL语言模型 MRoPE example:
  *              merged grid row-major, h outer).  gh and gw must be multiples of m.
  *   out      : dev [gt*gh*gw, E] of dtype out_dt.
- * Requires p even and p <= PE_MAX_PATCH.  The [N, K] patch matrix is never
- * written to memory.  Errors: as pe_forward_patches plus PE_ERR_SHAPE,
- * PE_ERR_UNSUPPORTED.
+ * Requires p even and p <= PE_MAX_PATCH.  Two execution paths give identical
+ * results: the fused path (one kernel; the normalised [N, K] patch matrix only
+ * ever exists tile by tile in shared memory) and, for bf16 frames with tp = 2,
+ * p in {14, 16} and at least 8192 patches, the staged path (a prepare kernel
+ * writes the normalised patch matrix once into the handle's grow-only
+ * workspace, then the TMA-fed contraction reads it back).  The environment
+ * variable PE_FRAMES_PATH=fused|staged overrides the choice.
+ * Errors: as pe_forward_patches plus PE_ERR_SHAPE, PE_ERR_UNSUPPORTED.
  */
 pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H,
                             int W, const int32_t grid_thw[3], int merge, void *out,

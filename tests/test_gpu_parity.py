@@ -329,3 +329,34 @@ def test_error_paths():
     assert e.value.status == "PE_ERR_UNSUPPORTED"
     torch.cuda.synchronize()
     assert pe.last_error() == 0
+
+
+# ------------------------------------------------------ staged vs fused path
+
+@pytest.mark.parametrize("case", ["images", "video_odd_T", "mixed"])
+def test_staged_and_fused_paths_agree(case, monkeypatch):
+    """Both frames paths compute the same contraction in the same k order and
+    tile shape: outputs must be bit-identical, and within tolerance of the oracle."""
+    C, tp, p, E = 3, 2, 14, 1280
+    if case == "images":
+        grids = [(1, 12, 18), (1, 20, 10), (1, 8, 8)]
+        Ts = [1, 1, 1]
+    elif case == "video_odd_T":
+        grids = [(3, 10, 12)]
+        Ts = [5]
+    else:
+        grids = [(1, 10, 14), (2, 8, 8), (1, 6, 10)]
+        Ts = [1, 4, 1]
+    items = [workloads.Item(workloads.uniform01((T, C, g[1] * p, g[2] * p), 120 + i), g)
+             for i, (T, g) in enumerate(zip(Ts, grids))]
+    wl = workloads.Workload("staged_" + case, E, C, tp, p,
+                            workloads.normal((E, C, tp, p, p), 121, std=0.02, dtype=torch.bfloat16),
+                            workloads.normal((E,), 122, std=0.02, dtype=torch.bfloat16), torch.bfloat16,
+                            merge=2, items=items, mean=workloads.CLIP_MEAN, std=workloads.CLIP_STD)
+    outs = {}
+    for path in ("fused", "staged"):
+        monkeypatch.setenv("PE_FRAMES_PATH", path)
+        _, out, ref, mag = _run_frames(wl)
+        outs[path] = out
+        assert_within_tolerance(out, ref, mag, what=f"{case} {path}")
+    assert torch.equal(outs["fused"], outs["staged"])

@@ -39,6 +39,9 @@ struct pe_handle {
     ItemDesc *items_dev = nullptr;
     ItemDesc *items_pinned = nullptr;
     int items_cap = 0;
+    // staged frames path: normalised patch rows [N, K] (grow-only)
+    uint16_t *stage_rows = nullptr;
+    size_t stage_bytes = 0;
     cudaEvent_t items_evt = nullptr;
     bool items_evt_pending = false;
 };
@@ -300,9 +303,76 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
     return PE_OK;
 }
 
-pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st) {
+// Staged frames path: prepare kernel writes A once (frames k order), then the
+// TMA-fed pair GEMM reads it with the frames-order weight.  Chosen for large
+// inputs (the fused producer repeats its gather for every weight tile of a
+// row block), or forced with PE_FRAMES_PATH=staged / fused.
+constexpr int64_t kStagedMinRows = 8192;
+
+bool staged_eligible(const pe_handle *h, int f_dt) {
+    return f_dt == PE_BF16 && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
+}
+
+bool want_staged(const pe_handle *h, const FwdParams &P, int f_dt) {
+    if (!staged_eligible(h, f_dt)) return false;
+    const char *e = std::getenv("PE_FRAMES_PATH");
+    if (e && std::strcmp(e, "fused") == 0) return false;
+    if (e && std::strcmp(e, "staged") == 0) return true;
+    return P.N >= kStagedMinRows;
+}
+
+template <int PT>
+cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool dupall, uint16_t *A, cudaStream_t st) {
+    const int grid = (int)((P.N + kBM - 1) / kBM);
+    if (all_scaled) {
+        if (dupall) pe_prep_kernel<PT, 1, true><<<grid, 256, 0, st>>>(P, A);
+        else pe_prep_kernel<PT, 1, false><<<grid, 256, 0, st>>>(P, A);
+    } else {
+        if (dupall) pe_prep_kernel<PT, 2, true><<<grid, 256, 0, st>>>(P, A);
+        else pe_prep_kernel<PT, 2, false><<<grid, 256, 0, st>>>(P, A);
+    }
+    return cudaGetLastError();
+}
+
+pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool dupall, cudaStream_t st) {
+    const size_t need = (size_t)P.N * h->K * 2;
+    if (need > h->stage_bytes) {
+        if (h->stage_rows) {
+            if (cudaStreamSynchronize(st) != cudaSuccess) return PE_ERR_CUDA;
+            cudaFree(h->stage_rows);
+        }
+        h->stage_rows = nullptr;
+        h->stage_bytes = 0;
+        if (cudaMalloc(&h->stage_rows, need) != cudaSuccess) return PE_ERR_CUDA;
+        h->stage_bytes = need;
+    }
+    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, dupall, h->stage_rows, st)
+                                 : launch_prep<16>(P, all_scaled, dupall, h->stage_rows, st);
+    if (e != cudaSuccess) return PE_ERR_CUDA;
+    FwdParams G = P;
+    G.x = h->stage_rows;
+    G.x_f32 = 0;
+    G.x_vec = 1;
+    int grid = 0;
+    bool ok = true;
+    plan_tiles(h, G, G.N, false, grid, ok);
+    if (!ok) return PE_ERR_UNSUPPORTED;
+    const size_t smem = plan_pipeline(h, G, kAModeTma);
+    CUtensorMap tx, to;
+    if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)h->K, (uint64_t)h->K, kBM)) return PE_ERR_CUDA;
+    if (!make_out_tmap(&to, out, G.out_f32, G.N, G.E)) return PE_ERR_CUDA;
+    return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st));
+}
+
+pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st,
+                     bool allow_staged = true) {
     P.out_f32 = out_dt == PE_F32;
     if (P.N == 0) return PE_OK;
+    if (allow_staged && want_staged(h, P, f_dt)) {
+        bool all_scaled = true;
+        for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
+        return run_frames_staged(h, P, out, all_scaled, h->tp == 2 && P.all_t1, st);
+    }
     int grid = 0;
     bool ok = true;
     plan_tiles(h, P, P.N, true, grid, ok);
@@ -425,6 +495,7 @@ void pe_destroy(pe_handle *h) {
     if (h->err) cudaFree(h->err);
     if (h->items_dev) cudaFree(h->items_dev);
     if (h->items_pinned) cudaFreeHost(h->items_pinned);
+    if (h->stage_rows) cudaFree(h->stage_rows);
     if (h->items_evt) cudaEventDestroy(h->items_evt);
     delete h;
 }
@@ -618,7 +689,7 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
         }
         P.items_dev = table;
     }
-    return run_frames(h, P, f_dt, out, out_dt, st);
+    return run_frames(h, P, f_dt, out, out_dt, st, /*allow_staged=*/false);   // never allocates
 }
 
 pe_status pe_last_error(pe_handle *h) {

@@ -993,6 +993,82 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
     }
 }
 
+// Staged frames path, first half: the normalised patch rows A[N, K] written
+// once, in the frames k order k' = ((c*p + i)*tp + t)*p + j that the
+// frames-order weight uses, for the TMA-fed contraction to read back.  Each
+// CTA owns 128 rows; each thread owns MAXIT (row, word) units exactly as the
+// fused producer does (coalesced 32-bit loads along image rows), walks the
+// (c, i) pairs four at a time, and stores the normalised words -- once per
+// temporal slice, the same word twice when the row's item is a single frame.
+template <int PT, int NORM, bool DUPALL>
+__global__ void __launch_bounds__(256) pe_prep_kernel(const __grid_constant__ FwdParams P, uint16_t *A) {
+    constexpr int p = PT, ws = p / 2, units = kBM * ws, kThr = 256;
+    constexpr int MAXIT = (units + kThr - 1) / kThr;
+    const int64_t m0 = (int64_t)blockIdx.x * kBM;
+    const int nci = P.C * p;
+    const int K = P.K;
+    const char *src[MAXIT];
+    uint16_t *dst[MAXIT];
+    int32_t sW[MAXIT], sHW[MAXIT], sT1[MAXIT];
+    uint32_t rok = 0, dup = 0;
+#pragma unroll
+    for (int v = 0; v < MAXIT; ++v) {
+        const int u = threadIdx.x + kThr * v;
+        src[v] = nullptr;
+        dst[v] = nullptr;
+        sW[v] = sHW[v] = sT1[v] = 0;
+        if (u >= units) continue;
+        int r, jw;
+        unit_to_row_word(u, ws, P.merge, r, jw);
+        if (m0 + r >= P.N) continue;
+        const RowSrc rs = locate_row(P, m0 + r, 2);
+        src[v] = rs.base + 4 * jw;
+        dst[v] = A + (m0 + r) * (int64_t)K + 2 * jw;
+        sW[v] = rs.W * 2;
+        sHW[v] = rs.HW * 2;
+        sT1[v] = rs.tmax > 0 ? rs.CHW * 2 : 0;
+        rok |= 1u << v;
+        if (rs.tmax == 0) dup |= 1u << v;
+    }
+    constexpr int NT = DUPALL ? 1 : 2;
+    for (int ci0 = 0; ci0 < nci; ci0 += 4) {
+        uint32_t raw[4][NT][MAXIT];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int ci = ci0 + q;
+            const int c = ci / p, i = ci - (ci / p) * p;
+#pragma unroll
+            for (int v = 0; v < MAXIT; ++v) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t) raw[q][t][v] = 0u;
+                if (ci < nci && (rok >> v & 1u)) {
+                    const char *a = src[v] + (int64_t)c * sHW[v] + (int64_t)i * sW[v];
+                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[q][0][v]) : "l"(a));
+                    if constexpr (!DUPALL) {
+                        if (sT1[v] != 0)
+                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[q][NT - 1][v]) : "l"(a + sT1[v]));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int ci = ci0 + q;
+            if (ci >= nci) break;
+            const NormConst nc = norm_const(P, ci / p);
+#pragma unroll
+            for (int v = 0; v < MAXIT; ++v) {
+                if (!(rok >> v & 1u)) continue;
+                const uint32_t w0 = norm_word<NORM>(raw[q][0][v], nc);
+                const uint32_t w1 = (DUPALL || (dup >> v & 1u)) ? w0 : norm_word<NORM>(raw[q][NT - 1][v], nc);
+                uint16_t *d = dst[v] + (int64_t)ci * (2 * p);   // k' of (c, i, t = 0, j)
+                *reinterpret_cast<uint32_t *>(d) = w0;
+                *reinterpret_cast<uint32_t *>(d + p) = w1;
+            }
+        }
+    }
+}
+
 // rows[R, k] for every output row R, in the view(-1, C, tp, p, p) order: the
 // frames producer's gather and normalisation written to memory (bf16 or fp32
 // values; bf16-exact either way).
