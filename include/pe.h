@@ -211,6 +211,23 @@ pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f
 int64_t pe_num_patches(const int32_t *grid_thw, int n);
 
 /*
+ * pe_profile_begin / pe_profile_end -- device time of each forward call's
+ * contraction kernel (the fused kernel, or the GEMM of the staged path),
+ * recorded with a CUDA event pair on the call's stream around that launch.
+ * pe_profile_begin creates event pairs for up to max_calls calls (1..1e6) and
+ * starts recording; pe_profile_end waits for the recorded events, writes the
+ * elapsed milliseconds of the first min(*n, recorded) calls to host ms[] and
+ * that count to *n, writes to *launches (if not NULL) how many kernels the
+ * forward calls launched in the window (the staged frames path launches two
+ * per call, every other forward one), then frees the events and stops
+ * recording.  Profiling is a measurement aid: it allocates events and must not
+ * overlap another profiling window on the same handle.
+ * Errors: PE_ERR_INVALID_ARG, PE_ERR_CUDA.
+ */
+pe_status pe_profile_begin(pe_handle *h, int max_calls);
+pe_status pe_profile_end(pe_handle *h, float *ms, int *n, int64_t *launches);
+
+/*
  * pe_last_error -- read and clear the handle's device error word.  Call after
  * synchronising the streams the handle ran on.  Returns PE_OK, or
  * PE_ERR_DEVICE_TIMEOUT if a kernel stopped waiting on its pipeline (it then

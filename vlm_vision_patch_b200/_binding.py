@@ -28,7 +28,7 @@ PE_NOALLOC_MAX_ITEMS = 1024
 EXPORTS = (
     "pe_create", "pe_set_weight", "pe_set_norm", "pe_forward_patches", "pe_forward_frames",
     "pe_forward_frames_grouped", "pe_forward_frames_grouped_noalloc", "pe_patchify", "pe_num_patches", "pe_last_error",
-    "pe_status_string", "pe_destroy", "pe_device",
+    "pe_status_string", "pe_destroy", "pe_device", "pe_profile_begin", "pe_profile_end",
 )
 
 
@@ -69,6 +69,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_status_string": ([i32], ctypes.c_char_p),
         "pe_destroy": ([vp], None),
         "pe_device": ([vp], i32),
+        "pe_profile_begin": ([vp, i32], i32),
+        "pe_profile_end": ([vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(i32),
+                            ctypes.POINTER(ctypes.c_int64)], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -164,6 +167,19 @@ def pe_patchify(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence
 def pe_num_patches(grid_thw: Sequence[Sequence[int]]) -> int:
     flat = [v for g in grid_thw for v in g]
     return int(load().pe_num_patches(_i32arr(flat) if flat else None, len(grid_thw)))
+
+
+def pe_profile_begin(h: int, max_calls: int) -> None:
+    _check("pe_profile_begin", load().pe_profile_begin(h, max_calls))
+
+
+def pe_profile_end(h: int, max_calls: int):
+    """Returns (per-call contraction-kernel ms, kernels launched in the window)."""
+    ms = (ctypes.c_float * max(1, max_calls))()
+    n = ctypes.c_int(max_calls)
+    launches = ctypes.c_int64(0)
+    _check("pe_profile_end", load().pe_profile_end(h, ms, ctypes.byref(n), ctypes.byref(launches)))
+    return [float(ms[i]) for i in range(n.value)], int(launches.value)
 
 
 def pe_last_error(h: int) -> int:

@@ -42,6 +42,11 @@ struct pe_handle {
     // staged frames path: normalised patch rows [N, K] (grow-only)
     uint16_t *stage_rows = nullptr;
     size_t stage_bytes = 0;
+    // profiling: one event pair per call around the contraction kernel
+    std::vector<cudaEvent_t> prof_ev;
+    int prof_cap = 0, prof_n = 0;
+    int64_t prof_launches = 0;   // kernels launched by forward calls while profiling
+    bool prof_on = false;
     cudaEvent_t items_evt = nullptr;
     bool items_evt_pending = false;
 };
@@ -135,15 +140,31 @@ int choose_bn(int64_t N, int E, int num_pairs, bool gather_fed) {
     return 64;
 }
 
+thread_local pe_handle *t_prof_handle = nullptr;   // handle of the call being launched
+
 template <int AMODE, int PT, bool F32IN, int NORM = 2, bool DUPALL = false>
 cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensorMap &tx, const CUtensorMap &to,
                        size_t smem, int grid, cudaStream_t st) {
     auto kern = pe_fwd_kernel<AMODE, PT, F32IN, NORM, DUPALL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    pe_handle *h = t_prof_handle;
+    const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
+    if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
     kern<<<grid, threads_for(AMODE), smem, st>>>(tw, tx, to, P);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (prof) {
+        cudaEventRecord(h->prof_ev[2 * h->prof_n + 1], st);
+        ++h->prof_n;
+    }
+    if (h && h->prof_on) ++h->prof_launches;
+    return e;
 }
+
+struct ProfScope {   // makes the handle's profiling events visible to launch_fwd
+    explicit ProfScope(pe_handle *h) { t_prof_handle = h; }
+    ~ProfScope() { t_prof_handle = nullptr; }
+};
 
 int bn_index(int bn) { return bn == 64 ? 0 : (bn == 128 ? 1 : 2); }
 
@@ -348,6 +369,7 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     }
     cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, dupall, h->stage_rows, st)
                                  : launch_prep<16>(P, all_scaled, dupall, h->stage_rows, st);
+    if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
     FwdParams G = P;
     G.x = h->stage_rows;
@@ -497,6 +519,7 @@ void pe_destroy(pe_handle *h) {
     if (h->items_pinned) cudaFreeHost(h->items_pinned);
     if (h->stage_rows) cudaFree(h->stage_rows);
     if (h->items_evt) cudaEventDestroy(h->items_evt);
+    for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
     delete h;
 }
 
@@ -543,6 +566,7 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
     if (!x || !out) return PE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(out)) return PE_ERR_ALIGN;
     DeviceGuard g(h->dev);
+    ProfScope ps(h);
     FwdParams P;
     fill_common(h, P);
     P.N = N;
@@ -576,6 +600,7 @@ pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *fram
     if (!valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (!h->weight_set) return PE_ERR_NO_WEIGHT;
     DeviceGuard g(h->dev);
+    ProfScope ps(h);
     FwdParams P;
     const pe_status s = setup_frames(h, n, frames, f_dt, THW, grid_thw, merge, out, P, (cudaStream_t)stream);
     if (s != PE_OK) return s;
@@ -650,6 +675,7 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
     if ((h->p & 1) || h->p > PE_MAX_PATCH) return PE_ERR_UNSUPPORTED;
     if (!aligned16(out)) return PE_ERR_ALIGN;
     DeviceGuard g(h->dev);
+    ProfScope ps(h);
     cudaStream_t st = (cudaStream_t)stream;
     FwdParams P;
     fill_common(h, P);
@@ -690,6 +716,39 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
         P.items_dev = table;
     }
     return run_frames(h, P, f_dt, out, out_dt, st, /*allow_staged=*/false);   // never allocates
+}
+
+pe_status pe_profile_begin(pe_handle *h, int max_calls) {
+    if (!h || max_calls < 1 || max_calls > 1000000) return PE_ERR_INVALID_ARG;
+    DeviceGuard g(h->dev);
+    for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
+    h->prof_ev.assign((size_t)2 * max_calls, nullptr);
+    for (auto &e : h->prof_ev)
+        if (cudaEventCreate(&e) != cudaSuccess) return PE_ERR_CUDA;
+    h->prof_cap = max_calls;
+    h->prof_n = 0;
+    h->prof_launches = 0;
+    h->prof_on = true;
+    return PE_OK;
+}
+
+pe_status pe_profile_end(pe_handle *h, float *ms, int *n, int64_t *launches) {
+    if (!h || !n || (*n > 0 && !ms)) return PE_ERR_INVALID_ARG;
+    if (launches) *launches = h->prof_launches;
+    DeviceGuard g(h->dev);
+    const int cnt = std::min(h->prof_n, *n);
+    pe_status st = PE_OK;
+    for (int i = 0; i < cnt; ++i) {
+        if (cudaEventSynchronize(h->prof_ev[2 * i + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms[i], h->prof_ev[2 * i], h->prof_ev[2 * i + 1]) != cudaSuccess)
+            st = PE_ERR_CUDA;
+    }
+    *n = cnt;
+    for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
+    h->prof_ev.clear();
+    h->prof_cap = h->prof_n = 0;
+    h->prof_on = false;
+    return st;
 }
 
 pe_status pe_last_error(pe_handle *h) {
