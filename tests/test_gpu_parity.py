@@ -333,30 +333,43 @@ def test_error_paths():
 
 # ------------------------------------------------------ staged vs fused path
 
-@pytest.mark.parametrize("case", ["images", "video_odd_T", "mixed"])
+@pytest.mark.parametrize("case", ["images", "video_odd_T", "mixed", "images_p16_raster"])
 def test_staged_and_fused_paths_agree(case, monkeypatch):
-    """Both frames paths compute the same contraction in the same k order and
-    tile shape: outputs must be bit-identical, and within tolerance of the oracle."""
-    C, tp, p, E = 3, 2, 14, 1280
+    """Both frames paths must be within tolerance of the oracle.  Where some
+    item has more than one frame, both run the contraction in the same k order
+    and tile shape, so their outputs must also be bit-identical.  When every
+    item is a single frame the staged path stores one temporal slice per row
+    and meets it with both slices of the weight (a different summation order),
+    so only the tolerance applies."""
+    C, tp, p, E, merge = 3, 2, 14, 1280, 2
     if case == "images":
         grids = [(1, 12, 18), (1, 20, 10), (1, 8, 8)]
         Ts = [1, 1, 1]
     elif case == "video_odd_T":
         grids = [(3, 10, 12)]
         Ts = [5]
-    else:
+    elif case == "mixed":
         grids = [(1, 10, 14), (2, 8, 8), (1, 6, 10)]
         Ts = [1, 4, 1]
+    else:   # p = 16: slice length 768 needs no padding; raster order; ragged row count
+        p, E, merge = 16, 1152, 1
+        grids = [(1, 7, 9), (1, 5, 11), (1, 13, 3)]
+        Ts = [1, 1, 1]
     items = [workloads.Item(workloads.uniform01((T, C, g[1] * p, g[2] * p), 120 + i), g)
              for i, (T, g) in enumerate(zip(Ts, grids))]
     wl = workloads.Workload("staged_" + case, E, C, tp, p,
                             workloads.normal((E, C, tp, p, p), 121, std=0.02, dtype=torch.bfloat16),
                             workloads.normal((E,), 122, std=0.02, dtype=torch.bfloat16), torch.bfloat16,
-                            merge=2, items=items, mean=workloads.CLIP_MEAN, std=workloads.CLIP_STD)
+                            merge=merge, items=items, mean=workloads.CLIP_MEAN, std=workloads.CLIP_STD)
     outs = {}
     for path in ("fused", "staged"):
         monkeypatch.setenv("PE_FRAMES_PATH", path)
         _, out, ref, mag = _run_frames(wl)
         outs[path] = out
         assert_within_tolerance(out, ref, mag, what=f"{case} {path}")
-    assert torch.equal(outs["fused"], outs["staged"])
+    if any(T > 1 for T in Ts):
+        assert torch.equal(outs["fused"], outs["staged"])
+    if case == "images":   # fp32 output from the staged path
+        _, out, ref, mag = _run_frames(wl, out_dtype=torch.float32)
+        assert out.dtype == torch.float32
+        assert_within_tolerance(out, ref, mag, what=f"{case} staged fp32 out")

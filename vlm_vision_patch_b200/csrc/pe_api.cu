@@ -23,16 +23,19 @@ using namespace pe;
 struct pe_handle {
     int dev = -1;
     int E = 0, C = 0, tp = 0, p = 0, K = 0, Kpad = 0;
+    int Kh = 0;                 // C*p*p rounded up to 16: one temporal slice of the slice-major weight
     bool has_bias = false;
     bool weight_set = false;
     uint16_t *wpack = nullptr;  // dev [E, Kpad] bf16, view(-1, C, tp, p, p) k order
     uint16_t *wpack_f = nullptr; // dev [E, Kpad] bf16, k order of the frames producer
+    uint16_t *wpack_t = nullptr; // dev [E, 2*Kh] bf16, slice-major (tp == 2 only)
     float *bias = nullptr;      // dev [E] fp32 (has_bias)
     int *err = nullptr;         // dev error word
     float mean[4] = {0, 0, 0, 0};
     float stdv[4] = {1, 1, 1, 1};
     CUtensorMap tmap_w[3];      // weight boxes of 32, 64, 128 rows (half a pair tile)
     CUtensorMap tmap_wf[3];     // same for the frames-order weight
+    CUtensorMap tmap_wt[3];     // same for the slice-major weight
     int num_sms = 0;
     int smem_optin = 0;
     // item table for grouped calls beyond PE_INLINE_ITEMS
@@ -187,6 +190,7 @@ void fill_common(const pe_handle *h, FwdParams &P) {
     P.P = h->p;
     P.K = h->K;
     P.Kpad = h->Kpad;
+    P.Kh = h->Kh;
     for (int c = 0; c < 4; ++c) {
         const float mu = h->mean[c], sd = h->stdv[c];
         uint32_t mu_bits;
@@ -212,6 +216,11 @@ void fill_common(const pe_handle *h, FwdParams &P) {
 // Ring depths and per-tile stage counts; returns the dynamic shared memory size.
 size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
     P.num_ksteps = (P.K + 15) / 16;
+    P.b_slot_bytes = kBStageBytes;
+    if (amode == kAModeTmaShared) {
+        P.num_ksteps = P.Kh / 16;            // k-steps per slice; each is issued once per slice
+        P.b_slot_bytes = 2 * kBStageBytes;   // weight tiles of both slices
+    }
     P.n_b_stages = (P.num_ksteps + 3) / 4;
     if (amode == kAModeFrames) {
         P.a_stage_bytes = 2048 * P.P;  // 8 segments of p pixels, 128 rows
@@ -221,7 +230,7 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
         P.n_a_stages = P.n_b_stages;
     }
     const size_t epi_bytes = (size_t)4 * 8192;   // staging ring of the 4 epilogue warps
-    auto rings = [&](int nb, int na) { return (size_t)nb * kBStageBytes + (size_t)na * P.a_stage_bytes; };
+    auto rings = [&](int nb, int na) { return (size_t)nb * P.b_slot_bytes + (size_t)na * P.a_stage_bytes; };
     auto total = [&](int nb, int na) {
         const size_t r = (rings(nb, na) + 1023) / 1024 * 1024;
         return 1024 + r + epi_bytes + (size_t)(2 * nb + 2 * na + 5) * 8 + 16;
@@ -242,7 +251,7 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
     }
     P.nb = nb;
     P.na = na;
-    P.n_iss = std::min(amode == kAModeTma ? 5 : 3, std::min(nb, na));
+    P.n_iss = std::min(tma_fed(amode) ? 5 : 3, std::min(nb, na));
     P.epi_offset = (int)((rings(nb, na) + 1023) / 1024 * 1024);
     return total(nb, na);
 }
@@ -342,21 +351,32 @@ bool want_staged(const pe_handle *h, const FwdParams &P, int f_dt) {
     return P.N >= kStagedMinRows;
 }
 
-template <int PT>
-cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool dupall, uint16_t *A, cudaStream_t st) {
-    const int grid = (int)((P.N + kBM - 1) / kBM);
-    if (all_scaled) {
-        if (dupall) pe_prep_kernel<PT, 1, true><<<grid, 256, 0, st>>>(P, A);
-        else pe_prep_kernel<PT, 1, false><<<grid, 256, 0, st>>>(P, A);
-    } else {
-        if (dupall) pe_prep_kernel<PT, 2, true><<<grid, 256, 0, st>>>(P, A);
-        else pe_prep_kernel<PT, 2, false><<<grid, 256, 0, st>>>(P, A);
-    }
+template <int PT, int NORM, bool SHARED>
+cudaError_t launch_prep_rows(const FwdParams &P, uint16_t *A, int row_elems, cudaStream_t st) {
+    auto kern = pe_prep_rows_kernel<PT, NORM, SHARED>;
+    const int smem = kPrepRows * row_elems * 2;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (P.N + kPrepRows - 1) / kPrepRows;
+    kern<<<(unsigned)grid, kPrepRows * PT / 2, smem, st>>>(P, A, row_elems);
     return cudaGetLastError();
 }
 
-pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool dupall, cudaStream_t st) {
-    const size_t need = (size_t)P.N * h->K * 2;
+template <int PT>
+cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool shared, uint16_t *A, int row_elems,
+                        cudaStream_t st) {
+    if (all_scaled)
+        return shared ? launch_prep_rows<PT, 1, true>(P, A, row_elems, st)
+                      : launch_prep_rows<PT, 1, false>(P, A, row_elems, st);
+    return shared ? launch_prep_rows<PT, 2, true>(P, A, row_elems, st)
+                  : launch_prep_rows<PT, 2, false>(P, A, row_elems, st);
+}
+
+// shared: every row is a single frame (tp == 2), so A holds one slice per row
+// (A[N, Kh]) and the contraction meets it with the slice-major weight.
+pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, cudaStream_t st) {
+    const int row_elems = shared ? h->Kh : h->K;
+    const size_t need = (size_t)P.N * row_elems * 2;
     if (need > h->stage_bytes) {
         if (h->stage_rows) {
             if (cudaStreamSynchronize(st) != cudaSuccess) return PE_ERR_CUDA;
@@ -367,8 +387,8 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
         if (cudaMalloc(&h->stage_rows, need) != cudaSuccess) return PE_ERR_CUDA;
         h->stage_bytes = need;
     }
-    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, dupall, h->stage_rows, st)
-                                 : launch_prep<16>(P, all_scaled, dupall, h->stage_rows, st);
+    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, h->stage_rows, row_elems, st)
+                                 : launch_prep<16>(P, all_scaled, shared, h->stage_rows, row_elems, st);
     if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
     FwdParams G = P;
@@ -379,10 +399,14 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     bool ok = true;
     plan_tiles(h, G, G.N, false, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
-    const size_t smem = plan_pipeline(h, G, kAModeTma);
+    const int amode = shared ? kAModeTmaShared : kAModeTma;
+    const size_t smem = plan_pipeline(h, G, amode);
     CUtensorMap tx, to;
-    if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)h->K, (uint64_t)h->K, kBM)) return PE_ERR_CUDA;
+    if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
+        return PE_ERR_CUDA;
     if (!make_out_tmap(&to, out, G.out_f32, G.N, G.E)) return PE_ERR_CUDA;
+    if (shared)
+        return finish(launch_fwd<kAModeTmaShared, 0, false>(h->tmap_wt[bn_index(G.bn)], G, tx, to, smem, grid, st));
     return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st));
 }
 
@@ -393,7 +417,7 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
     if (allow_staged && want_staged(h, P, f_dt)) {
         bool all_scaled = true;
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
-        return run_frames_staged(h, P, out, all_scaled, h->tp == 2 && P.all_t1, st);
+        return run_frames_staged(h, P, out, all_scaled, h->tp == 2 && P.all_t1 && h->wpack_t, st);
     }
     int grid = 0;
     bool ok = true;
@@ -487,6 +511,7 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
     h->p = p;
     h->K = (int)K;
     h->Kpad = (int)((K + 63) / 64 * 64);
+    h->Kh = (C * p * p + 15) / 16 * 16;
     h->has_bias = has_bias != 0;
     bool ok = cudaMalloc(&h->wpack, sizeof(uint16_t) * (size_t)E * h->Kpad) == cudaSuccess &&
               cudaMalloc(&h->wpack_f, sizeof(uint16_t) * (size_t)E * h->Kpad) == cudaSuccess &&
@@ -494,13 +519,16 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
               cudaMemset(h->err, 0, sizeof(int)) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->items_evt, cudaEventDisableTiming) == cudaSuccess;
     if (ok && h->has_bias) ok = cudaMalloc(&h->bias, sizeof(float) * E) == cudaSuccess;
+    if (ok && tp == 2) ok = cudaMalloc(&h->wpack_t, sizeof(uint16_t) * (size_t)E * 2 * h->Kh) == cudaSuccess;
     if (ok) {
         const uint32_t boxes[3] = {32, 64, 128};   // half of BN = 64, 128, 256
         for (int i = 0; i < 3 && ok; ++i)
             ok = make_tmap_bf16(&h->tmap_w[i], h->wpack, (uint64_t)E, (uint64_t)h->Kpad, (uint64_t)h->Kpad,
                                 boxes[i]) &&
                  make_tmap_bf16(&h->tmap_wf[i], h->wpack_f, (uint64_t)E, (uint64_t)h->Kpad, (uint64_t)h->Kpad,
-                                boxes[i]);
+                                boxes[i]) &&
+                 (!h->wpack_t || make_tmap_bf16(&h->tmap_wt[i], h->wpack_t, (uint64_t)E, (uint64_t)(2 * h->Kh),
+                                                (uint64_t)(2 * h->Kh), boxes[i]));
     }
     if (!ok) { pe_destroy(h); return PE_ERR_CUDA; }
     *out = h;
@@ -513,6 +541,7 @@ void pe_destroy(pe_handle *h) {
     cudaDeviceSynchronize();
     if (h->wpack) cudaFree(h->wpack);
     if (h->wpack_f) cudaFree(h->wpack_f);
+    if (h->wpack_t) cudaFree(h->wpack_t);
     if (h->bias) cudaFree(h->bias);
     if (h->err) cudaFree(h->err);
     if (h->items_dev) cudaFree(h->items_dev);
@@ -533,12 +562,18 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
     const int64_t total = (int64_t)h->E * h->Kpad;
     const int threads = 256;
     const int blocks = (int)std::min<int64_t>((total + threads - 1) / threads, (int64_t)h->num_sms * 8);
-    pe_pack_weight_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
-        w, w_dt == PE_F32, bias, b_dt == PE_F32, h->wpack, h->bias, h->E, h->C, h->tp, h->p, h->Kpad, 0);
+    cudaStream_t st = (cudaStream_t)stream;
+    pe_pack_weight_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, bias, b_dt == PE_F32, h->wpack, h->bias,
+                                                      h->E, h->C, h->tp, h->p, h->Kpad, 0, h->Kh);
     if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
-    pe_pack_weight_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
-        w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_f, nullptr, h->E, h->C, h->tp, h->p, h->Kpad, 1);
+    pe_pack_weight_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_f,
+                                                      nullptr, h->E, h->C, h->tp, h->p, h->Kpad, 1, h->Kh);
     if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    if (h->wpack_t) {
+        pe_pack_weight_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_t,
+                                                          nullptr, h->E, h->C, h->tp, h->p, 2 * h->Kh, 2, h->Kh);
+        if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    }
     h->weight_set = true;
     return PE_OK;
 }

@@ -30,7 +30,7 @@ namespace pe {
 
 constexpr int kThreads = 640;       // 20 warps (A produced by threads)
 constexpr int kThreadsTma = 320;    // 10 warps (A fetched by TMA)
-__host__ __device__ constexpr int threads_for(int amode) { return amode == 0 ? kThreadsTma : kThreads; }
+__host__ __device__ constexpr int threads_for(int amode) { return (amode == 0 || amode == 3) ? kThreadsTma : kThreads; }
 constexpr int kBM = 128;           // rows per CTA (pair tile: 256 rows)
 constexpr int kMaxBN = 256;        // largest pair-MMA N
 constexpr int kBK = 64;            // weight K per TMA stage (one 128-byte swizzle row)
@@ -39,7 +39,15 @@ constexpr int kProdWarps = 12;
 constexpr int kEpiWarp0 = 4;
 constexpr int kBStageBytes = (kMaxBN / 2) * kBK * 2;   // 16 KB: this CTA's half of the weight tile
 
-enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2 };
+// How the A operand reaches shared memory:
+//   kAModeTma          TMA tiles of bf16 rows A[N, K] (patches, or the staged frames rows)
+//   kAModePatchThreads fp32 / unaligned patch rows converted by producer warps
+//   kAModeFrames       the fused gather from raw frames by producer warps
+//   kAModeTmaShared    TMA tiles of single-frame rows A[N, Kh] that both temporal
+//                      slices share: every A tile meets the weight tiles of
+//                      slice 0 and slice 1 at the same in-slice k (tp = 2).
+enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2, kAModeTmaShared = 3 };
+__host__ __device__ constexpr bool tma_fed(int amode) { return amode == kAModeTma || amode == kAModeTmaShared; }
 
 struct ItemDesc {
     const void *frames;  // [T, C, H, W]
@@ -50,11 +58,13 @@ struct ItemDesc {
 
 struct FwdParams {
     int32_t E, C, TP, P, K, Kpad;
+    int32_t Kh;                                     // slice length of the shared-slice weight (C*p*p rounded to 16)
     int32_t bn, n_tiles_n, num_tiles, num_ksteps;   // num_tiles counts pair tiles
     int32_t n_b_stages, n_a_stages;                 // per tile
     int32_t nb, na;                                 // ring depths
     int32_t n_iss;                                  // TMA issuer warps, <= min(nb, na)
     int32_t a_stage_bytes;
+    int32_t b_slot_bytes;                           // weight ring slot: 16 KB, or 32 KB (two slices)
     int32_t epi_offset;                             // staging area offset past the rings
     int32_t merge, n_items;
     int32_t all_t1;                   // every item is a single frame (host-side kernel choice)
@@ -220,12 +230,13 @@ template <> struct PixPair<true> {
 // Unit u of a segment (one 2-pixel word of one tile row) -> (tile row, word).
 // For merge = 2 the order walks patch-row halves of the windows so that
 // consecutive u read consecutive words of one image row.
+template <int RB = kBM>
 __device__ __forceinline__ void unit_to_row_word(int u, int ws, int merge, int &r, int &jw) {
     jw = u % ws;
     const int t1 = u / ws;
     if (merge == 2) {
         const int dw = t1 & 1, t2 = t1 >> 1;
-        const int q = t2 & 31, dh = t2 >> 5;
+        const int q = t2 % (RB / 4), dh = t2 / (RB / 4);
         r = 4 * q + 2 * dh + dw;
     } else {
         r = t1;
@@ -692,6 +703,57 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
     mbar_wait(smem_addr(mma_done), 0, abort);
 }
 
+// Shared-slice issue (kAModeTmaShared): ring slot s holds the A tile of
+// in-slice k in [64s, 64s + 64) and the weight tiles of slice 0 and slice 1 at
+// the same k; each A k-step is issued against both, so the single-frame rows
+// are fetched once for the two temporal slices they stand for.
+__device__ __forceinline__ void mma_issue_shared(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring,
+                                                 uint64_t *full_b, uint64_t *empty_b, uint64_t *tfull,
+                                                 uint64_t *tempty, uint64_t *mma_done, uint32_t tmem_base,
+                                                 volatile int *abort) {
+    constexpr uint16_t kPair = 0x3;
+    constexpr uint32_t kSlice1 = (uint32_t)kBStageBytes >> 4;   // slice-1 weight tile, descriptor units
+    const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
+    const uint64_t a0 = smem_desc(smem_addr(a_ring), 16, 1024, kLayoutSw128);
+    const uint64_t b0 = smem_desc(smem_addr(b_ring), 16, 1024, kLayoutSw128);
+    const uint32_t a_lo0 = (uint32_t)a0, b_lo0 = (uint32_t)b0;
+    const uint32_t a_slot = (uint32_t)P.a_stage_bytes >> 4, b_slot = (uint32_t)P.b_slot_bytes >> 4;
+    const int nk = P.num_ksteps, nst = P.n_b_stages;
+    int bs = 0, acc = 0;
+    uint32_t bph = 0, accph = 0;
+    for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+        if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) return;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)acc * kMaxBN;
+        for (int st = 0; st < nst; ++st) {
+            if (!mbar_wait(smem_addr(&full_b[bs]), bph, abort)) return;
+            tc_fence_after();
+            const uint32_t a_lo = a_lo0 + (uint32_t)bs * a_slot, b_lo = b_lo0 + (uint32_t)bs * b_slot;
+            const int kin = nk - 4 * st;
+            if (kin >= 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t ad = desc_with_lo(a0, a_lo + 2u * j);
+                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + 2u * j), idesc, (st | j) ? 1u : 0u);
+                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
+                }
+            } else {
+                for (int j = 0; j < kin; ++j) {
+                    const uint64_t ad = desc_with_lo(a0, a_lo + 2u * j);
+                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + 2u * j), idesc, (st | j) ? 1u : 0u);
+                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
+                }
+            }
+            mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
+            if (++bs == P.nb) { bs = 0; bph ^= 1; }
+        }
+        mma_commit_pair(smem_addr(&tfull[acc]), kPair);
+        if (++acc == 2) { acc = 0; accph ^= 1; }
+    }
+    mma_commit_pair(smem_addr(mma_done), 0x1);
+    mbar_wait(smem_addr(mma_done), 0, abort);
+}
+
 // Runtime-p frames path (p not 14 or 16): the same protocol, not unrolled.
 __device__ __noinline__ void mma_issue_generic(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring,
                                                uint64_t *full_a, uint64_t *empty_a, uint64_t *full_b,
@@ -744,7 +806,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *b_ring = smem;
-    uint8_t *a_ring = b_ring + (size_t)P.nb * kBStageBytes;
+    uint8_t *a_ring = b_ring + (size_t)P.nb * P.b_slot_bytes;
+    constexpr bool kTmaA = tma_fed(AMODE);
     uint8_t *epi = smem + P.epi_offset;
     uint64_t *bars = reinterpret_cast<uint64_t *>(epi + 4 * 8192);   // 8 KB staging per epilogue warp
     uint64_t *full_b = bars;
@@ -767,7 +830,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             mbar_init(smem_addr(&empty_b[s]), 1);
         }
         for (int s = 0; s < P.na; ++s) {
-            mbar_init(smem_addr(&full_a[s]), AMODE == kAModeTma ? 1 : 2 * kProdWarps);
+            mbar_init(smem_addr(&full_a[s]), kTmaA ? 1 : 2 * kProdWarps);
             mbar_init(smem_addr(&empty_a[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -781,7 +844,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_w);
         prefetch_tmap(&tmap_out);
-        if (AMODE == kAModeTma) prefetch_tmap(&tmap_x);
+        if (kTmaA) prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_addr(tmem_holder), 512);
@@ -796,7 +859,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
     // P.n_iss of them issue, and P.n_iss never exceeds a ring depth: an issuer
     // then can never lap a slot, so its parity waits cannot alias.
     const int iss = (warp == 0) ? 0 : (warp == 2 || warp == 3) ? warp - 1
-                  : (AMODE == kAModeTma && warp >= 8 && warp < 10) ? warp - 5 : -1;
+                  : (kTmaA && warp >= 8 && warp < 10) ? warp - 5 : -1;
     const int n_iss = P.n_iss;
     if (iss >= 0) {
         // ---------------- TMA issuers (both CTAs; bytes complete on the leader's barriers).
@@ -818,14 +881,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     // In the TMA-fed path A and weight share ring slot and barriers.
                     const int bs = g % P.nb;
                     if (!mbar_wait(smem_addr(&empty_b[bs]), ((g / P.nb) & 1) ^ 1, abort)) { ok = false; break; }
+                    constexpr uint32_t kSlices = (AMODE == kAModeTmaShared) ? 2u : 1u;
                     if (leader)
-                        mbar_arrive_expect_tx(smem_addr(&full_b[bs]),
-                                              2 * (b_bytes + (AMODE == kAModeTma ? a_bytes : 0u)));
-                    if (AMODE == kAModeTma)
+                        mbar_arrive_expect_tx(smem_addr(&full_b[bs]), 2 * (kSlices * b_bytes + (kTmaA ? a_bytes : 0u)));
+                    if (kTmaA)
                         tma_load_2d_pair(smem_addr(a_ring + (size_t)bs * P.a_stage_bytes), &tmap_x, fb0 + 8u * bs,
                                          kb * kBK, m_blk * (2 * kBM) + (int)rank * kBM, pol_x);
-                    tma_load_2d_pair(smem_addr(b_ring + (size_t)bs * kBStageBytes), &tmap_w, fb0 + 8u * bs,
-                                     kb * kBK, n_blk * P.bn + (int)rank * (P.bn / 2), pol_w);
+                    const uint32_t bdst = smem_addr(b_ring + (size_t)bs * P.b_slot_bytes);
+                    const int wrow = n_blk * P.bn + (int)rank * (P.bn / 2);
+                    tma_load_2d_pair(bdst, &tmap_w, fb0 + 8u * bs, kb * kBK, wrow, pol_w);
+                    if (AMODE == kAModeTmaShared)
+                        tma_load_2d_pair(bdst + kBStageBytes, &tmap_w, fb0 + 8u * bs, P.Kh + kb * kBK, wrow, pol_w);
                 }
             }
         }
@@ -833,7 +899,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         // ---------------- MMA issuer (leader CTA only)
         if (leader && lane == 0) {
             constexpr int KSA = (AMODE == kAModeFrames) ? (PT ? PT / 2 : 0) : 4;
-            if constexpr (KSA > 0)
+            if constexpr (AMODE == kAModeTmaShared)
+                mma_issue_shared(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
+            else if constexpr (KSA > 0)
                 mma_issue<KSA, AMODE == kAModeFrames, AMODE != kAModeTma>(P, a_ring, b_ring, full_a, empty_a, full_b,
                                                                           empty_b, tfull, tempty, mma_done, tmem_base,
                                                                           abort);
@@ -898,7 +966,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             tc_fence_after();
             const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
             const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
-            if constexpr (AMODE == kAModeTma) {
+            if constexpr (kTmaA) {
                 // registers to spare: the next chunk's TMEM load overlaps this chunk's work
                 uint32_t va[32], vb[32];
                 tmem_ld_32x32b_x32(tbase, va);
@@ -925,7 +993,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         }
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
-    } else if (warp >= 8 && AMODE != kAModeTma) {
+    } else if (warp >= 8 && !kTmaA) {
         // ---------------- A producers (both CTAs)
         ProdCtx X;
         X.a_ring = a_ring;
@@ -957,28 +1025,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
 
 // ------------------------------------------------------------- helpers
 
-// Weight packing.  Ŵ[e, k] = bf16_rne(W[e, k]) for k < K and 0 for K <= k < Kpad,
-// stored either in the view(-1, C, tp, p, p) order k = ((c*tp + t)*p + i)*p + j
-// (patches path) or, with `frames_order`, in the order
-// k' = ((c*p + i)*tp + t)*p + j the frames producer fills its stages in.
-// The bias is widened exactly to fp32.
+// Weight packing.  Ŵ[e, k] = bf16_rne(W[e, k]), the bias widened exactly to
+// fp32.  Row e of the packed weight holds `ld` columns, in one of three orders:
+//   0  the view(-1, C, tp, p, p) order k = ((c*tp + t)*p + i)*p + j (patches
+//      path), zero past K;
+//   1  k' = ((c*p + i)*tp + t)*p + j, the order the frames producer fills its
+//      stages in, zero past K;
+//   2  slice-major: column t*Kh + (c*p + i)*p + j, slice t of the kernel in its
+//      own block of Kh >= C*p*p columns (zero past C*p*p), for rows that share
+//      one A row across the temporal slices.
 __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias, int b_f32,
                                       uint16_t *wpack, float *bias32, int E, int C, int TP, int P,
-                                      int Kpad, int frames_order) {
+                                      int ld, int order, int Kh) {
     const int K = C * TP * P * P;
-    const int64_t total = (int64_t)E * Kpad;
+    const int64_t total = (int64_t)E * ld;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t e = idx / Kpad;
-        const int kd = (int)(idx - e * Kpad);
-        uint16_t v = 0;
-        if (kd < K) {
-            int k = kd;
-            if (frames_order) {
+        const int64_t e = idx / ld;
+        const int kd = (int)(idx - e * ld);
+        int k = -1;
+        if (order == 0) {
+            if (kd < K) k = kd;
+        } else if (order == 1) {
+            if (kd < K) {
                 const int j = kd % P, t = (kd / P) % TP, ci = kd / (P * TP);
                 const int c = ci / P, i = ci % P;
                 k = ((c * TP + t) * P + i) * P + j;
             }
+        } else {
+            const int t = kd / Kh, kk = kd - t * Kh;
+            if (t < TP && kk < C * P * P) {
+                const int j = kk % P, i = (kk / P) % P, c = kk / (P * P);
+                k = ((c * TP + t) * P + i) * P + j;
+            }
+        }
+        uint16_t v = 0;
+        if (k >= 0) {
             if (w_f32) {
                 const __nv_bfloat16 b = __float2bfloat16_rn(reinterpret_cast<const float *>(w)[e * K + k]);
                 v = *reinterpret_cast<const uint16_t *>(&b);
@@ -993,79 +1075,86 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
     }
 }
 
-// Staged frames path, first half: the normalised patch rows A[N, K] written
-// once, in the frames k order k' = ((c*p + i)*tp + t)*p + j that the
-// frames-order weight uses, for the TMA-fed contraction to read back.  Each
-// CTA owns 128 rows; each thread owns MAXIT (row, word) units exactly as the
-// fused producer does (coalesced 32-bit loads along image rows), walks the
-// (c, i) pairs four at a time, and stores the normalised words -- once per
-// temporal slice, the same word twice when the row's item is a single frame.
-template <int PT, int NORM, bool DUPALL>
-__global__ void __launch_bounds__(256) pe_prep_kernel(const __grid_constant__ FwdParams P, uint16_t *A) {
-    constexpr int p = PT, ws = p / 2, units = kBM * ws, kThr = 256;
-    constexpr int MAXIT = (units + kThr - 1) / kThr;
-    const int64_t m0 = (int64_t)blockIdx.x * kBM;
+// Staged frames path, prepare step: normalised patch rows written once for
+// the TMA-fed contraction, through shared memory so that both sides of the
+// copy are coalesced.  A CTA owns kPrepRows consecutive output rows and one
+// (row, word) unit per thread; consecutive threads read consecutive words of
+// one image row.  Each thread walks the channels, loads its word of the p image
+// rows of every temporal slice, normalises them and writes them into the CTA's
+// row block in shared memory; one bulk copy then stores the contiguous block of
+// rows.
+//   SHARED  single-frame rows in the slice layout A[N, Kh], column
+//           (c*p + i)*p + j, zero up to Kh (the weight is slice-major);
+//   else    A[N, K] in the frames order k' = ((c*p + i)*tp + t)*p + j, the
+//           last frame repeated where a temporal patch runs past T.
+constexpr int kPrepRows = 32;
+
+template <int PT, int NORM, bool SHARED>
+__global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const __grid_constant__ FwdParams P,
+                                                                        uint16_t *A, int row_elems) {
+    constexpr int p = PT, ws = p / 2, NT = SHARED ? 1 : 2;
+    extern __shared__ __align__(128) uint8_t prep_smem[];
+    const int64_t m0 = (int64_t)blockIdx.x * kPrepRows;
+    const int64_t left = P.N - m0;
+    const int rows = left < kPrepRows ? (int)left : kPrepRows;
     const int nci = P.C * p;
-    const int K = P.K;
-    const char *src[MAXIT];
-    uint16_t *dst[MAXIT];
-    int32_t sW[MAXIT], sHW[MAXIT], sT1[MAXIT];
-    uint32_t rok = 0, dup = 0;
-#pragma unroll
-    for (int v = 0; v < MAXIT; ++v) {
-        const int u = threadIdx.x + kThr * v;
-        src[v] = nullptr;
-        dst[v] = nullptr;
-        sW[v] = sHW[v] = sT1[v] = 0;
-        if (u >= units) continue;
-        int r, jw;
-        unit_to_row_word(u, ws, P.merge, r, jw);
-        if (m0 + r >= P.N) continue;
+    int r, jw;
+    unit_to_row_word<kPrepRows>((int)threadIdx.x, ws, P.merge, r, jw);
+    const uint32_t srow = smem_addr(prep_smem) + (uint32_t)(r * row_elems * 2);
+    if (r < rows) {
         const RowSrc rs = locate_row(P, m0 + r, 2);
-        src[v] = rs.base + 4 * jw;
-        dst[v] = A + (m0 + r) * (int64_t)K + 2 * jw;
-        sW[v] = rs.W * 2;
-        sHW[v] = rs.HW * 2;
-        sT1[v] = rs.tmax > 0 ? rs.CHW * 2 : 0;
-        rok |= 1u << v;
-        if (rs.tmax == 0) dup |= 1u << v;
-    }
-    constexpr int NT = DUPALL ? 1 : 2;
-    for (int ci0 = 0; ci0 < nci; ci0 += 4) {
-        uint32_t raw[4][NT][MAXIT];
+        const char *src = rs.base + 4 * jw;
+        const int sW = rs.W * 2, sHW = rs.HW * 2;
+        const int sT1 = (!SHARED && rs.tmax > 0) ? rs.CHW * 2 : 0;
+        // One channel (p image rows, every temporal slice) per register buffer;
+        // the loads of channel c + 1 are in flight while channel c is stored.
+        uint32_t raw[2][NT][p];
+        auto load = [&](const int b, const int c) {
+            const char *a = src + (int64_t)c * sHW;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int ci = ci0 + q;
-            const int c = ci / p, i = ci - (ci / p) * p;
-#pragma unroll
-            for (int v = 0; v < MAXIT; ++v) {
-#pragma unroll
-                for (int t = 0; t < NT; ++t) raw[q][t][v] = 0u;
-                if (ci < nci && (rok >> v & 1u)) {
-                    const char *a = src[v] + (int64_t)c * sHW[v] + (int64_t)i * sW[v];
-                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[q][0][v]) : "l"(a));
-                    if constexpr (!DUPALL) {
-                        if (sT1[v] != 0)
-                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[q][NT - 1][v]) : "l"(a + sT1[v]));
-                    }
+            for (int i = 0; i < p; ++i) {
+                asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][0][i]) : "l"(a + (int64_t)i * sW));
+                if constexpr (!SHARED) {
+                    raw[b][NT - 1][i] = 0u;
+                    if (sT1 != 0)
+                        asm volatile("ld.global.nc.b32 %0, [%1];"
+                                     : "=r"(raw[b][NT - 1][i]) : "l"(a + (int64_t)i * sW + sT1));
                 }
             }
-        }
+        };
+        auto store = [&](const int b, const int c) {
+            const NormConst nc = norm_const(P, c);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int ci = ci0 + q;
-            if (ci >= nci) break;
-            const NormConst nc = norm_const(P, ci / p);
-#pragma unroll
-            for (int v = 0; v < MAXIT; ++v) {
-                if (!(rok >> v & 1u)) continue;
-                const uint32_t w0 = norm_word<NORM>(raw[q][0][v], nc);
-                const uint32_t w1 = (DUPALL || (dup >> v & 1u)) ? w0 : norm_word<NORM>(raw[q][NT - 1][v], nc);
-                uint16_t *d = dst[v] + (int64_t)ci * (2 * p);   // k' of (c, i, t = 0, j)
-                *reinterpret_cast<uint32_t *>(d) = w0;
-                *reinterpret_cast<uint32_t *>(d + p) = w1;
+            for (int i = 0; i < p; ++i) {
+                const int ci = c * p + i;
+                const uint32_t w0 = norm_word<NORM>(raw[b][0][i], nc);
+                if constexpr (SHARED) {
+                    sts32(srow + (uint32_t)((ci * p + 2 * jw) * 2), w0);
+                } else {
+                    const uint32_t w1 = sT1 ? norm_word<NORM>(raw[b][NT - 1][i], nc) : w0;
+                    sts32(srow + (uint32_t)((ci * 2 * p + 2 * jw) * 2), w0);
+                    sts32(srow + (uint32_t)((ci * 2 * p + p + 2 * jw) * 2), w1);
+                }
             }
+        };
+        const int C = P.C;
+        load(0, 0);
+        for (int c = 0; c < C; c += 2) {
+            if (c + 1 < C) load(1, c + 1);
+            store(0, c);
+            if (c + 1 >= C) break;
+            if (c + 2 < C) load(0, c + 2);
+            store(1, c + 1);
         }
+        if (SHARED && 2 * jw < row_elems - nci * p)   // zero columns up to Kh
+            sts32(srow + (uint32_t)((nci * p + 2 * jw) * 2), 0u);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0 && rows > 0) {
+        bulk_store(A + m0 * row_elems, smem_addr(prep_smem), (uint32_t)(rows * row_elems * 2));
+        bulk_commit();
+        bulk_wait<0>();
     }
 }
 
