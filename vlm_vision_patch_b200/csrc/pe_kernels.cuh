@@ -703,14 +703,17 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
     mbar_wait(smem_addr(mma_done), 0, abort);
 }
 
-// Shared-slice issue (kAModeTmaShared): ring slot s holds the A tile of
-// in-slice k in [64s, 64s + 64) and the weight tiles of slice 0 and slice 1 at
-// the same k; each A k-step is issued against both, so the single-frame rows
-// are fetched once for the two temporal slices they stand for.
-__device__ __forceinline__ void mma_issue_shared(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring,
-                                                 uint64_t *full_b, uint64_t *empty_b, uint64_t *tfull,
-                                                 uint64_t *tempty, uint64_t *mma_done, uint32_t tmem_base,
-                                                 volatile int *abort) {
+// Issue loop of the TMA-fed modes: ring slot s holds one A tile (64 k) and
+// SLICES weight tiles; every stage is 4 k-steps, each issued once per slice,
+// unrolled so that the issuing thread spends a few instructions per MMA and
+// keeps the tensor pipe fed.  SLICES == 2 (kAModeTmaShared): the A tile holds
+// in-slice k of single-frame rows and slot s also holds the weight tiles of
+// slice 0 and slice 1 at the same k, so the rows are fetched once for the two
+// temporal slices they stand for.
+template <int SLICES>
+__device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring, uint64_t *full_b,
+                                              uint64_t *empty_b, uint64_t *tfull, uint64_t *tempty,
+                                              uint64_t *mma_done, uint32_t tmem_base, volatile int *abort) {
     constexpr uint16_t kPair = 0x3;
     constexpr uint32_t kSlice1 = (uint32_t)kBStageBytes >> 4;   // slice-1 weight tile, descriptor units
     const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
@@ -735,13 +738,15 @@ __device__ __forceinline__ void mma_issue_shared(const FwdParams &P, uint8_t *a_
                 for (int j = 0; j < 4; ++j) {
                     const uint64_t ad = desc_with_lo(a0, a_lo + 2u * j);
                     mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + 2u * j), idesc, (st | j) ? 1u : 0u);
-                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
+                    if constexpr (SLICES == 2)
+                        mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
                 }
             } else {
                 for (int j = 0; j < kin; ++j) {
                     const uint64_t ad = desc_with_lo(a0, a_lo + 2u * j);
                     mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + 2u * j), idesc, (st | j) ? 1u : 0u);
-                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
+                    if constexpr (SLICES == 2)
+                        mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
                 }
             }
             mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
@@ -899,8 +904,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         // ---------------- MMA issuer (leader CTA only)
         if (leader && lane == 0) {
             constexpr int KSA = (AMODE == kAModeFrames) ? (PT ? PT / 2 : 0) : 4;
-            if constexpr (AMODE == kAModeTmaShared)
-                mma_issue_shared(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
+            if constexpr (kTmaA)
+                mma_issue_tma<AMODE == kAModeTmaShared ? 2 : 1>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty,
+                                                                mma_done, tmem_base, abort);
             else if constexpr (KSA > 0)
                 mma_issue<KSA, AMODE == kAModeFrames, AMODE != kAModeTma>(P, a_ring, b_ring, full_a, empty_a, full_b,
                                                                           empty_b, tfull, tempty, mma_done, tmem_base,
