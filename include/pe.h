@@ -214,14 +214,16 @@ int64_t pe_num_patches(const int32_t *grid_thw, int n);
  * pe_profile_begin / pe_profile_end -- device time of each forward call's
  * contraction kernel (the fused kernel, or the GEMM of the staged path),
  * recorded with a CUDA event pair on the call's stream around that launch.
- * pe_profile_begin creates event pairs for up to max_calls calls (1..1e6) and
- * starts recording; pe_profile_end waits for the recorded events, writes the
+ * pe_profile_begin creates event pairs for up to max_calls calls (0..1e6; 0
+ * records no events and only counts launches) and starts recording; pe_profile_end waits for the recorded events, writes the
  * elapsed milliseconds of the first min(*n, recorded) calls to host ms[] and
  * that count to *n, writes to *launches (if not NULL) how many kernels the
  * forward calls launched in the window (the staged frames path launches two
  * per call, every other forward one), then frees the events and stops
  * recording.  Profiling is a measurement aid: it allocates events and must not
- * overlap another profiling window on the same handle.
+ * overlap another profiling window on the same handle.  An event recorded
+ * between two kernels of one call serialises them, so a window with events
+ * runs the staged path a few microseconds slower than a window without.
  * Errors: PE_ERR_INVALID_ARG, PE_ERR_CUDA.
  */
 pe_status pe_profile_begin(pe_handle *h, int max_calls);

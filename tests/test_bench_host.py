@@ -1,0 +1,75 @@
+"""Host logic of bench.py's multi-rank run, on CPU: world_size-2 gloo ranks
+(127.0.0.1 rendezvous) agree on the slowest rank's time, and the whole-job
+value counts every rank's units over that time (weak scaling).  Also the
+reference arm's rank rule: only rank 0 works and prints."""
+import io
+import contextlib
+import json
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    local_ms = [12.5, 40.0][rank]
+    m = bench.max_over_ranks(local_ms, dist, "cpu")
+    v = bench.weak_scaling_value(1000, 4, world, m)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, m, v))
+
+
+def test_two_gloo_ranks_agree_on_slowest_time_and_weak_scaling_value():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, m, v in got:
+        assert m == 40.0
+        assert v == pytest.approx(1000 * 4 * 2 / 0.040)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.weak_scaling_value(10, 2, 1, 20.0) == pytest.approx(1000.0)
+
+
+def test_reference_arm_other_ranks_exit_without_output():
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        ns = type("A", (), dict(workload="image_224x896", ref_rows=8, steps=1, warmup=3))()
+        assert bench.run_reference(ns, 1, 2) == 0
+    assert buf.getvalue() == ""
+
+
+def test_reference_arm_prints_one_line_on_rank0():
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        assert bench.main(["--impl", "reference", "--workload", "image_224x896", "--ref-rows", "8",
+                           "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(buf.getvalue().strip())
+    assert line["impl"] == "reference" and line["unit"] == "patches/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0

@@ -145,17 +145,35 @@ int choose_bn(int64_t N, int E, int num_pairs, bool gather_fed) {
 
 thread_local pe_handle *t_prof_handle = nullptr;   // handle of the call being launched
 
+// `after_prep`: the kernel reads rows written by the kernel launched just
+// before it on `st`; it is launched with programmatic stream serialisation so
+// that its prologue overlaps that kernel's tail (its TMA issuers wait on
+// griddepcontrol.wait before the first load).
 template <int AMODE, int PT, bool F32IN, int NORM = 2, bool DUPALL = false>
 cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensorMap &tx, const CUtensorMap &to,
-                       size_t smem, int grid, cudaStream_t st) {
+                       size_t smem, int grid, cudaStream_t st, bool after_prep = false) {
     auto kern = pe_fwd_kernel<AMODE, PT, F32IN, NORM, DUPALL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     pe_handle *h = t_prof_handle;
     const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
     if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
-    kern<<<grid, threads_for(AMODE), smem, st>>>(tw, tx, to, P);
-    e = cudaGetLastError();
+    if (after_prep) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3((unsigned)threads_for(AMODE));
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, tw, tx, to, P);
+    } else {
+        kern<<<grid, threads_for(AMODE), smem, st>>>(tw, tx, to, P);
+        e = cudaGetLastError();
+    }
     if (prof) {
         cudaEventRecord(h->prof_ev[2 * h->prof_n + 1], st);
         ++h->prof_n;
@@ -387,10 +405,8 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
         if (cudaMalloc(&h->stage_rows, need) != cudaSuccess) return PE_ERR_CUDA;
         h->stage_bytes = need;
     }
-    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, h->stage_rows, row_elems, st)
-                                 : launch_prep<16>(P, all_scaled, shared, h->stage_rows, row_elems, st);
-    if (h->prof_on) ++h->prof_launches;
-    if (e != cudaSuccess) return PE_ERR_CUDA;
+    // All host-side planning first, so that the two launches leave the host
+    // back to back and the contraction is queued before the prepare kernel ends.
     FwdParams G = P;
     G.x = h->stage_rows;
     G.x_f32 = 0;
@@ -405,9 +421,14 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
         return PE_ERR_CUDA;
     if (!make_out_tmap(&to, out, G.out_f32, G.N, G.E)) return PE_ERR_CUDA;
+    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, h->stage_rows, row_elems, st)
+                                 : launch_prep<16>(P, all_scaled, shared, h->stage_rows, row_elems, st);
+    if (h->prof_on) ++h->prof_launches;
+    if (e != cudaSuccess) return PE_ERR_CUDA;
     if (shared)
-        return finish(launch_fwd<kAModeTmaShared, 0, false>(h->tmap_wt[bn_index(G.bn)], G, tx, to, smem, grid, st));
-    return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st));
+        return finish(
+            launch_fwd<kAModeTmaShared, 0, false>(h->tmap_wt[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
+    return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
 }
 
 pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st,
@@ -754,7 +775,7 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
 }
 
 pe_status pe_profile_begin(pe_handle *h, int max_calls) {
-    if (!h || max_calls < 1 || max_calls > 1000000) return PE_ERR_INVALID_ARG;
+    if (!h || max_calls < 0 || max_calls > 1000000) return PE_ERR_INVALID_ARG;
     DeviceGuard g(h->dev);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
     h->prof_ev.assign((size_t)2 * max_calls, nullptr);

@@ -872,6 +872,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         // thread's bulk copies are serviced one after another, so several
         // issuing warps keep several copies in flight.
         if (lane == 0 && iss < n_iss) {
+            // The A rows may come from the kernel launched just before this
+            // one (the staged prepare step): nothing is loaded before it ends.
+            griddep_wait();
             const uint64_t pol_w = l2_policy_evict_last();
             const uint64_t pol_x = l2_policy_evict_first();
             const uint32_t b_bytes = (uint32_t)(P.bn / 2) * kBK * 2;
@@ -1100,6 +1103,7 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
                                                                         uint16_t *A, int row_elems) {
     constexpr int p = PT, ws = p / 2, NT = SHARED ? 1 : 2;
     extern __shared__ __align__(128) uint8_t prep_smem[];
+    griddep_launch_dependents();   // the contraction may start its prologue
     const int64_t m0 = (int64_t)blockIdx.x * kPrepRows;
     const int64_t left = P.N - m0;
     const int rows = left < kPrepRows ? (int)left : kPrepRows;
