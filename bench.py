@@ -62,7 +62,11 @@ def load_peaks():
 # launch, from an ncu capture, keyed by workload and path, together with the
 # SHA-256 of the kernel sources it was taken on.  A changed kernel invalidates
 # the figure (reported as null) until it is captured again.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/pe_fwd_kernel_grouped_16_images.md, profiles/pe_fwd_kernel_long_video_64x896.md
+    ("grouped_16_images", "staged"): {"bytes": 108142080 + 97811200, "kernel_sha": "4d18c8dc51006a52"},
+    ("long_video_64x896", "staged"): {"bytes": 515314176 + 281386240, "kernel_sha": "4d18c8dc51006a52"},
+}
 KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh")
 
 

@@ -158,7 +158,7 @@ cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensor
     pe_handle *h = t_prof_handle;
     const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
     if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
-    if (after_prep) {
+    if (after_prep && !prof) {   // an event between the two kernels serialises them anyway
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid);
         cfg.blockDim = dim3((unsigned)threads_for(AMODE));
