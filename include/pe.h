@@ -136,13 +136,21 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
  *              README §3.2 PatchMerger and §4.1; Qwen2.5VL语言模型 MRoPE example:
  *              merged grid row-major, h outer).  gh and gw must be multiples of m.
  *   out      : dev [gt*gh*gw, E] of dtype out_dt.
- * Requires p even and p <= PE_MAX_PATCH.  Two execution paths give identical
- * results: the fused path (one kernel; the normalised [N, K] patch matrix only
- * ever exists tile by tile in shared memory) and, for bf16 frames with tp = 2,
- * p in {14, 16} and at least 8192 patches, the staged path (a prepare kernel
- * writes the normalised patch matrix once into the handle's grow-only
- * workspace, then the TMA-fed contraction reads it back).  The environment
- * variable PE_FRAMES_PATH=fused|staged overrides the choice.
+ * Requires p even and p <= PE_MAX_PATCH.  Three execution paths, all within
+ * the same tolerance of the exact result:
+ *   fused    one kernel; the normalised [N, K] patch matrix only ever exists
+ *            tile by tile in shared memory (small inputs, fp32 frames, other p);
+ *   staged   (default for bf16 frames with tp = 2, p in {14, 16} and at least
+ *            8192 patches) a prepare kernel writes the normalised rows once
+ *            into the handle's grow-only workspace, then the TMA-fed
+ *            contraction reads them back;
+ *   streamed one cooperative kernel: producer warps write the same rows while
+ *            the contraction consumes the completed row blocks (an option:
+ *            slower than staged on B200).
+ * When every item is a single frame, the streamed and staged paths store one
+ * temporal slice per row and multiply it by both temporal slices of the
+ * weight.  The environment variable PE_FRAMES_PATH=fused|streamed|staged
+ * overrides the choice.
  * Errors: as pe_forward_patches plus PE_ERR_SHAPE, PE_ERR_UNSUPPORTED.
  */
 pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H,

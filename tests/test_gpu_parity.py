@@ -335,12 +335,13 @@ def test_error_paths():
 
 @pytest.mark.parametrize("case", ["images", "video_odd_T", "mixed", "images_p16_raster"])
 def test_staged_and_fused_paths_agree(case, monkeypatch):
-    """Both frames paths must be within tolerance of the oracle.  Where some
-    item has more than one frame, both run the contraction in the same k order
+    """All three frames paths (fused kernel, staged pair, streamed kernel) must
+    be within tolerance of the oracle.  Where some item has more than one
+    frame, the fused and staged paths run the contraction in the same k order
     and tile shape, so their outputs must also be bit-identical.  When every
-    item is a single frame the staged path stores one temporal slice per row
-    and meets it with both slices of the weight (a different summation order),
-    so only the tolerance applies."""
+    item is a single frame, the staged and streamed paths both store one
+    temporal slice per row and meet it with both slices of the weight in the
+    same order, so those two must be bit-identical."""
     C, tp, p, E, merge = 3, 2, 14, 1280, 2
     if case == "images":
         grids = [(1, 12, 18), (1, 20, 10), (1, 8, 8)]
@@ -362,13 +363,15 @@ def test_staged_and_fused_paths_agree(case, monkeypatch):
                             workloads.normal((E,), 122, std=0.02, dtype=torch.bfloat16), torch.bfloat16,
                             merge=merge, items=items, mean=workloads.CLIP_MEAN, std=workloads.CLIP_STD)
     outs = {}
-    for path in ("fused", "staged"):
+    for path in ("fused", "staged", "streamed"):
         monkeypatch.setenv("PE_FRAMES_PATH", path)
         _, out, ref, mag = _run_frames(wl)
         outs[path] = out
         assert_within_tolerance(out, ref, mag, what=f"{case} {path}")
     if any(T > 1 for T in Ts):
         assert torch.equal(outs["fused"], outs["staged"])
+    else:   # staged and streamed: the same rows, tile shape and summation order
+        assert torch.equal(outs["staged"], outs["streamed"])
     if case == "images":   # fp32 output from the staged path
         _, out, ref, mag = _run_frames(wl, out_dtype=torch.float32)
         assert out.dtype == torch.float32

@@ -45,6 +45,11 @@ struct pe_handle {
     // staged frames path: normalised patch rows [N, K] (grow-only)
     uint16_t *stage_rows = nullptr;
     size_t stage_bytes = 0;
+    // streamed frames path: two arrays of per-M-block ready counters, used by
+    // alternate calls (each call zeroes the other one)
+    uint32_t *ready = nullptr;
+    int ready_cap = 0;
+    int ready_parity = 0;
     // profiling: one event pair per call around the contraction kernel
     std::vector<cudaEvent_t> prof_ev;
     int prof_cap = 0, prof_n = 0;
@@ -149,26 +154,38 @@ thread_local pe_handle *t_prof_handle = nullptr;   // handle of the call being l
 // before it on `st`; it is launched with programmatic stream serialisation so
 // that its prologue overlaps that kernel's tail (its TMA issuers wait on
 // griddepcontrol.wait before the first load).
+// `coop`: every CTA must be resident at once (CTAs wait for rows that other
+// CTAs produce): cooperative launch.
 template <int AMODE, int PT, bool F32IN, int NORM = 2, bool DUPALL = false>
 cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensorMap &tx, const CUtensorMap &to,
-                       size_t smem, int grid, cudaStream_t st, bool after_prep = false) {
+                       size_t smem, int grid, cudaStream_t st, bool after_prep = false, bool coop = false) {
     auto kern = pe_fwd_kernel<AMODE, PT, F32IN, NORM, DUPALL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     pe_handle *h = t_prof_handle;
     const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
     if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
-    if (after_prep && !prof) {   // an event between the two kernels serialises them anyway
+    const bool pdl = after_prep && !prof;   // an event between the two kernels serialises them anyway
+    if (pdl || coop) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid);
         cfg.blockDim = dim3((unsigned)threads_for(AMODE));
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchAttribute at[2];
+        int na = 0;
+        if (pdl) {
+            at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            at[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        if (coop) {
+            at[na].id = cudaLaunchAttributeCooperative;
+            at[na].val.cooperative = 1;
+            ++na;
+        }
         cfg.attrs = at;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = na;
         e = cudaLaunchKernelEx(&cfg, kern, tw, tx, to, P);
     } else {
         kern<<<grid, threads_for(AMODE), smem, st>>>(tw, tx, to, P);
@@ -361,12 +378,19 @@ bool staged_eligible(const pe_handle *h, int f_dt) {
     return f_dt == PE_BF16 && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
 }
 
-bool want_staged(const pe_handle *h, const FwdParams &P, int f_dt) {
-    if (!staged_eligible(h, f_dt)) return false;
+// Large bf16 frame batches: 0 = fused kernel, 1 = staged pair (the default),
+// 2 = streamed kernel.  PE_FRAMES_PATH=fused|staged|streamed overrides.  The
+// streamed kernel overlaps row production with the contraction but its
+// producer warps' scattered loads and stores slow the contraction down more
+// than the separate prepare kernel costs (measured on B200), so it is not the
+// default.
+int large_path(const pe_handle *h, const FwdParams &P, int f_dt) {
+    if (!staged_eligible(h, f_dt)) return 0;
     const char *e = std::getenv("PE_FRAMES_PATH");
-    if (e && std::strcmp(e, "fused") == 0) return false;
-    if (e && std::strcmp(e, "staged") == 0) return true;
-    return P.N >= kStagedMinRows;
+    if (e && std::strcmp(e, "fused") == 0) return 0;
+    if (e && std::strcmp(e, "staged") == 0) return 1;
+    if (e && std::strcmp(e, "streamed") == 0) return 2;
+    return P.N >= kStagedMinRows ? 1 : 0;
 }
 
 template <int PT, int NORM, bool SHARED>
@@ -431,14 +455,88 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
 }
 
+// Streamed frames path: one cooperative kernel whose producer warps write the
+// normalised rows (slice-major, one slice for single-frame rows, two
+// otherwise) into the handle's row buffer while its TMA-fed pair GEMM consumes
+// the completed M-blocks.
+pe_status run_frames_streamed(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, cudaStream_t st) {
+    const int row_elems = (shared ? 1 : 2) * h->Kh;
+    const size_t need = (size_t)P.N * row_elems * 2;
+    const int64_t mt = (P.N + 2 * kBM - 1) / (2 * kBM);
+    if (mt > INT32_MAX / 2) return PE_ERR_UNSUPPORTED;
+    if (need > h->stage_bytes || mt > h->ready_cap) {
+        if (cudaStreamSynchronize(st) != cudaSuccess) return PE_ERR_CUDA;
+    }
+    if (need > h->stage_bytes) {
+        if (h->stage_rows) cudaFree(h->stage_rows);
+        h->stage_rows = nullptr;
+        h->stage_bytes = 0;
+        if (cudaMalloc(&h->stage_rows, need) != cudaSuccess) return PE_ERR_CUDA;
+        h->stage_bytes = need;
+    }
+    if (mt > h->ready_cap) {
+        if (h->ready) cudaFree(h->ready);
+        h->ready = nullptr;
+        h->ready_cap = 0;
+        const int cap = (int)std::max<int64_t>(mt, 1024);
+        if (cudaMalloc(&h->ready, sizeof(uint32_t) * 2 * (size_t)cap) != cudaSuccess) return PE_ERR_CUDA;
+        if (cudaMemsetAsync(h->ready, 0, sizeof(uint32_t) * 2 * (size_t)cap, st) != cudaSuccess) return PE_ERR_CUDA;
+        h->ready_cap = cap;
+        h->ready_parity = 0;
+    }
+    FwdParams G = P;
+    G.x = h->stage_rows;
+    G.x_f32 = 0;
+    G.x_vec = 1;
+    G.a_rows = h->stage_rows;
+    G.row_elems = row_elems;
+    G.ready = h->ready + (size_t)h->ready_parity * h->ready_cap;
+    G.ready_next = h->ready + (size_t)(h->ready_parity ^ 1) * h->ready_cap;
+    G.n_mblocks = (int)mt;
+    int grid = 0;
+    bool ok = true;
+    plan_tiles(h, G, G.N, false, grid, ok);
+    if (!ok) return PE_ERR_UNSUPPORTED;
+    G.ready_target = (uint32_t)(kStreamProdWarps * 2 * G.n_tiles_n);
+    const size_t smem = plan_pipeline(h, G, shared ? kAModeTmaShared : kAModeTma);
+    if (!shared) {   // both slices of a row in sequence against the slice-major weight
+        G.num_ksteps = row_elems / 16;
+        G.n_b_stages = (G.num_ksteps + 3) / 4;
+        G.n_a_stages = G.n_b_stages;
+    } else {
+        G.num_ksteps = h->Kh / 16;
+        G.n_b_stages = (G.num_ksteps + 3) / 4;
+        G.n_a_stages = G.n_b_stages;
+    }
+    CUtensorMap tx, to;
+    if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
+        return PE_ERR_CUDA;
+    if (!make_out_tmap(&to, out, G.out_f32, G.N, G.E)) return PE_ERR_CUDA;
+    const CUtensorMap &tw = h->tmap_wt[bn_index(G.bn)];
+    h->ready_parity ^= 1;
+    cudaError_t e;
+#define PE_LAUNCH_STREAM(PP, NN)                                                                                    \
+    (shared ? launch_fwd<kAModeTmaStream, PP, false, NN, true>(tw, G, tx, to, smem, grid, st, false, true)          \
+            : launch_fwd<kAModeTmaStream, PP, false, NN, false>(tw, G, tx, to, smem, grid, st, false, true))
+    if (h->p == 14)
+        e = all_scaled ? PE_LAUNCH_STREAM(14, 1) : PE_LAUNCH_STREAM(14, 2);
+    else
+        e = all_scaled ? PE_LAUNCH_STREAM(16, 1) : PE_LAUNCH_STREAM(16, 2);
+#undef PE_LAUNCH_STREAM
+    return finish(e);
+}
+
 pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st,
                      bool allow_staged = true) {
     P.out_f32 = out_dt == PE_F32;
     if (P.N == 0) return PE_OK;
-    if (allow_staged && want_staged(h, P, f_dt)) {
+    const int lp = allow_staged ? large_path(h, P, f_dt) : 0;
+    if (lp != 0) {
         bool all_scaled = true;
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
-        return run_frames_staged(h, P, out, all_scaled, h->tp == 2 && P.all_t1 && h->wpack_t, st);
+        const bool shared = h->tp == 2 && P.all_t1 && h->wpack_t;
+        if (lp == 2) return run_frames_streamed(h, P, out, all_scaled, shared, st);
+        return run_frames_staged(h, P, out, all_scaled, shared, st);
     }
     int grid = 0;
     bool ok = true;
@@ -568,6 +666,7 @@ void pe_destroy(pe_handle *h) {
     if (h->items_dev) cudaFree(h->items_dev);
     if (h->items_pinned) cudaFreeHost(h->items_pinned);
     if (h->stage_rows) cudaFree(h->stage_rows);
+    if (h->ready) cudaFree(h->ready);
     if (h->items_evt) cudaEventDestroy(h->items_evt);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
     delete h;

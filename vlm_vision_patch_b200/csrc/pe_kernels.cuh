@@ -31,6 +31,8 @@ namespace pe {
 constexpr int kThreads = 640;       // 20 warps (A produced by threads)
 constexpr int kThreadsTma = 320;    // 10 warps (A fetched by TMA)
 __host__ __device__ constexpr int threads_for(int amode) { return (amode == 0 || amode == 3) ? kThreadsTma : kThreads; }
+constexpr int kStreamProdWarp0 = 8;   // kAModeTmaStream: warps 8..15 produce rows
+constexpr int kStreamProdWarps = 8;
 constexpr int kBM = 128;           // rows per CTA (pair tile: 256 rows)
 constexpr int kMaxBN = 256;        // largest pair-MMA N
 constexpr int kBK = 64;            // weight K per TMA stage (one 128-byte swizzle row)
@@ -46,8 +48,15 @@ constexpr int kBStageBytes = (kMaxBN / 2) * kBK * 2;   // 16 KB: this CTA's half
 //   kAModeTmaShared    TMA tiles of single-frame rows A[N, Kh] that both temporal
 //                      slices share: every A tile meets the weight tiles of
 //                      slice 0 and slice 1 at the same in-slice k (tp = 2).
-enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2, kAModeTmaShared = 3 };
-__host__ __device__ constexpr bool tma_fed(int amode) { return amode == kAModeTma || amode == kAModeTmaShared; }
+//   kAModeTmaStream    the rows are written by producer warps of the same grid
+//                      into a global buffer in the slice-major layout and read
+//                      back by TMA once their M-block is complete: single-frame
+//                      rows as in kAModeTmaShared (DUPALL), otherwise both
+//                      slices per row against the slice-major weight.
+enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2, kAModeTmaShared = 3, kAModeTmaStream = 4 };
+__host__ __device__ constexpr bool tma_fed(int amode) {
+    return amode == kAModeTma || amode == kAModeTmaShared || amode == kAModeTmaStream;
+}
 
 struct ItemDesc {
     const void *frames;  // [T, C, H, W]
@@ -80,6 +89,13 @@ struct FwdParams {
     int32_t out_f32;
     const float *bias;                // fp32 [E] or nullptr
     int *err;                         // device error word
+    // kAModeTmaStream
+    uint16_t *a_rows;                 // [N, row_elems] rows written by the producers
+    int32_t row_elems;                // slices * Kh
+    uint32_t *ready;                  // per M-block count of finished producer parts (this call)
+    uint32_t *ready_next;             // the next call's counters, zeroed by this call
+    uint32_t ready_target;            // count that marks an M-block complete
+    int32_t n_mblocks;
 };
 
 // ------------------------------------------------------------ row decoding
@@ -703,6 +719,109 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
     mbar_wait(smem_addr(mma_done), 0, abort);
 }
 
+// Streamed frames producer (kAModeTmaStream), warps 8..15 of every CTA.
+//
+// Each pair tile (m, n) of this CTA carries one part of M-block m's rows: the
+// M-block's 256 rows x (row_elems / 8) 16-byte chunks are enumerated chunk-
+// major in warp iterations of 32 rows, and split into 2 * n_tiles_n parts, so
+// that the CTAs of the tiles of an M-block produce it together.  In an
+// iteration each lane assembles one 16-byte chunk (8 columns of the
+// slice-major row: t*Kh + (c*p + i)*p + j) of its row from at most two image
+// row segments (4-byte loads), normalises it and stores it.  After each part a
+// warp adds 1 to the M-block's counter with release semantics; the TMA
+// issuers wait for all 8 * 2 * n_tiles_n counts before loading the block.
+// Producers wait for nothing, so all counts arrive once every CTA runs.
+template <int PT, int NORM, bool DUPALL>
+__device__ __forceinline__ void produce_rows_stream(const FwdParams &P, int pw, int lane, uint32_t rank) {
+    constexpr int p = PT, pp = PT * PT;
+    constexpr int NT = DUPALL ? 1 : 2;   // slices stored per row
+    constexpr int U = 4;                 // chunks in flight per lane
+    const int Kh = P.Kh, qh = Kh / 8, nq = NT * qh;
+    const int C = P.C, cpp = C * pp;
+    const int row_elems = P.row_elems;
+    // The next call's counters: nobody touches them during this call.
+    for (int i = (blockIdx.x * kStreamProdWarps + pw) * 32 + lane; i < P.n_mblocks;
+         i += gridDim.x * kStreamProdWarps * 32)
+        P.ready_next[i] = 0u;
+    const int nparts = 2 * P.n_tiles_n;
+    const int wi = 8 * nq;               // warp iterations per M-block
+    for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+        const int m = tile / P.n_tiles_n, n = tile - m * P.n_tiles_n;
+        const int part = 2 * n + (int)rank;
+        const int it0 = (int)((int64_t)part * wi / nparts), it1 = (int)((int64_t)(part + 1) * wi / nparts);
+        int it = it0 + pw;
+        if (it < it1) {
+            // iterations it, it + 8, ...: one row group of 32 rows for this warp
+            const int64_t row = (int64_t)m * (2 * kBM) + (it & 7) * 32 + lane;
+            const bool live = row < P.N;
+            const char *base0 = nullptr, *base1 = nullptr;
+            int sW = 0, sHW = 0;
+            uint16_t *dst = P.a_rows;
+            if (live) {
+                const RowSrc rs = locate_row(P, row, 2);
+                base0 = rs.base;
+                base1 = rs.tmax > 0 ? rs.base + (int64_t)rs.CHW * 2 : rs.base;
+                sW = rs.W * 2;
+                sHW = rs.HW * 2;
+                dst = P.a_rows + row * row_elems;
+            }
+            for (; it < it1; it += 8 * U) {
+                uint32_t w[U][4];
+                int col[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int itu = it + 8 * u;
+                    col[u] = -1;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) w[u][k] = 0u;
+                    if (itu >= it1) continue;
+                    const int q = itu >> 3;
+                    const int t = (NT == 2 && q >= qh) ? 1 : 0;
+                    const int kk0 = (q - t * qh) * 8;
+                    col[u] = t * Kh + kk0;
+                    if (!live || kk0 >= cpp) continue;
+                    const int c = kk0 / pp, r2 = kk0 - c * pp, i = r2 / p, j0 = r2 - i * p;
+                    const int n1 = (p - j0) < 8 ? (p - j0) : 8;
+                    const int i2 = (i + 1 < p) ? i + 1 : 0, c2 = (i + 1 < p) ? c : c + 1;
+                    const char *bt = t ? base1 : base0;
+                    const char *s1 = bt + (int64_t)c * sHW + (int64_t)i * sW + j0 * 2;
+                    const char *s2 = bt + (int64_t)c2 * sHW + (int64_t)i2 * sW;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (2 * k < n1)
+                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[u][k]) : "l"(s1 + 4 * k));
+                        else if (c2 < C)
+                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[u][k]) : "l"(s2 + (2 * k - n1) * 2));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (col[u] < 0 || !live) continue;
+                    const int kk0 = col[u] >= Kh ? col[u] - Kh : col[u];
+                    if (kk0 < cpp) {
+                        const int c = kk0 / pp, r2 = kk0 - c * pp, j0 = r2 - (r2 / p) * p;
+                        const int n1 = (p - j0) < 8 ? (p - j0) : 8;
+                        const NormConst n1c = norm_const(P, c);
+                        const NormConst n2c = norm_const(P, c + 1 < C ? c + 1 : c);
+                        const bool wrap = (r2 / p) + 1 >= p;   // second segment starts the next channel
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            if (2 * k < n1) w[u][k] = norm_word<NORM>(w[u][k], n1c);
+                            else if (!wrap) w[u][k] = norm_word<NORM>(w[u][k], n1c);
+                            else if (c + 1 < C) w[u][k] = norm_word<NORM>(w[u][k], n2c);
+                        }
+                    }
+                    st_global_v4(dst + col[u], w[u][0], w[u][1], w[u][2], w[u][3]);
+                }
+            }
+        }
+        fence_proxy_async_global();   // this lane's rows visible to TMA readers ...
+        __threadfence();              // ... and ordered before lane 0's release
+        __syncwarp();
+        if (lane == 0) red_release_add(P.ready + m, 1u);
+    }
+}
+
 // Issue loop of the TMA-fed modes: ring slot s holds one A tile (64 k) and
 // SLICES weight tiles; every stage is 4 k-steps, each issued once per slice,
 // unrolled so that the issuing thread spends a few instructions per MMA and
@@ -864,6 +983,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
     // P.n_iss of them issue, and P.n_iss never exceeds a ring depth: an issuer
     // then can never lap a slot, so its parity waits cannot alias.
     const int iss = (warp == 0) ? 0 : (warp == 2 || warp == 3) ? warp - 1
+                  : (AMODE == kAModeTmaStream) ? ((warp == 16 || warp == 17) ? warp - 13 : -1)
                   : (kTmaA && warp >= 8 && warp < 10) ? warp - 5 : -1;
     const int n_iss = P.n_iss;
     if (iss >= 0) {
@@ -882,14 +1002,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             const uint32_t fb0 = mapa_shared(smem_addr(&full_b[0]), 0);
             int g = 0;
             bool ok = true;
+            int ready_m = -1;
             for (int tile = blockIdx.x >> 1; tile < P.num_tiles && ok; tile += gridDim.x >> 1) {
                 const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
                 for (int kb = 0; kb < P.n_b_stages && ok; ++kb, ++g) {
                     if (g % n_iss != iss) continue;
+                    if (AMODE == kAModeTmaStream && m_blk != ready_m) {
+                        // rows of this M-block come from producer warps across the grid
+                        if (!wait_count(P.ready + m_blk, P.ready_target, abort)) { ok = false; break; }
+                        fence_proxy_async_global();
+                        ready_m = m_blk;
+                    }
                     // In the TMA-fed path A and weight share ring slot and barriers.
                     const int bs = g % P.nb;
                     if (!mbar_wait(smem_addr(&empty_b[bs]), ((g / P.nb) & 1) ^ 1, abort)) { ok = false; break; }
-                    constexpr uint32_t kSlices = (AMODE == kAModeTmaShared) ? 2u : 1u;
+                    constexpr uint32_t kSlices =
+                        (AMODE == kAModeTmaShared || (AMODE == kAModeTmaStream && DUPALL)) ? 2u : 1u;
                     if (leader)
                         mbar_arrive_expect_tx(smem_addr(&full_b[bs]), 2 * (kSlices * b_bytes + (kTmaA ? a_bytes : 0u)));
                     if (kTmaA)
@@ -898,7 +1026,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     const uint32_t bdst = smem_addr(b_ring + (size_t)bs * P.b_slot_bytes);
                     const int wrow = n_blk * P.bn + (int)rank * (P.bn / 2);
                     tma_load_2d_pair(bdst, &tmap_w, fb0 + 8u * bs, kb * kBK, wrow, pol_w);
-                    if (AMODE == kAModeTmaShared)
+                    if (kSlices == 2)
                         tma_load_2d_pair(bdst + kBStageBytes, &tmap_w, fb0 + 8u * bs, P.Kh + kb * kBK, wrow, pol_w);
                 }
             }
@@ -908,8 +1036,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         if (leader && lane == 0) {
             constexpr int KSA = (AMODE == kAModeFrames) ? (PT ? PT / 2 : 0) : 4;
             if constexpr (kTmaA)
-                mma_issue_tma<AMODE == kAModeTmaShared ? 2 : 1>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty,
-                                                                mma_done, tmem_base, abort);
+                mma_issue_tma<(AMODE == kAModeTmaShared || (AMODE == kAModeTmaStream && DUPALL)) ? 2 : 1>(
+                    P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
             else if constexpr (KSA > 0)
                 mma_issue<KSA, AMODE == kAModeFrames, AMODE != kAModeTma>(P, a_ring, b_ring, full_a, empty_a, full_b,
                                                                           empty_b, tfull, tempty, mma_done, tmem_base,
@@ -975,7 +1103,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             tc_fence_after();
             const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
             const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
-            if constexpr (kTmaA) {
+            if constexpr (kTmaA && AMODE != kAModeTmaStream) {
                 // registers to spare: the next chunk's TMEM load overlaps this chunk's work
                 uint32_t va[32], vb[32];
                 tmem_ld_32x32b_x32(tbase, va);
@@ -1002,6 +1130,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         }
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
+    } else if (AMODE == kAModeTmaStream && warp >= kStreamProdWarp0 && warp < kStreamProdWarp0 + kStreamProdWarps) {
+        // ---------------- row producers (both CTAs)
+        if constexpr (AMODE == kAModeTmaStream && PT != 0)
+            produce_rows_stream<PT, NORM, DUPALL>(P, warp - kStreamProdWarp0, lane, rank);
     } else if (warp >= 8 && !kTmaA) {
         // ---------------- A producers (both CTAs)
         ProdCtx X;
