@@ -111,6 +111,23 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
 pe_status pe_set_norm(pe_handle *h, const float *mean, const float *std);
 
 /*
+ * pe_set_temporal_fold -- opt-in temporal folding for single-frame items.
+ * A single image is duplicated to tp = 2 frames before the Conv3d (patch详解
+ * §4.5 counts ceil(1/2) = 1 temporal patch), so both temporal slices of the
+ * kernel multiply the same pixels: out = x̂ · (Ŵ[:,:,0] + Ŵ[:,:,1]).  With
+ * folding enabled, frames calls whose items all have T == 1 (bf16 frames,
+ * p in {14, 16}) multiply by the folded weight bf16_rne(fp32(Ŵ0 + Ŵ1)) once,
+ * which halves the contraction (K = C*p*p instead of C*tp*p*p).  This changes
+ * the rounding of the result: each weight term carries one more bf16 rounding,
+ * at most 2^-8 of |Ŵ0 + Ŵ1|, so the worst-case bound is 2^-8 * sum |x̂ ŵ|
+ * rather than the unfolded path's fp32-accumulation bound.  Other calls (and
+ * pe_forward_frames_grouped_noalloc, which never uses the workspace that the
+ * folded path needs) are unaffected.  enable = 0 (the default) or 1.  Errors: PE_ERR_INVALID_ARG,
+ * PE_ERR_UNSUPPORTED (tp != 2).
+ */
+pe_status pe_set_temporal_fold(pe_handle *h, int enable);
+
+/*
  * pe_forward_patches -- out = x @ W^T (+ bias) on already patchified rows.
  *   x   : dev [N, K] of dtype x_dt (PE_BF16 or PE_F32), rows in
  *         view(-1, C, tp, p, p) order as the Qwen2-VL processor emits

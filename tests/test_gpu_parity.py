@@ -376,3 +376,82 @@ def test_staged_and_fused_paths_agree(case, monkeypatch):
         _, out, ref, mag = _run_frames(wl, out_dtype=torch.float32)
         assert out.dtype == torch.float32
         assert_within_tolerance(out, ref, mag, what=f"{case} staged fp32 out")
+
+
+# ------------------------------------------------------------ temporal folding
+
+def _folded_weight(w: torch.Tensor) -> torch.Tensor:
+    """The weight the folded path multiplies single frames by, as a Conv3d
+    weight of the original shape: bf16_rne(fp32(Ŵ0 + Ŵ1)) in slice 0, zeros in
+    slice 1 (a single frame is duplicated to both slices, patch详解 §4.5)."""
+    wb = w.to(torch.bfloat16).float()
+    f = (wb[:, :, 0] + wb[:, :, 1]).to(torch.bfloat16).float()
+    out = torch.zeros_like(wb)
+    out[:, :, 0] = f
+    return out
+
+
+@pytest.mark.parametrize("case", ["image_224x896", "grouped_small", "p16_raster_bias", "grouped_16_sampled"])
+def test_temporal_fold(case):
+    """Opt-in folding: (1) within the parity tolerance of the oracle run with the
+    folded weight (the same products, any summation order); (2) within the
+    folding bound 2^-8 * sum|x̂ ŵ| (+ fp32 accumulation and one bf16 ulp) of the
+    exact, unfolded result."""
+    rows = None
+    if case == "image_224x896":
+        wl = workloads.image_224x896()
+    elif case == "grouped_16_sampled":
+        wl = workloads.grouped_16_images()
+        offs = np.cumsum([0] + [g[0] * g[1] * g[2] for g in (it.grid for it in wl.items)])
+        rows = sample_rows(wl.N, 600, 77, extra=offs[1:-1])
+    else:
+        C, tp = 3, 2
+        if case == "grouped_small":
+            p, E, merge, bias = 14, 1280, 2, None
+            grids = [(1, 12, 18), (1, 20, 10), (1, 8, 8)]
+        else:
+            p, E, merge = 16, 1152, 1
+            grids = [(1, 7, 9), (1, 5, 11)]
+            bias = workloads.normal((E,), 132, std=0.02, dtype=torch.bfloat16)
+        items = [workloads.Item(workloads.uniform01((1, C, g[1] * p, g[2] * p), 130 + i), g)
+                 for i, g in enumerate(grids)]
+        wl = workloads.Workload("fold_" + case, E, C, tp, p,
+                                workloads.normal((E, C, tp, p, p), 131, std=0.02, dtype=torch.bfloat16),
+                                bias, torch.bfloat16, merge=merge, items=items,
+                                mean=workloads.CLIP_MEAN, std=workloads.CLIP_STD)
+    pe = _pe((wl.E, wl.C, wl.tp, wl.p), wl.weight, wl.bias, wl.mean, wl.std)
+    pe.set_temporal_fold(True)
+    frames = [it.frames.to(DEV) for it in wl.items]
+    out = pe.forward_frames_grouped(frames, [it.grid for it in wl.items], wl.merge)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    mask = None if rows is None else mask_of(rows, wl.N)
+    its = [(it.frames, it.grid) for it in wl.items]
+    ref_f, mag_f = oracle.conv3d_grouped(its, wl.merge, wl.mean, wl.std, _folded_weight(wl.weight), wl.bias,
+                                         wl.C, wl.tp, wl.p, row_mask=mask)
+    assert_within_tolerance(out, ref_f, mag_f, rows=rows, what=f"{case} folded-weight oracle")
+    ref, mag = oracle.conv3d_grouped(its, wl.merge, wl.mean, wl.std, wl.weight, wl.bias,
+                                     wl.C, wl.tp, wl.p, row_mask=mask)
+    assert_within_tolerance(out, ref, mag, rows=rows, what=f"{case} exact oracle, folding bound",
+                            rel=2.0 ** -8 + 1e-3)
+
+
+def test_temporal_fold_leaves_video_and_off_state_alone():
+    """Folding applies to single-frame items only; a video item, or the flag off,
+    gives the unfolded result bit for bit."""
+    C, tp, p, E = 3, 2, 14, 256
+    w = workloads.normal((E, C, tp, p, p), 140, std=0.02, dtype=torch.bfloat16)
+    vid = workloads.uniform01((4, C, 8 * p, 6 * p), 141).to(DEV)
+    img = workloads.uniform01((1, C, 8 * p, 6 * p), 142).to(DEV)
+    pe = _pe((E, C, tp, p), w, None, workloads.CLIP_MEAN, workloads.CLIP_STD)
+    base_v = pe.forward_frames(vid, (2, 8, 6), 2)
+    base_i = pe.forward_frames(img, (1, 8, 6), 2)
+    pe.set_temporal_fold(True)
+    fold_v = pe.forward_frames(vid, (2, 8, 6), 2)
+    fold_i = pe.forward_frames(img, (1, 8, 6), 2)
+    pe.set_temporal_fold(False)
+    again_i = pe.forward_frames(img, (1, 8, 6), 2)
+    torch.cuda.synchronize()
+    assert torch.equal(base_v, fold_v)
+    assert torch.equal(base_i, again_i)
+    assert not torch.equal(base_i, fold_i)   # the folded path really ran

@@ -74,6 +74,11 @@ class PatchEmbed:
     def set_norm(self, mean: Sequence[float], std: Sequence[float]) -> None:
         B.pe_set_norm(self.h, mean, std)
 
+    def set_temporal_fold(self, enable: bool) -> None:
+        """Opt-in: single-frame items use the summed temporal slices of the weight
+        (half the contraction; one more bf16 rounding per weight term)."""
+        B.pe_set_temporal_fold(self.h, enable)
+
     def last_error(self) -> int:
         return B.pe_last_error(self.h)
 

@@ -29,6 +29,7 @@ EXPORTS = (
     "pe_create", "pe_set_weight", "pe_set_norm", "pe_forward_patches", "pe_forward_frames",
     "pe_forward_frames_grouped", "pe_forward_frames_grouped_noalloc", "pe_patchify", "pe_num_patches", "pe_last_error",
     "pe_status_string", "pe_destroy", "pe_device", "pe_profile_begin", "pe_profile_end",
+    "pe_set_temporal_fold",
 )
 
 
@@ -59,6 +60,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_create": ([i32, i32, i32, i32, i32, ctypes.POINTER(vp)], i32),
         "pe_set_weight": ([vp, vp, i32, vp, i32, vp], i32),
         "pe_set_norm": ([vp, f32p, f32p], i32),
+        "pe_set_temporal_fold": ([vp, i32], i32),
         "pe_forward_patches": ([vp, vp, i32, i64, vp, i32, vp], i32),
         "pe_forward_frames": ([vp, vp, i32, i32, i32, i32, i32p, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
@@ -125,6 +127,10 @@ def pe_set_weight(h: int, w_ptr: int, w_dt: int, bias_ptr: Optional[int], b_dt: 
 
 def pe_set_norm(h: int, mean: Sequence[float], std: Sequence[float]) -> None:
     _check("pe_set_norm", load().pe_set_norm(h, _f32arr(mean), _f32arr(std)))
+
+
+def pe_set_temporal_fold(h: int, enable: bool) -> None:
+    _check("pe_set_temporal_fold", load().pe_set_temporal_fold(h, int(bool(enable))))
 
 
 def pe_forward_patches(h: int, x_ptr: int, x_dt: int, N: int, out_ptr: int, out_dt: int, stream: int) -> None:

@@ -29,6 +29,8 @@ struct pe_handle {
     uint16_t *wpack = nullptr;  // dev [E, Kpad] bf16, view(-1, C, tp, p, p) k order
     uint16_t *wpack_f = nullptr; // dev [E, Kpad] bf16, k order of the frames producer
     uint16_t *wpack_t = nullptr; // dev [E, 2*Kh] bf16, slice-major (tp == 2 only)
+    uint16_t *wpack_fold = nullptr; // dev [E, Kh] bf16, both slices summed (tp == 2 only)
+    bool fold = false;          // pe_set_temporal_fold
     float *bias = nullptr;      // dev [E] fp32 (has_bias)
     int *err = nullptr;         // dev error word
     float mean[4] = {0, 0, 0, 0};
@@ -36,6 +38,7 @@ struct pe_handle {
     CUtensorMap tmap_w[3];      // weight boxes of 32, 64, 128 rows (half a pair tile)
     CUtensorMap tmap_wf[3];     // same for the frames-order weight
     CUtensorMap tmap_wt[3];     // same for the slice-major weight
+    CUtensorMap tmap_wfold[3];  // same for the folded weight
     int num_sms = 0;
     int smem_optin = 0;
     // item table for grouped calls beyond PE_INLINE_ITEMS
@@ -249,19 +252,25 @@ void fill_common(const pe_handle *h, FwdParams &P) {
 }
 
 // Ring depths and per-tile stage counts; returns the dynamic shared memory size.
-size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode) {
-    P.num_ksteps = (P.K + 15) / 16;
+// `kcols`: columns of the TMA-fed A rows (default K).
+size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode, int kcols = -1) {
+    if (kcols < 0) kcols = P.K;
+    P.num_ksteps = (kcols + 15) / 16;
+    P.ksub = 1;
     P.b_slot_bytes = kBStageBytes;
     if (amode == kAModeTmaShared) {
         P.num_ksteps = P.Kh / 16;            // k-steps per slice; each is issued once per slice
         P.b_slot_bytes = 2 * kBStageBytes;   // weight tiles of both slices
+    } else if (amode == kAModeTma) {
+        P.ksub = 2;                          // 128 k per stage: 8 MMAs per barrier round trip
+        P.b_slot_bytes = 2 * kBStageBytes;
     }
-    P.n_b_stages = (P.num_ksteps + 3) / 4;
+    P.n_b_stages = (P.num_ksteps + 4 * P.ksub - 1) / (4 * P.ksub);
     if (amode == kAModeFrames) {
         P.a_stage_bytes = 2048 * P.P;  // 8 segments of p pixels, 128 rows
         P.n_a_stages = (P.C * P.TP * P.P + 7) / 8;
     } else {
-        P.a_stage_bytes = kBM * kBK * 2;
+        P.a_stage_bytes = P.ksub * kBM * kBK * 2;
         P.n_a_stages = P.n_b_stages;
     }
     const size_t epi_bytes = (size_t)4 * 8192;   // staging ring of the 4 epilogue warps
@@ -416,7 +425,9 @@ cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool shared, uint16
 
 // shared: every row is a single frame (tp == 2), so A holds one slice per row
 // (A[N, Kh]) and the contraction meets it with the slice-major weight.
-pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, cudaStream_t st) {
+// fold: single-frame rows against the folded weight (one product per pixel).
+pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, cudaStream_t st,
+                            bool fold = false) {
     const int row_elems = shared ? h->Kh : h->K;
     const size_t need = (size_t)P.N * row_elems * 2;
     if (need > h->stage_bytes) {
@@ -439,8 +450,8 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     bool ok = true;
     plan_tiles(h, G, G.N, false, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
-    const int amode = shared ? kAModeTmaShared : kAModeTma;
-    const size_t smem = plan_pipeline(h, G, amode);
+    const int amode = (shared && !fold) ? kAModeTmaShared : kAModeTma;
+    const size_t smem = plan_pipeline(h, G, amode, row_elems);
     CUtensorMap tx, to;
     if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
         return PE_ERR_CUDA;
@@ -449,6 +460,8 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
                                  : launch_prep<16>(P, all_scaled, shared, h->stage_rows, row_elems, st);
     if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
+    if (fold)
+        return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wfold[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
     if (shared)
         return finish(
             launch_fwd<kAModeTmaShared, 0, false>(h->tmap_wt[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
@@ -498,16 +511,9 @@ pe_status run_frames_streamed(pe_handle *h, FwdParams &P, void *out, bool all_sc
     plan_tiles(h, G, G.N, false, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
     G.ready_target = (uint32_t)(kStreamProdWarps * 2 * G.n_tiles_n);
-    const size_t smem = plan_pipeline(h, G, shared ? kAModeTmaShared : kAModeTma);
-    if (!shared) {   // both slices of a row in sequence against the slice-major weight
-        G.num_ksteps = row_elems / 16;
-        G.n_b_stages = (G.num_ksteps + 3) / 4;
-        G.n_a_stages = G.n_b_stages;
-    } else {
-        G.num_ksteps = h->Kh / 16;
-        G.n_b_stages = (G.num_ksteps + 3) / 4;
-        G.n_a_stages = G.n_b_stages;
-    }
+    // single-frame rows: one slice against both weight slices; otherwise both
+    // slices of a row in sequence against the slice-major weight
+    const size_t smem = plan_pipeline(h, G, shared ? kAModeTmaShared : kAModeTma, row_elems);
     CUtensorMap tx, to;
     if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
         return PE_ERR_CUDA;
@@ -530,6 +536,13 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
                      bool allow_staged = true) {
     P.out_f32 = out_dt == PE_F32;
     if (P.N == 0) return PE_OK;
+    // Temporal folding (opt-in): single-frame items meet the summed slices of
+    // the weight; the staged path's rows for them are already one slice wide.
+    if (allow_staged && h->fold && h->wpack_fold && P.all_t1 && staged_eligible(h, f_dt)) {
+        bool all_scaled = true;
+        for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
+        return run_frames_staged(h, P, out, all_scaled, true, st, true);
+    }
     const int lp = allow_staged ? large_path(h, P, f_dt) : 0;
     if (lp != 0) {
         bool all_scaled = true;
@@ -638,7 +651,8 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
               cudaMemset(h->err, 0, sizeof(int)) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->items_evt, cudaEventDisableTiming) == cudaSuccess;
     if (ok && h->has_bias) ok = cudaMalloc(&h->bias, sizeof(float) * E) == cudaSuccess;
-    if (ok && tp == 2) ok = cudaMalloc(&h->wpack_t, sizeof(uint16_t) * (size_t)E * 2 * h->Kh) == cudaSuccess;
+    if (ok && tp == 2) ok = cudaMalloc(&h->wpack_t, sizeof(uint16_t) * (size_t)E * 2 * h->Kh) == cudaSuccess &&
+                            cudaMalloc(&h->wpack_fold, sizeof(uint16_t) * (size_t)E * h->Kh) == cudaSuccess;
     if (ok) {
         const uint32_t boxes[3] = {32, 64, 128};   // half of BN = 64, 128, 256
         for (int i = 0; i < 3 && ok; ++i)
@@ -647,7 +661,9 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
                  make_tmap_bf16(&h->tmap_wf[i], h->wpack_f, (uint64_t)E, (uint64_t)h->Kpad, (uint64_t)h->Kpad,
                                 boxes[i]) &&
                  (!h->wpack_t || make_tmap_bf16(&h->tmap_wt[i], h->wpack_t, (uint64_t)E, (uint64_t)(2 * h->Kh),
-                                                (uint64_t)(2 * h->Kh), boxes[i]));
+                                                (uint64_t)(2 * h->Kh), boxes[i])) &&
+                 (!h->wpack_fold || make_tmap_bf16(&h->tmap_wfold[i], h->wpack_fold, (uint64_t)E, (uint64_t)h->Kh,
+                                                   (uint64_t)h->Kh, boxes[i]));
     }
     if (!ok) { pe_destroy(h); return PE_ERR_CUDA; }
     *out = h;
@@ -661,6 +677,7 @@ void pe_destroy(pe_handle *h) {
     if (h->wpack) cudaFree(h->wpack);
     if (h->wpack_f) cudaFree(h->wpack_f);
     if (h->wpack_t) cudaFree(h->wpack_t);
+    if (h->wpack_fold) cudaFree(h->wpack_fold);
     if (h->bias) cudaFree(h->bias);
     if (h->err) cudaFree(h->err);
     if (h->items_dev) cudaFree(h->items_dev);
@@ -694,7 +711,19 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
                                                           nullptr, h->E, h->C, h->tp, h->p, 2 * h->Kh, 2, h->Kh);
         if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
     }
+    if (h->wpack_fold) {
+        pe_pack_weight_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_fold,
+                                                          nullptr, h->E, h->C, h->tp, h->p, h->Kh, 3, h->Kh);
+        if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    }
     h->weight_set = true;
+    return PE_OK;
+}
+
+pe_status pe_set_temporal_fold(pe_handle *h, int enable) {
+    if (!h) return PE_ERR_INVALID_ARG;
+    if (enable && h->tp != 2) return PE_ERR_UNSUPPORTED;
+    h->fold = enable != 0;
     return PE_OK;
 }
 

@@ -73,7 +73,8 @@ struct FwdParams {
     int32_t nb, na;                                 // ring depths
     int32_t n_iss;                                  // TMA issuer warps, <= min(nb, na)
     int32_t a_stage_bytes;
-    int32_t b_slot_bytes;                           // weight ring slot: 16 KB, or 32 KB (two slices)
+    int32_t b_slot_bytes;                           // weight ring slot: ksub * slices * 16 KB
+    int32_t ksub;                                   // TMA-fed modes: 64-wide k sub-tiles per stage (1 or 2)
     int32_t epi_offset;                             // staging area offset past the rings
     int32_t merge, n_items;
     int32_t all_t1;                   // every item is a single frame (host-side kernel choice)
@@ -822,19 +823,21 @@ __device__ __forceinline__ void produce_rows_stream(const FwdParams &P, int pw, 
     }
 }
 
-// Issue loop of the TMA-fed modes: ring slot s holds one A tile (64 k) and
-// SLICES weight tiles; every stage is 4 k-steps, each issued once per slice,
-// unrolled so that the issuing thread spends a few instructions per MMA and
-// keeps the tensor pipe fed.  SLICES == 2 (kAModeTmaShared): the A tile holds
-// in-slice k of single-frame rows and slot s also holds the weight tiles of
-// slice 0 and slice 1 at the same k, so the rows are fetched once for the two
-// temporal slices they stand for.
-template <int SLICES>
+// Issue loop of the TMA-fed modes.  Ring slot s holds KSUB A tiles of 64 k
+// (16 KB each) and KSUB * SLICES weight tiles; every stage is 4 * KSUB
+// k-steps, each issued once per slice, unrolled so that the issuing thread
+// spends a few instructions per MMA and keeps the tensor pipe fed.
+//   SLICES == 2 (single-frame rows): the A tile holds in-slice k and the slot
+//   also holds the weight tiles of slice 0 and slice 1 at the same k, so the
+//   rows are fetched once for the two temporal slices they stand for.
+//   KSUB == 2: 128 k per stage (8 MMAs per barrier round trip).
+template <int SLICES, int KSUB>
 __device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring, uint64_t *full_b,
                                               uint64_t *empty_b, uint64_t *tfull, uint64_t *tempty,
                                               uint64_t *mma_done, uint32_t tmem_base, volatile int *abort) {
     constexpr uint16_t kPair = 0x3;
-    constexpr uint32_t kSlice1 = (uint32_t)kBStageBytes >> 4;   // slice-1 weight tile, descriptor units
+    constexpr uint32_t kTile = (uint32_t)kBStageBytes >> 4;   // one 16 KB tile, descriptor units
+    constexpr int KS = 4 * KSUB;                               // k-steps per stage
     const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
     const uint64_t a0 = smem_desc(smem_addr(a_ring), 16, 1024, kLayoutSw128);
     const uint64_t b0 = smem_desc(smem_addr(b_ring), 16, 1024, kLayoutSw128);
@@ -843,6 +846,13 @@ __device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_rin
     const int nk = P.num_ksteps, nst = P.n_b_stages;
     int bs = 0, acc = 0;
     uint32_t bph = 0, accph = 0;
+    auto issue = [&](uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, int ks, bool first) {
+        const int sub = ks / 4, j = ks % 4;
+        const uint64_t ad = desc_with_lo(a0, a_lo + (uint32_t)sub * kTile + 2u * j);
+        const uint32_t bl = b_lo + (uint32_t)(sub * SLICES) * kTile + 2u * j;
+        mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, bl), idesc, first ? 0u : 1u);
+        if constexpr (SLICES == 2) mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, bl + kTile), idesc, 1u);
+    };
     for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
         if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) return;
         tc_fence_after();
@@ -851,22 +861,12 @@ __device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_rin
             if (!mbar_wait(smem_addr(&full_b[bs]), bph, abort)) return;
             tc_fence_after();
             const uint32_t a_lo = a_lo0 + (uint32_t)bs * a_slot, b_lo = b_lo0 + (uint32_t)bs * b_slot;
-            const int kin = nk - 4 * st;
-            if (kin >= 4) {
+            const int kin = nk - KS * st;
+            if (kin >= KS) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint64_t ad = desc_with_lo(a0, a_lo + 2u * j);
-                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + 2u * j), idesc, (st | j) ? 1u : 0u);
-                    if constexpr (SLICES == 2)
-                        mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
-                }
+                for (int ks = 0; ks < KS; ++ks) issue(d_tmem, a_lo, b_lo, ks, st == 0 && ks == 0);
             } else {
-                for (int j = 0; j < kin; ++j) {
-                    const uint64_t ad = desc_with_lo(a0, a_lo + 2u * j);
-                    mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + 2u * j), idesc, (st | j) ? 1u : 0u);
-                    if constexpr (SLICES == 2)
-                        mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, b_lo + kSlice1 + 2u * j), idesc, 1u);
-                }
+                for (int ks = 0; ks < kin; ++ks) issue(d_tmem, a_lo, b_lo, ks, st == 0 && ks == 0);
             }
             mma_commit_pair(smem_addr(&empty_b[bs]), kPair);
             if (++bs == P.nb) { bs = 0; bph ^= 1; }
@@ -1018,16 +1018,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     if (!mbar_wait(smem_addr(&empty_b[bs]), ((g / P.nb) & 1) ^ 1, abort)) { ok = false; break; }
                     constexpr uint32_t kSlices =
                         (AMODE == kAModeTmaShared || (AMODE == kAModeTmaStream && DUPALL)) ? 2u : 1u;
+                    const int ksub = kTmaA ? P.ksub : 1;
                     if (leader)
-                        mbar_arrive_expect_tx(smem_addr(&full_b[bs]), 2 * (kSlices * b_bytes + (kTmaA ? a_bytes : 0u)));
-                    if (kTmaA)
-                        tma_load_2d_pair(smem_addr(a_ring + (size_t)bs * P.a_stage_bytes), &tmap_x, fb0 + 8u * bs,
-                                         kb * kBK, m_blk * (2 * kBM) + (int)rank * kBM, pol_x);
+                        mbar_arrive_expect_tx(smem_addr(&full_b[bs]),
+                                              2u * (uint32_t)ksub * (kSlices * b_bytes + (kTmaA ? a_bytes : 0u)));
+                    const uint32_t adst = smem_addr(a_ring + (size_t)bs * P.a_stage_bytes);
                     const uint32_t bdst = smem_addr(b_ring + (size_t)bs * P.b_slot_bytes);
                     const int wrow = n_blk * P.bn + (int)rank * (P.bn / 2);
-                    tma_load_2d_pair(bdst, &tmap_w, fb0 + 8u * bs, kb * kBK, wrow, pol_w);
-                    if (kSlices == 2)
-                        tma_load_2d_pair(bdst + kBStageBytes, &tmap_w, fb0 + 8u * bs, P.Kh + kb * kBK, wrow, pol_w);
+                    for (int sub = 0; sub < ksub; ++sub) {
+                        const int kx = (kb * ksub + sub) * kBK;
+                        if (kTmaA)
+                            tma_load_2d_pair(adst + (uint32_t)sub * kBStageBytes, &tmap_x, fb0 + 8u * bs, kx,
+                                             m_blk * (2 * kBM) + (int)rank * kBM, pol_x);
+                        const uint32_t bsub = bdst + (uint32_t)(sub * (int)kSlices) * kBStageBytes;
+                        tma_load_2d_pair(bsub, &tmap_w, fb0 + 8u * bs, kx, wrow, pol_w);
+                        if (kSlices == 2)
+                            tma_load_2d_pair(bsub + kBStageBytes, &tmap_w, fb0 + 8u * bs, P.Kh + kx, wrow, pol_w);
+                    }
                 }
             }
         }
@@ -1035,9 +1042,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         // ---------------- MMA issuer (leader CTA only)
         if (leader && lane == 0) {
             constexpr int KSA = (AMODE == kAModeFrames) ? (PT ? PT / 2 : 0) : 4;
-            if constexpr (kTmaA)
-                mma_issue_tma<(AMODE == kAModeTmaShared || (AMODE == kAModeTmaStream && DUPALL)) ? 2 : 1>(
-                    P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
+            if constexpr (kTmaA) {
+                constexpr int kSl = (AMODE == kAModeTmaShared || (AMODE == kAModeTmaStream && DUPALL)) ? 2 : 1;
+                if (kSl == 1 && P.ksub == 2)
+                    mma_issue_tma<kSl, 2>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
+                else
+                    mma_issue_tma<kSl, 1>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
+            }
             else if constexpr (KSA > 0)
                 mma_issue<KSA, AMODE == kAModeFrames, AMODE != kAModeTma>(P, a_ring, b_ring, full_a, empty_a, full_b,
                                                                           empty_b, tfull, tempty, mma_done, tmem_base,
@@ -1174,7 +1185,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
 //      stages in, zero past K;
 //   2  slice-major: column t*Kh + (c*p + i)*p + j, slice t of the kernel in its
 //      own block of Kh >= C*p*p columns (zero past C*p*p), for rows that share
-//      one A row across the temporal slices.
+//      one A row across the temporal slices;
+//   3  folded: column (c*p + i)*p + j holds bf16_rne(Ŵ[e,c,0,i,j] + Ŵ[e,c,1,i,j])
+//      (the two bf16-rounded slices summed in fp32, rounded once), zero past
+//      C*p*p: single-frame rows meet both slices in one product (tp = 2).
 __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias, int b_f32,
                                       uint16_t *wpack, float *bias32, int E, int C, int TP, int P,
                                       int ld, int order, int Kh) {
@@ -1193,7 +1207,7 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
                 const int c = ci / P, i = ci % P;
                 k = ((c * TP + t) * P + i) * P + j;
             }
-        } else {
+        } else if (order == 2) {
             const int t = kd / Kh, kk = kd - t * Kh;
             if (t < TP && kk < C * P * P) {
                 const int j = kk % P, i = (kk / P) % P, c = kk / (P * P);
@@ -1201,6 +1215,21 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
             }
         }
         uint16_t v = 0;
+        if (order == 3) {
+            k = -1;
+            if (kd < C * P * P) {
+                const int j = kd % P, i = (kd / P) % P, c = kd / (P * P);
+                float sum = 0.f;
+                for (int t = 0; t < TP; ++t) {
+                    const int64_t kt = ((c * TP + t) * P + i) * P + j;
+                    const float wt = w_f32 ? __bfloat162float(__float2bfloat16_rn(reinterpret_cast<const float *>(w)[e * K + kt]))
+                                           : __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(w)[e * K + kt] << 16);
+                    sum = __fadd_rn(sum, wt);
+                }
+                const __nv_bfloat16 b = __float2bfloat16_rn(sum);
+                v = *reinterpret_cast<const uint16_t *>(&b);
+            }
+        }
         if (k >= 0) {
             if (w_f32) {
                 const __nv_bfloat16 b = __float2bfloat16_rn(reinterpret_cast<const float *>(w)[e * K + k]);
