@@ -1249,15 +1249,16 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
 // the TMA-fed contraction, through shared memory so that both sides of the
 // copy are coalesced.  A CTA owns kPrepRows consecutive output rows and one
 // (row, word) unit per thread; consecutive threads read consecutive words of
-// one image row.  Each thread walks the channels, loads its word of the p image
-// rows of every temporal slice, normalises them and writes them into the CTA's
-// row block in shared memory; one bulk copy then stores the contiguous block of
-// rows.
+// one image row.  Each thread loads its word of the p image rows of every
+// channel (single-frame rows: all channels at once; otherwise one channel of
+// both temporal slices ahead of the one being stored), normalises them and
+// writes them into the CTA's row block in shared memory; one bulk copy then
+// stores the contiguous block of rows.
 //   SHARED  single-frame rows in the slice layout A[N, Kh], column
 //           (c*p + i)*p + j, zero up to Kh (the weight is slice-major);
 //   else    A[N, K] in the frames order k' = ((c*p + i)*tp + t)*p + j, the
 //           last frame repeated where a temporal patch runs past T.
-constexpr int kPrepRows = 32;
+constexpr int kPrepRows = 16;
 
 template <int PT, int NORM, bool SHARED>
 __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const __grid_constant__ FwdParams P,
@@ -1309,13 +1310,34 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
             }
         };
         const int C = P.C;
-        load(0, 0);
-        for (int c = 0; c < C; c += 2) {
-            if (c + 1 < C) load(1, c + 1);
-            store(0, c);
-            if (c + 1 >= C) break;
-            if (c + 2 < C) load(0, c + 2);
-            store(1, c + 1);
+        if constexpr (SHARED) {
+            // one slice per row: every channel's loads in flight at once
+            uint32_t all[4][p];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c >= C) break;
+                const char *a = src + (int64_t)c * sHW;
+#pragma unroll
+                for (int i = 0; i < p; ++i)
+                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(all[c][i]) : "l"(a + (int64_t)i * sW));
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c >= C) break;
+                const NormConst nc = norm_const(P, c);
+#pragma unroll
+                for (int i = 0; i < p; ++i)
+                    sts32(srow + (uint32_t)(((c * p + i) * p + 2 * jw) * 2), norm_word<NORM>(all[c][i], nc));
+            }
+        } else {
+            load(0, 0);
+            for (int c = 0; c < C; c += 2) {
+                if (c + 1 < C) load(1, c + 1);
+                store(0, c);
+                if (c + 1 >= C) break;
+                if (c + 2 < C) load(0, c + 2);
+                store(1, c + 1);
+            }
         }
         if (SHARED && 2 * jw < row_elems - nci * p)   // zero columns up to Kh
             sts32(srow + (uint32_t)((nci * p + 2 * jw) * 2), 0u);
