@@ -79,8 +79,8 @@ def kernel_sha():
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload, staged):
-    rec = TRAFFIC.get((workload, "staged" if staged else "fused"))
+def measured_traffic(workload, path):
+    rec = TRAFFIC.get((workload, path))
     if not rec or rec["kernel_sha"] != kernel_sha():
         return None
     return rec["bytes"]
@@ -375,13 +375,20 @@ def run_ours(args, rank, world, local):
         achieved = flop / (gemm_ms / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
         staged = launches == 2 * args.steps
+        if wl.patches is not None:
+            path = ("patches: fp32 rows cast to bf16 by a kernel, then the TMA-fed pair GEMM"
+                    if wl.patches.dtype == torch.float32 else "patches: bf16 rows, TMA-fed pair GEMM")
+        elif staged:
+            path = "staged: prepare kernel writes the normalised rows, then the TMA-fed pair GEMM"
+        else:
+            path = "fused: one kernel from frames to embeddings"
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             r, dt, th = oracle_sample_rate(wl, args.cpu_rows, 7)
             cpu = {"value": r, "unit": UNIT, "cores": th, "kind": "oracle",
                    "sample": f"{args.cpu_rows} seeded random output rows of {wl.name} (of {wl.N}), "
                              f"{dt:.1f} s; direct fp64 Conv3d, OpenMP over rows"}
-        traffic = measured_traffic(wl.name, staged)
+        traffic = measured_traffic(wl.name, "staged" if staged else "single")
         context = None if (args.no_context or world > 1) else library_context(wl, dev, flush_buf)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -393,8 +400,7 @@ def run_ours(args, rank, world, local):
             "pct_of_peak": {"bf16_burst_measured": step_tflops / peak,
                             "bf16_sustained_measured": step_tflops / float(peaks.get("bf16_tflops_sustained", peak))},
             "step_ms": {"mean": mean_ms, "median": statistics.median(times), "min": min(times)},
-            "path": "staged: prepare kernel writes A[N,K] bf16, then TMA-fed pair GEMM" if staged
-                    else "fused: one kernel from frames/patches to embeddings",
+            "path": path,
             "kernel_ms": {"contraction_mean": gemm_ms, "contraction_min": min(gemm_times),
                           "step_mean_with_kernel_events": statistics.mean(times_k),
                           "rest_of_step_mean": statistics.mean(times_k) - gemm_ms},

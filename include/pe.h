@@ -134,11 +134,31 @@ pe_status pe_set_temporal_fold(pe_handle *h, int enable);
  *         pixel_values (mytransformer README §3.2: pixel_values [N, 1176]).
  *   out : dev [N, E] of dtype out_dt.
  * Rows are processed in the given order; N may be 0 (nothing is launched).
+ * Compute dtype bf16: fp32 rows are rounded to bf16 (nearest even).  With fp32
+ * rows and K % 8 == 0 a small kernel casts them once into the handle's
+ * grow-only workspace and the TMA-fed contraction reads them back (calls that
+ * use the workspace must be serialised on one stream); PE_PATCHES_PATH=threads
+ * converts inside the contraction kernel instead.  bf16 rows are read directly.
  * Errors: PE_ERR_INVALID_ARG, PE_ERR_DTYPE, PE_ERR_ALIGN, PE_ERR_NO_WEIGHT,
  * PE_ERR_CUDA.
  */
 pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
                              void *out, pe_dtype out_dt, pe_stream_t stream);
+
+/*
+ * pe_forward_patches_pos -- pe_forward_patches with a position-embedding
+ * table added in the same epilogue: out[r, e] = (x @ W^T)[r, e] + bias[e] +
+ * pos[r, e], summed in fp32 before the output cast.  The vision model adds the
+ * interpolated position embeddings to the patch embeddings right after the
+ * PatchEmbed ("Optimize VLM PatchEmbed", the Qwen3-VL vision model forward:
+ * hidden_states + pos_embeds); the table's interpolation is the caller's.
+ *   pos    : dev [N, E] of dtype pos_dt (PE_F32 or PE_BF16), dense, 16-byte
+ *            aligned, in the same row order as out.
+ * Errors: as pe_forward_patches; a NULL or unaligned pos (with N > 0) gives
+ * PE_ERR_INVALID_ARG / PE_ERR_ALIGN, a bad pos_dt PE_ERR_DTYPE.
+ */
+pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, const void *pos,
+                                 pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream);
 
 /*
  * pe_forward_frames -- fused patchify + normalise + embed of one image/video.
@@ -156,11 +176,11 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
  * Requires p even and p <= PE_MAX_PATCH.  Three execution paths, all within
  * the same tolerance of the exact result:
  *   fused    one kernel; the normalised [N, K] patch matrix only ever exists
- *            tile by tile in shared memory (small inputs, fp32 frames, other p);
- *   staged   (default for bf16 frames with tp = 2, p in {14, 16} and at least
- *            8192 patches) a prepare kernel writes the normalised rows once
- *            into the handle's grow-only workspace, then the TMA-fed
- *            contraction reads them back;
+ *            tile by tile in shared memory (fp32 frames, tp != 2, p not in
+ *            {14, 16}, and the allocation-free call);
+ *   staged   (default for bf16 frames with tp = 2 and p in {14, 16}) a prepare
+ *            kernel writes the normalised rows once into the handle's
+ *            grow-only workspace, then the TMA-fed contraction reads them back;
  *   streamed one cooperative kernel: producer warps write the same rows while
  *            the contraction consumes the completed row blocks (an option:
  *            slower than staged on B200).
@@ -188,6 +208,21 @@ pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int
 pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
                                     const int32_t *THW, const int32_t *grid_thw, int merge,
                                     void *out, pe_dtype out_dt, pe_stream_t stream);
+
+/*
+ * pe_forward_frames_grouped_pos -- pe_forward_frames_grouped with a
+ * position-embedding table added in the same epilogue, as in
+ * pe_forward_patches_pos: out[r, e] = conv[r, e] + bias[e] + pos[r, e] in fp32
+ * before the output cast.
+ *   pos    : dev [N, E] of dtype pos_dt, N = the items' total patch count, rows
+ *            in the output's order (items in list order, merge order inside
+ *            an item), dense, 16-byte aligned.
+ * Errors: as pe_forward_frames_grouped; a NULL or unaligned pos gives
+ * PE_ERR_INVALID_ARG / PE_ERR_ALIGN, a bad pos_dt PE_ERR_DTYPE.
+ */
+pe_status pe_forward_frames_grouped_pos(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                        const int32_t *THW, const int32_t *grid_thw, int merge, const void *pos,
+                                        pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream);
 
 /* Largest item count pe_forward_frames_grouped_noalloc accepts. */
 #define PE_NOALLOC_MAX_ITEMS 1024

@@ -455,3 +455,80 @@ def test_temporal_fold_leaves_video_and_off_state_alone():
     assert torch.equal(base_v, fold_v)
     assert torch.equal(base_i, again_i)
     assert not torch.equal(base_i, fold_i)   # the folded path really ran
+
+
+# ------------------------------------------------- position-embedding epilogue
+
+@pytest.mark.parametrize("form,path,pos_dtype,out_dtype", [
+    ("frames", "fused", torch.bfloat16, torch.bfloat16),
+    ("frames", "staged", torch.float32, torch.bfloat16),
+    ("frames", "fused", torch.float32, torch.float32),
+    ("frames", "staged", torch.bfloat16, torch.float32),
+    ("patches", "-", torch.bfloat16, torch.bfloat16),
+    ("patches_f32", "-", torch.float32, torch.float32),
+])
+def test_position_embedding_add(form, path, pos_dtype, out_dtype, monkeypatch):
+    """out = conv + bias + pos with pos a [N, E] table in output row order,
+    added in fp32 before the cast (the vision model's hidden_states +
+    pos_embeds right after the PatchEmbed).  Reference: the oracle's conv plus
+    the table, tolerance over sum|x̂ ŵ| + |pos|."""
+    C, tp, p, E = 3, 2, 14, 256
+    w = workloads.normal((E, C, tp, p, p), 150, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 151, std=0.02, dtype=torch.bfloat16)
+    pe = _pe((E, C, tp, p), w, b, workloads.CLIP_MEAN, workloads.CLIP_STD)
+    if form == "frames":
+        monkeypatch.setenv("PE_FRAMES_PATH", path)
+        grids = [(1, 6, 10), (2, 4, 6), (1, 10, 4)]
+        Ts = [1, 3, 1]
+        items = [(workloads.uniform01((T, C, g[1] * p, g[2] * p), 152 + i), g) for i, (T, g) in enumerate(zip(Ts, grids))]
+        N = sum(g[0] * g[1] * g[2] for g in grids)
+        pos = workloads.normal((N, E), 160, std=1.0, dtype=pos_dtype)
+        out = pe.forward_frames_grouped([f.to(DEV) for f, _ in items], grids, 2, out_dtype=out_dtype, pos=pos.to(DEV))
+        ref, mag = oracle.conv3d_grouped(items, 2, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
+    else:
+        N = 300
+        xdt = torch.float32 if form == "patches_f32" else torch.bfloat16
+        x = workloads.normal((N, C * tp * p * p), 161, dtype=xdt)
+        pos = workloads.normal((N, E), 162, std=1.0, dtype=pos_dtype)
+        out = pe.forward_patches(x.to(DEV), out_dtype=out_dtype, pos=pos.to(DEV))
+        ref, mag = oracle.conv3d_patches(x, w, b, C, tp, p)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    pv = pos.double().numpy()
+    assert_within_tolerance(out, ref + pv, mag + np.abs(pv), what=f"pos {form} {path}")
+
+
+def test_position_embedding_argument_errors():
+    C, tp, p, E = 3, 2, 14, 64
+    pe = _pe((E, C, tp, p), workloads.normal((E, C, tp, p, p), 170, std=0.02), None)
+    x = torch.zeros(8, C * tp * p * p, dtype=torch.bfloat16, device=DEV)
+    out = torch.empty(8, E, dtype=torch.bfloat16, device=DEV)
+    pos = torch.zeros(8 * E + 8, dtype=torch.bfloat16, device=DEV)
+    from vlm_vision_patch_b200 import _binding as B
+    s = torch.cuda.current_stream().cuda_stream
+    with pytest.raises(PEError) as e:
+        B.pe_forward_patches_pos(pe.h, x.data_ptr(), B.PE_BF16, 8, 0, B.PE_BF16, out.data_ptr(), B.PE_BF16, s)
+    assert e.value.status == "PE_ERR_INVALID_ARG"
+    with pytest.raises(PEError) as e:
+        B.pe_forward_patches_pos(pe.h, x.data_ptr(), B.PE_BF16, 8, pos.data_ptr() + 2, B.PE_BF16, out.data_ptr(),
+                                 B.PE_BF16, s)
+    assert e.value.status == "PE_ERR_ALIGN"
+    with pytest.raises(PEError) as e:
+        B.pe_forward_patches_pos(pe.h, x.data_ptr(), B.PE_BF16, 8, pos.data_ptr(), 7, out.data_ptr(), B.PE_BF16, s)
+    assert e.value.status == "PE_ERR_DTYPE"
+
+
+@pytest.mark.parametrize("path", ["cast", "threads"])
+def test_fp32_patches_both_paths(path, monkeypatch):
+    """fp32 rows: cast to bf16 by a separate kernel, then the TMA-fed contraction
+    (default), or converted by producer warps inside the contraction kernel.
+    Both must be within tolerance of the oracle."""
+    C, tp, p, E = 3, 2, 14, 1280
+    x = workloads.normal((700, C * tp * p * p), 180)
+    w = workloads.kaiming_uniform_conv((E, C, tp, p, p), 181)
+    pe = _pe((E, C, tp, p), w, None)
+    ref, mag = oracle.conv3d_patches(x, w, None, C, tp, p)
+    monkeypatch.setenv("PE_PATCHES_PATH", path)
+    out = pe.forward_patches(x.to(DEV), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_within_tolerance(out, ref, mag, what=f"fp32 patches {path}")

@@ -89,10 +89,16 @@ class PatchEmbed:
         return out
 
     def forward_patches(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
-                        out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+                        out_dtype: torch.dtype = torch.bfloat16, stream=None,
+                        pos: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """out = x @ W^T (+ bias) (+ pos, a [N, E] table added in the same epilogue)."""
         out = self._out(x.shape[0], out, out_dtype, x.device)
-        B.pe_forward_patches(self.h, _dev(x, "x"), _dt(x.dtype), x.shape[0], _dev(out, "out"),
-                             _dt(out.dtype), _stream(stream))
+        if pos is None:
+            B.pe_forward_patches(self.h, _dev(x, "x"), _dt(x.dtype), x.shape[0], _dev(out, "out"),
+                                 _dt(out.dtype), _stream(stream))
+        else:
+            B.pe_forward_patches_pos(self.h, _dev(x, "x"), _dt(x.dtype), x.shape[0], _dev(pos, "pos"),
+                                     _dt(pos.dtype), _dev(out, "out"), _dt(out.dtype), _stream(stream))
         return out
 
     def forward_frames(self, frames: torch.Tensor, grid_thw: Sequence[int], merge: int = 2,
@@ -107,15 +113,24 @@ class PatchEmbed:
 
     def forward_frames_grouped(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]],
                                merge: int = 2, out: Optional[torch.Tensor] = None,
-                               out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+                               out_dtype: torch.dtype = torch.bfloat16, stream=None,
+                               pos: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """All items in one launch; `pos`, if given, is a [N, E] table in output row
+        order added in the same epilogue."""
         n = sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
         out = self._out(n, out, out_dtype, frames[0].device)
         dts = {f.dtype for f in frames}
         if len(dts) != 1:
             raise TypeError("all items must share one dtype")
-        B.pe_forward_frames_grouped(self.h, [_dev(f, "frames") for f in frames], _dt(frames[0].dtype),
-                                    [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames], grid_thw,
-                                    merge, _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        ptrs = [_dev(f, "frames") for f in frames]
+        thw = [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames]
+        if pos is None:
+            B.pe_forward_frames_grouped(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
+                                        _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        else:
+            B.pe_forward_frames_grouped_pos(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
+                                            _dev(pos, "pos"), _dt(pos.dtype), _dev(out, "out"), _dt(out.dtype),
+                                            _stream(stream))
         return out
 
     def patchify(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]], merge: int = 2,

@@ -29,7 +29,7 @@ EXPORTS = (
     "pe_create", "pe_set_weight", "pe_set_norm", "pe_forward_patches", "pe_forward_frames",
     "pe_forward_frames_grouped", "pe_forward_frames_grouped_noalloc", "pe_patchify", "pe_num_patches", "pe_last_error",
     "pe_status_string", "pe_destroy", "pe_device", "pe_profile_begin", "pe_profile_end",
-    "pe_set_temporal_fold",
+    "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos",
 )
 
 
@@ -62,6 +62,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_set_norm": ([vp, f32p, f32p], i32),
         "pe_set_temporal_fold": ([vp, i32], i32),
         "pe_forward_patches": ([vp, vp, i32, i64, vp, i32, vp], i32),
+        "pe_forward_patches_pos": ([vp, vp, i32, i64, vp, i32, vp, i32, vp], i32),
+        "pe_forward_frames_grouped_pos": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp, i32, vp],
+                                          i32),
         "pe_forward_frames": ([vp, vp, i32, i32, i32, i32, i32p, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped_noalloc": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
@@ -135,6 +138,21 @@ def pe_set_temporal_fold(h: int, enable: bool) -> None:
 
 def pe_forward_patches(h: int, x_ptr: int, x_dt: int, N: int, out_ptr: int, out_dt: int, stream: int) -> None:
     _check("pe_forward_patches", load().pe_forward_patches(h, x_ptr, x_dt, N, out_ptr, out_dt, stream))
+
+
+def pe_forward_patches_pos(h: int, x_ptr: int, x_dt: int, N: int, pos_ptr: int, pos_dt: int, out_ptr: int,
+                           out_dt: int, stream: int) -> None:
+    _check("pe_forward_patches_pos",
+           load().pe_forward_patches_pos(h, x_ptr, x_dt, N, pos_ptr, pos_dt, out_ptr, out_dt, stream))
+
+
+def pe_forward_frames_grouped_pos(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence[int]],
+                                  grid_thw: Sequence[Sequence[int]], merge: int, pos_ptr: int, pos_dt: int,
+                                  out_ptr: int, out_dt: int, stream: int) -> None:
+    n = len(f_ptrs)
+    _check("pe_forward_frames_grouped_pos", load().pe_forward_frames_grouped_pos(
+        h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
+        _i32arr([v for g in grid_thw for v in g]), merge, pos_ptr, pos_dt, out_ptr, out_dt, stream))
 
 
 def pe_forward_frames(h: int, f_ptr: int, f_dt: int, T: int, H: int, W: int, grid_thw: Sequence[int],

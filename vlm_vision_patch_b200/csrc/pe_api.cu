@@ -377,18 +377,19 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
     return PE_OK;
 }
 
-// Staged frames path: prepare kernel writes A once (frames k order), then the
-// TMA-fed pair GEMM reads it with the frames-order weight.  Chosen for large
-// inputs (the fused producer repeats its gather for every weight tile of a
-// row block), or forced with PE_FRAMES_PATH=staged / fused.
-constexpr int64_t kStagedMinRows = 8192;
+// Staged frames path: prepare kernel writes A once, then the TMA-fed pair
+// GEMM reads it back.  The fused producer repeats its gather for every weight
+// tile of a row block; measured on B200 the staged pair is faster at every
+// size (about 2x at ~1000 patches, where both are latency-bound, 1.8x at
+// 59k), so it runs whenever it can: bf16 frames, tp = 2, p in {14, 16}.
 
 bool staged_eligible(const pe_handle *h, int f_dt) {
     return f_dt == PE_BF16 && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
 }
 
-// Large bf16 frame batches: 0 = fused kernel, 1 = staged pair (the default),
-// 2 = streamed kernel.  PE_FRAMES_PATH=fused|staged|streamed overrides.  The
+// bf16 frames with tp = 2 and p in {14, 16}: 0 = fused kernel, 1 = staged
+// pair (the default), 2 = streamed kernel.  PE_FRAMES_PATH=fused|staged|streamed
+// overrides.  The
 // streamed kernel overlaps row production with the contraction but its
 // producer warps' scattered loads and stores slow the contraction down more
 // than the separate prepare kernel costs (measured on B200), so it is not the
@@ -399,7 +400,8 @@ int large_path(const pe_handle *h, const FwdParams &P, int f_dt) {
     if (e && std::strcmp(e, "fused") == 0) return 0;
     if (e && std::strcmp(e, "staged") == 0) return 1;
     if (e && std::strcmp(e, "streamed") == 0) return 2;
-    return P.N >= kStagedMinRows ? 1 : 0;
+    (void)P;
+    return 1;
 }
 
 template <int PT, int NORM, bool SHARED>
@@ -741,8 +743,13 @@ pe_status pe_set_norm(pe_handle *h, const float *mean, const float *std) {
     return PE_OK;
 }
 
-pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, void *out,
-                             pe_dtype out_dt, pe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of pe_forward_patches and pe_forward_patches_pos.
+pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, const void *pos, int pos_dt,
+                          void *out, pe_dtype out_dt, pe_stream_t stream) {
     if (!h || N < 0) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(x_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (!h->weight_set) return PE_ERR_NO_WEIGHT;
@@ -757,9 +764,47 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
     P.x = x;
     P.x_f32 = x_dt == PE_F32;
     P.out_f32 = out_dt == PE_F32;
+    P.pos = pos;
+    P.pos_f32 = pos_dt == PE_F32;
     P.merge = 1;
     const bool tma = (x_dt == PE_BF16) && (h->K % 8 == 0);
     P.x_vec = (x_dt == PE_BF16) ? (h->K % 8 == 0) : (h->K % 4 == 0);
+    // fp32 rows with K % 8 == 0: cast them to bf16 once into the workspace and
+    // run the TMA-fed contraction (PE_PATCHES_PATH=threads keeps the producer
+    // warps converting inside the contraction kernel).
+    const char *pp = std::getenv("PE_PATCHES_PATH");
+    if (x_dt == PE_F32 && (h->K % 8) == 0 && !(pp && std::strcmp(pp, "threads") == 0)) {
+        const size_t need = (size_t)N * h->K * 2;
+        cudaStream_t st = (cudaStream_t)stream;
+        if (need > h->stage_bytes) {
+            if (h->stage_rows) {
+                if (cudaStreamSynchronize(st) != cudaSuccess) return PE_ERR_CUDA;
+                cudaFree(h->stage_rows);
+            }
+            h->stage_rows = nullptr;
+            h->stage_bytes = 0;
+            if (cudaMalloc(&h->stage_rows, need) != cudaSuccess) return PE_ERR_CUDA;
+            h->stage_bytes = need;
+        }
+        int grid = 0;
+        bool ok = true;
+        plan_tiles(h, P, N, false, grid, ok);
+        if (!ok) return PE_ERR_UNSUPPORTED;
+        const size_t smem = plan_pipeline(h, P, kAModeTma);
+        CUtensorMap tx, to;
+        if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)N, (uint64_t)h->K, (uint64_t)h->K, kBM)) return PE_ERR_CUDA;
+        if (!make_out_tmap(&to, out, P.out_f32, N, h->E)) return PE_ERR_CUDA;
+        const int64_t n8 = (int64_t)N * h->K / 8;
+        const int cb = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)h->num_sms * 8);
+        pe_cast_rows_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(x), h->stage_rows, n8);
+        if (h->prof_on) ++h->prof_launches;
+        if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+        FwdParams G = P;
+        G.x = h->stage_rows;
+        G.x_f32 = 0;
+        G.x_vec = 1;
+        return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_w[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
+    }
     int grid = 0;
     bool ok = true;
     plan_tiles(h, P, N, !tma, grid, ok);
@@ -777,9 +822,10 @@ pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t
     return finish(launch_fwd<kAModePatchThreads, 0, false>(tw, P, tx, to, smem, grid, st));
 }
 
-pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
-                                    const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
-                                    pe_dtype out_dt, pe_stream_t stream) {
+// Shared body of pe_forward_frames_grouped and pe_forward_frames_grouped_pos.
+pe_status forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                 const int32_t *THW, const int32_t *grid_thw, int merge, const void *pos,
+                                 int pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream) {
     if (!h) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (!h->weight_set) return PE_ERR_NO_WEIGHT;
@@ -788,7 +834,48 @@ pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *fram
     FwdParams P;
     const pe_status s = setup_frames(h, n, frames, f_dt, THW, grid_thw, merge, out, P, (cudaStream_t)stream);
     if (s != PE_OK) return s;
+    P.pos = pos;
+    P.pos_f32 = pos_dt == PE_F32;
     return run_frames(h, P, f_dt, out, out_dt, (cudaStream_t)stream);
+}
+
+pe_status check_pos(const void *pos, int pos_dt) {
+    if (!pos) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(pos_dt)) return PE_ERR_DTYPE;
+    if (!aligned16(pos)) return PE_ERR_ALIGN;
+    return PE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, void *out,
+                             pe_dtype out_dt, pe_stream_t stream) {
+    return forward_patches(h, x, x_dt, N, nullptr, PE_BF16, out, out_dt, stream);
+}
+
+pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, const void *pos,
+                                 pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream) {
+    if (N > 0) {
+        const pe_status s = check_pos(pos, pos_dt);
+        if (s != PE_OK) return s;
+    }
+    return forward_patches(h, x, x_dt, N, pos, pos_dt, out, out_dt, stream);
+}
+
+pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                    const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
+                                    pe_dtype out_dt, pe_stream_t stream) {
+    return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, nullptr, PE_BF16, out, out_dt, stream);
+}
+
+pe_status pe_forward_frames_grouped_pos(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
+                                        const int32_t *THW, const int32_t *grid_thw, int merge, const void *pos,
+                                        pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream) {
+    const pe_status s = check_pos(pos, pos_dt);
+    if (s != PE_OK) return s;
+    return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, pos, pos_dt, out, out_dt, stream);
 }
 
 pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H, int W,

@@ -23,6 +23,8 @@
 // one tile overlaps the MMAs of the next.  Every pipeline wait is bounded.
 #pragma once
 
+#include <type_traits>
+
 #include "pe_device.cuh"
 #include "../../include/pe.h"
 
@@ -89,6 +91,8 @@ struct FwdParams {
     int32_t x_vec;                    // patch rows allow 16-byte vector loads
     int32_t out_f32;
     const float *bias;                // fp32 [E] or nullptr
+    const void *pos;                  // [N, E] added in the epilogue, or nullptr
+    int32_t pos_f32;                  // pos dtype is fp32 (else bf16)
     int *err;                         // device error word
     // kAModeTmaStream
     uint16_t *a_rows;                 // [N, row_elems] rows written by the producers
@@ -1069,9 +1073,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         const int nch = P.bn / 32;   // 2, 4 or 8
         int acc = 0, nbuf = 0;
         uint32_t accph = 0;
-        auto emit = [&](const uint32_t (&v)[32], int cc, int64_t row0, int n_blk) {
+        auto emit = [&](auto kPos, const uint32_t (&v)[32], int cc, int64_t row0, int n_blk) {
+            constexpr bool has_pos = decltype(kPos)::value;
             const int col0 = n_blk * P.bn + cc * 32;
             if (row0 >= P.N || col0 >= P.E) return;   // whole box outside: nothing to store
+            // position-embedding row segment of this lane's row (E % 8 == 0, so a
+            // 16-byte piece is either wholly inside the row or wholly past it)
+            uint4 pq[8];
+            if constexpr (has_pos) {
+                const int64_t r = row0 + lane;
+                const int nq = P.pos_f32 ? 8 : 4;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    pq[q] = make_uint4(0u, 0u, 0u, 0u);
+                    const int c0 = col0 + q * (P.pos_f32 ? 4 : 8);
+                    if (q < nq && r < P.N && c0 < P.E) {
+                        const char *a = reinterpret_cast<const char *>(P.pos) +
+                                        (r * P.E + c0) * (int64_t)(P.pos_f32 ? 4 : 2);
+                        asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
+                                     : "l"(a));
+                    }
+                }
+            }
             float f[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
@@ -1085,6 +1109,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 if (nbufs == 4) bulk_wait_read<3>(); else bulk_wait_read<1>();
             }
             __syncwarp();
+            if constexpr (has_pos) {   // out = acc + bias + pos, in fp32, before the output cast
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t w4[4] = {pq[q].x, pq[q].y, pq[q].z, pq[q].w};
+                    if (P.pos_f32) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) f[4 * q + u] += __uint_as_float(w4[u]);
+                    } else if (q < 4) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            f[8 * q + 2 * u] += bf16lo_to_f32(w4[u]);
+                            f[8 * q + 2 * u + 1] += bf16hi_to_f32(w4[u]);
+                        }
+                    }
+                }
+            }
             uint8_t *buf = stage_buf + (size_t)nbuf * (P.out_f32 ? 4096 : 2048);
             if (P.out_f32) {
                 // 128-byte rows, 128-byte swizzle: chunk c of row r at (c ^ (r & 7))
@@ -1108,37 +1148,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             }
             if (++nbuf == nbufs) nbuf = 0;
         };
-        for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
-            const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
-            if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
-            tc_fence_after();
-            const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
-            const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
-            if constexpr (kTmaA && AMODE != kAModeTmaStream) {
-                // registers to spare: the next chunk's TMEM load overlaps this chunk's work
-                uint32_t va[32], vb[32];
-                tmem_ld_32x32b_x32(tbase, va);
-                for (int cc = 0; cc < nch; cc += 2) {
-                    tmem_ld_wait();
-                    tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 1) * 32, vb);
-                    emit(va, cc, row0, n_blk);
-                    tmem_ld_wait();
-                    if (cc + 2 < nch) tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 2) * 32, va);
-                    emit(vb, cc + 1, row0, n_blk);
+        // the tile loop, compiled with and without the position-embedding add
+        auto tiles = [&](auto kPos) {
+            for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
+                const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
+                if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
+                tc_fence_after();
+                const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
+                const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
+                if constexpr (kTmaA && AMODE != kAModeTmaStream) {
+                    // registers to spare: the next chunk's TMEM load overlaps this chunk's work
+                    uint32_t va[32], vb[32];
+                    tmem_ld_32x32b_x32(tbase, va);
+                    for (int cc = 0; cc < nch; cc += 2) {
+                        tmem_ld_wait();
+                        tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 1) * 32, vb);
+                        emit(kPos, va, cc, row0, n_blk);
+                        tmem_ld_wait();
+                        if (cc + 2 < nch) tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 2) * 32, va);
+                        emit(kPos, vb, cc + 1, row0, n_blk);
+                    }
+                } else {
+                    uint32_t va[32];
+                    for (int cc = 0; cc < nch; ++cc) {
+                        tmem_ld_32x32b_x32(tbase + (uint32_t)cc * 32, va);
+                        tmem_ld_wait();
+                        emit(kPos, va, cc, row0, n_blk);
+                    }
                 }
-            } else {
-                uint32_t va[32];
-                for (int cc = 0; cc < nch; ++cc) {
-                    tmem_ld_32x32b_x32(tbase + (uint32_t)cc * 32, va);
-                    tmem_ld_wait();
-                    emit(va, cc, row0, n_blk);
-                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
+                if (++acc == 2) { acc = 0; accph ^= 1; }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * (uint32_t)acc);
-            if (++acc == 2) { acc = 0; accph ^= 1; }
-        }
+        };
+        if (P.pos) tiles(std::true_type{});
+        else tiles(std::false_type{});
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
     } else if (AMODE == kAModeTmaStream && warp >= kStreamProdWarp0 && warp < kStreamProdWarp0 + kStreamProdWarps) {
@@ -1348,6 +1393,18 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
         bulk_store(A + m0 * row_elems, smem_addr(prep_smem), (uint32_t)(rows * row_elems * 2));
         bulk_commit();
         bulk_wait<0>();
+    }
+}
+
+// fp32 patch rows -> bf16 (round to nearest even) rows for the TMA-fed
+// contraction: the same rounding the contraction applies to fp32 inputs
+// everywhere.  8 elements per thread (32-byte loads, 16-byte stores).
+__global__ void pe_cast_rows_kernel(const float *__restrict__ x, uint16_t *__restrict__ A, int64_t n8) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
+        *(reinterpret_cast<uint4 *>(A) + i) =
+            make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
     }
 }
 
