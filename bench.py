@@ -64,8 +64,8 @@ def load_peaks():
 # the figure (reported as null) until it is captured again.
 TRAFFIC = {
     # profiles/pe_fwd_kernel_grouped_16_images.md, profiles/pe_fwd_kernel_long_video_64x896.md
-    ("grouped_16_images", "staged"): {"bytes": 108142080 + 97811200, "kernel_sha": "4d18c8dc51006a52"},
-    ("long_video_64x896", "staged"): {"bytes": 515314176 + 281386240, "kernel_sha": "4d18c8dc51006a52"},
+    ("grouped_16_images", "staged"): {"bytes": 100918784 + 101084160, "kernel_sha": "f06edeebd016f432"},
+    ("long_video_64x896", "staged"): {"bytes": 388124928 + 281637120, "kernel_sha": "f06edeebd016f432"},
 }
 KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh")
 
