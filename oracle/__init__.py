@@ -67,6 +67,7 @@ def _load():
         lib.oracle_conv3d_patches.argtypes = [
             f32p, ctypes.c_int64, f32p, f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, u8p, f64p, f64p]
+        lib.oracle_conv3d_patches_fp32.argtypes = lib.oracle_conv3d_patches.argtypes
         lib.oracle_conv3d_frames.argtypes = [
             f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, f32p, f32p, f32p, f32p, ctypes.c_int, ctypes.c_int,
@@ -138,6 +139,27 @@ def conv3d_patches(x, w, bias, C: int, tp: int, p: int, row_mask=None
                                   _p(b, ctypes.c_float), E, C, tp, p,
                                   _p(m, ctypes.c_uint8), _p(out, ctypes.c_double),
                                   _p(mag, ctypes.c_double))
+    return out, mag
+
+
+def conv3d_patches_fp32(x, w, bias, C: int, tp: int, p: int, row_mask=None
+                        ) -> Tuple[np.ndarray, np.ndarray]:
+    """Patches form on the fp32 values as given (no bf16 rounding): the Conv3d
+    definition in fp64.  Returns (out[N,E], absdot[N,E]); masked-out rows NaN."""
+    x = _f32(x)
+    w = _f32(w)
+    E = int(w.shape[0])
+    K = C * tp * p * p
+    assert w.size == E * K and x.ndim == 2 and x.shape[1] == K
+    N = int(x.shape[0])
+    b = None if bias is None else _f32(bias)
+    out = np.full((N, E), np.nan)
+    mag = np.full((N, E), np.nan)
+    m = _mask(row_mask, N)
+    _load().oracle_conv3d_patches_fp32(_p(x, ctypes.c_float), N, _p(w, ctypes.c_float),
+                                       _p(b, ctypes.c_float), E, C, tp, p,
+                                       _p(m, ctypes.c_uint8), _p(out, ctypes.c_double),
+                                       _p(mag, ctypes.c_double))
     return out, mag
 
 

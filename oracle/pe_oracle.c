@@ -142,6 +142,38 @@ void oracle_conv3d_patches(const float *x, int64_t N, const float *w, const floa
     free(wb);
 }
 
+/* Patches form on the fp32 values exactly as given (no bf16 rounding of x or
+ * w): the Conv3d definition in fp64, the reference for contractions that keep
+ * more than bf16 precision of fp32 inputs.  Same layout and outputs as
+ * oracle_conv3d_patches. */
+void oracle_conv3d_patches_fp32(const float *x, int64_t N, const float *w, const float *bias,
+                                int E, int C, int tp, int p, const uint8_t *row_mask,
+                                double *out, double *absdot)
+{
+    const int64_t K = (int64_t)C * tp * p * p;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        if (row_mask && !row_mask[n])
+            continue;
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0, mag = 0.0;
+            for (int c = 0; c < C; ++c)
+                for (int t = 0; t < tp; ++t)
+                    for (int i = 0; i < p; ++i)
+                        for (int j = 0; j < p; ++j) {
+                            const int64_t k = (((int64_t)c * tp + t) * p + i) * p + j;
+                            const double xv = (double)x[n * K + k];
+                            const double wv = (double)w[(int64_t)e * K + k];
+                            acc += xv * wv;
+                            mag += fabs(xv * wv);
+                        }
+            out[n * E + e] = acc + (bias ? (double)bias[e] : 0.0);
+            if (absdot)
+                absdot[n * E + e] = mag;
+        }
+    }
+}
+
 /* The normalised, time-padded volume Fh[tau, c, y, x] for tau < tp*gt:
  * Fp[tau] = F[min(tau, T-1)], Fh = bf16(fp32(fp32(Fp - mean_c) / std_c)). */
 static float *normalized_volume(const float *frames, int T, int C, int H, int W,

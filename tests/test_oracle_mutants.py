@@ -40,6 +40,10 @@ MUTANTS = {
                        "u = (u + 0x8000u) & 0xffff0000u;"),
     "input_not_rounded": ("const double xv = (double)oracle_bf16_round(x[n * K + k]);",
                           "const double xv = (double)x[n * K + k];"),
+    "fp32_form_rounds_input": ("const double xv = (double)x[n * K + k];",
+                               "const double xv = (double)oracle_bf16_round(x[n * K + k]);"),
+    "fp32_form_neighbour_column": ("const double xv = (double)x[n * K + k];",
+                                   "const double xv = (double)x[n * K + (k ^ 1)];"),
     "patchify_drops_time_offset": ("const int64_t tau = g_t * tp + t;\n                        rows",
                                    "const int64_t tau = g_t * tp;\n                        rows"),
 }

@@ -310,3 +310,35 @@ def test_kaiming_bound_of_config_weight():
     b = 1.0 / np.sqrt(1176.0)
     assert abs(b - 0.02916) < 1e-5
     assert float(w.abs().max()) <= b and float(w.abs().max()) > 0.99 * b
+
+
+# ------------------------------------------------ fp32-exact patches form
+
+@pytest.mark.parametrize("C,tp,p,E", [(3, 2, 2, 5), (1, 1, 3, 4), (2, 2, 4, 3)])
+def test_patches_fp32_matches_torch_conv3d(C, tp, p, E):
+    """The unrounded patches form equals torch's fp64 Conv3d on the fp32 values
+    (a library routine), with values that bf16 cannot represent."""
+    K = C * tp * p * p
+    g = torch.Generator().manual_seed(300 + K)
+    x = torch.randn(7, K, generator=g) * 1.2345
+    w = torch.randn(E, C, tp, p, p, generator=g) * 0.4321
+    b = torch.randn(E, generator=g)
+    out, mag = oracle.conv3d_patches_fp32(x, w, b, C, tp, p)
+    ref = torch.nn.functional.conv3d(x.double().view(-1, C, tp, p, p), w.double(), b.double()).view(7, E)
+    assert np.allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    absref = torch.nn.functional.conv3d(x.double().abs().view(-1, C, tp, p, p), w.double().abs()).view(7, E)
+    assert np.allclose(mag, absref.numpy(), rtol=1e-12, atol=1e-12)
+    # and it really does not round: bf16-rounded inputs give a different result
+    out_b, _ = oracle.conv3d_patches(x, w, b, C, tp, p)
+    assert not np.allclose(out, out_b, rtol=1e-6, atol=0)
+
+
+def test_patches_fp32_equals_rounded_form_on_bf16_values():
+    """On bf16-representable inputs both patches forms are the same definition."""
+    C, tp, p, E = 3, 2, 3, 6
+    K = C * tp * p * p
+    x = workloads.normal((9, K), 310).to(torch.bfloat16).float()
+    w = workloads.normal((E, C, tp, p, p), 311, std=0.1).to(torch.bfloat16).float()
+    a, ma = oracle.conv3d_patches_fp32(x, w, None, C, tp, p)
+    b, mb = oracle.conv3d_patches(x, w, None, C, tp, p)
+    assert np.array_equal(a, b) and np.array_equal(ma, mb)
