@@ -271,6 +271,8 @@ def run_ours(args, rank, world, local):
     pe.set_norm(wl.mean, wl.std)
     if args.fold:
         pe.set_temporal_fold(True)
+    if args.tf32:
+        pe.set_tf32(True)
     out = torch.empty((wl.N, wl.E), dtype=wl.out_dtype, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -393,7 +395,8 @@ def run_ours(args, rank, world, local):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_max_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "tf32" if (args.tf32 and wl.patches is not None and wl.patches.dtype == torch.float32) else "bf16",
             "data": "synthetic (seeded U[0,1) frames, N(0,0.02) weights)",
             "config": dict(config_of(wl, world), **({"temporal_fold": True, "K_contracted": k_eff} if folded else {})),
             "tflops": step_tflops,
@@ -436,6 +439,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the cuBLAS context timing")
+    ap.add_argument("--tf32", action="store_true",
+                    help="opt-in tf32 contraction of fp32 patch rows (the fp32 workloads); dtype reads tf32")
     ap.add_argument("--fold", action="store_true",
                     help="opt-in temporal folding of single-frame items (half the contraction; TFLOP/s then "
                          "counts the folded K)")

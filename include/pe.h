@@ -128,6 +128,20 @@ pe_status pe_set_norm(pe_handle *h, const float *mean, const float *std);
 pe_status pe_set_temporal_fold(pe_handle *h, int enable);
 
 /*
+ * pe_set_tf32 -- opt-in tf32 contraction for fp32 patch rows.
+ * Qwen2.5VL-Vision Encode-PatchEmbed checks the Conv3d against the matmul in
+ * fp32 (the python check: a max difference of about 4e-6); the default bf16
+ * compute keeps 8 significant bits of each input.  With tf32 enabled,
+ * pe_forward_patches on fp32 rows rounds the rows and the weight to tf32
+ * (10 fraction bits, nearest with ties away from zero) and contracts with
+ * kind::tf32 tensor-core MMAs accumulating in fp32: each product then carries
+ * at most about 2^-10 relative error instead of 2^-7.  Half the bf16 tensor
+ * rate.  Requires K % 4 == 0.  enable = 0 (default) or 1.  bf16 rows and the
+ * frames calls are unaffected.  Errors: PE_ERR_INVALID_ARG, PE_ERR_UNSUPPORTED.
+ */
+pe_status pe_set_tf32(pe_handle *h, int enable);
+
+/*
  * pe_forward_patches -- out = x @ W^T (+ bias) on already patchified rows.
  *   x   : dev [N, K] of dtype x_dt (PE_BF16 or PE_F32), rows in
  *         view(-1, C, tp, p, p) order as the Qwen2-VL processor emits

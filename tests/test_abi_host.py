@@ -23,7 +23,7 @@ def lib():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(pe_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(pe_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_matches_binding_exports():
@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol(lib):
     from vlm_vision_patch_b200 import _binding
     out = subprocess.run(["nm", "-D", "--defined-only", _binding.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (pe_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (pe_[a-z0-9_]+)\b", out))
     missing = [f for f in declared_functions() if f not in exported]
     assert not missing, missing
     for f in declared_functions():

@@ -532,3 +532,65 @@ def test_fp32_patches_both_paths(path, monkeypatch):
     out = pe.forward_patches(x.to(DEV), out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert_within_tolerance(out, ref, mag, what=f"fp32 patches {path}")
+
+
+# ------------------------------------------------------------ tf32 contraction
+
+def _tf32_round(t: torch.Tensor) -> torch.Tensor:
+    """fp32 -> nearest tf32 value (10 fraction bits, ties away from zero)."""
+    u = t.float().contiguous().view(torch.int32).numpy().astype(np.int64)
+    u = ((u + 0x1000) & 0xFFFFE000).astype(np.uint32).view(np.int32)
+    return torch.from_numpy(u.copy()).view(torch.float32)
+
+
+@pytest.mark.parametrize("N,E,bias,out_dtype", [
+    (1024, 1280, False, torch.float32),    # the fp32 [1024, 1176] workload shape
+    (300, 200, True, torch.float32),       # partial tiles in N and E
+    (129, 1280, False, torch.bfloat16),
+])
+def test_tf32_patches(N, E, bias, out_dtype):
+    """Opt-in tf32 contraction of fp32 rows: (1) within the tf32 bound
+    (2^-10 + 2^-13) * sum|x w| of the exact fp32-input Conv3d; (2) within fp32
+    accumulation (1e-4 * sum) of the oracle on the tf32-rounded values; (3)
+    several times closer to the exact result than the default bf16 path."""
+    C, tp, p = 3, 2, 14
+    K = C * tp * p * p
+    x = workloads.normal((N, K), 190 + N)
+    w = workloads.kaiming_uniform_conv((E, C, tp, p, p), 191)
+    b = workloads.normal((E,), 192, std=0.02) if bias else None
+    pe = _pe((E, C, tp, p), w, b)
+    xd = x.to(DEV)
+    base = pe.forward_patches(xd, out_dtype=torch.float32)        # bf16 compute
+    pe.set_tf32(True)
+    out = pe.forward_patches(xd, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    ref, mag = oracle.conv3d_patches_fp32(x, w, b, C, tp, p)
+    r_tf32 = assert_within_tolerance(out, ref, mag, what="tf32 vs exact", rel=2.0 ** -10 + 2.0 ** -13)
+    ref_r, mag_r = oracle.conv3d_patches_fp32(_tf32_round(x), _tf32_round(w), b, C, tp, p)
+    assert_within_tolerance(out, ref_r, mag_r, what="tf32 vs tf32-rounded oracle", rel=1e-4)
+    if out_dtype == torch.float32:
+        err_t = np.abs(out.cpu().double().numpy() - ref) / mag
+        err_b = np.abs(base.cpu().double().numpy() - ref) / mag
+        assert err_t.mean() * 4 < err_b.mean(), (err_t.mean(), err_b.mean())
+    assert r_tf32 <= 1.0
+
+
+def test_tf32_switch_is_per_handle_and_reversible():
+    C, tp, p, E = 3, 2, 14, 256
+    x = workloads.normal((64, C * tp * p * p), 195).to(DEV)
+    pe = _pe((E, C, tp, p), workloads.normal((E, C, tp, p, p), 196, std=0.05), None)
+    a = pe.forward_patches(x, out_dtype=torch.float32)
+    pe.set_tf32(True)
+    t = pe.forward_patches(x, out_dtype=torch.float32)
+    pe.set_tf32(False)
+    a2 = pe.forward_patches(x, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(a, a2) and not torch.equal(a, t)
+    xb = x.to(torch.bfloat16)           # bf16 rows are unaffected by the switch
+    pe.set_tf32(True)
+    u = pe.forward_patches(xb, out_dtype=torch.float32)
+    pe.set_tf32(False)
+    v = pe.forward_patches(xb, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(u, v)

@@ -74,6 +74,11 @@ class PatchEmbed:
     def set_norm(self, mean: Sequence[float], std: Sequence[float]) -> None:
         B.pe_set_norm(self.h, mean, std)
 
+    def set_tf32(self, enable: bool) -> None:
+        """Opt-in: fp32 patch rows are contracted in tf32 (rows and weight rounded
+        to tf32, fp32 accumulation) instead of bf16."""
+        B.pe_set_tf32(self.h, enable)
+
     def set_temporal_fold(self, enable: bool) -> None:
         """Opt-in: single-frame items use the summed temporal slices of the weight
         (half the contraction; one more bf16 rounding per weight term)."""

@@ -29,7 +29,7 @@ EXPORTS = (
     "pe_create", "pe_set_weight", "pe_set_norm", "pe_forward_patches", "pe_forward_frames",
     "pe_forward_frames_grouped", "pe_forward_frames_grouped_noalloc", "pe_patchify", "pe_num_patches", "pe_last_error",
     "pe_status_string", "pe_destroy", "pe_device", "pe_profile_begin", "pe_profile_end",
-    "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos",
+    "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos", "pe_set_tf32",
 )
 
 
@@ -61,6 +61,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_set_weight": ([vp, vp, i32, vp, i32, vp], i32),
         "pe_set_norm": ([vp, f32p, f32p], i32),
         "pe_set_temporal_fold": ([vp, i32], i32),
+        "pe_set_tf32": ([vp, i32], i32),
         "pe_forward_patches": ([vp, vp, i32, i64, vp, i32, vp], i32),
         "pe_forward_patches_pos": ([vp, vp, i32, i64, vp, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped_pos": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp, i32, vp],
@@ -134,6 +135,10 @@ def pe_set_norm(h: int, mean: Sequence[float], std: Sequence[float]) -> None:
 
 def pe_set_temporal_fold(h: int, enable: bool) -> None:
     _check("pe_set_temporal_fold", load().pe_set_temporal_fold(h, int(bool(enable))))
+
+
+def pe_set_tf32(h: int, enable: bool) -> None:
+    _check("pe_set_tf32", load().pe_set_tf32(h, int(bool(enable))))
 
 
 def pe_forward_patches(h: int, x_ptr: int, x_dt: int, N: int, out_ptr: int, out_dt: int, stream: int) -> None:

@@ -31,6 +31,9 @@ struct pe_handle {
     uint16_t *wpack_t = nullptr; // dev [E, 2*Kh] bf16, slice-major (tp == 2 only)
     uint16_t *wpack_fold = nullptr; // dev [E, Kh] bf16, both slices summed (tp == 2 only)
     bool fold = false;          // pe_set_temporal_fold
+    uint32_t *wpack32 = nullptr; // dev [E, Kp32] fp32 words, tf32-rounded, view order
+    int Kp32 = 0;               // K rounded up to 32
+    bool tf32 = false;          // pe_set_tf32
     float *bias = nullptr;      // dev [E] fp32 (has_bias)
     int *err = nullptr;         // dev error word
     float mean[4] = {0, 0, 0, 0};
@@ -39,6 +42,7 @@ struct pe_handle {
     CUtensorMap tmap_wf[3];     // same for the frames-order weight
     CUtensorMap tmap_wt[3];     // same for the slice-major weight
     CUtensorMap tmap_wfold[3];  // same for the folded weight
+    CUtensorMap tmap_w32[3];    // same for the tf32 weight (32 fp32 columns per box)
     int num_sms = 0;
     int smem_optin = 0;
     // item table for grouped calls beyond PE_INLINE_ITEMS
@@ -263,6 +267,10 @@ size_t plan_pipeline(const pe_handle *h, FwdParams &P, int amode, int kcols = -1
         P.b_slot_bytes = 2 * kBStageBytes;   // weight tiles of both slices
     } else if (amode == kAModeTma) {
         P.ksub = 2;                          // 128 k per stage: 8 MMAs per barrier round trip
+        P.b_slot_bytes = 2 * kBStageBytes;
+    } else if (amode == kAModeTmaTf32) {
+        P.num_ksteps = (kcols + 7) / 8;      // tf32 MMAs take 8 k each
+        P.ksub = 2;                          // 64 k per stage (two 32-column fp32 tiles)
         P.b_slot_bytes = 2 * kBStageBytes;
     }
     P.n_b_stages = (P.num_ksteps + 4 * P.ksub - 1) / (4 * P.ksub);
@@ -653,6 +661,8 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
               cudaMemset(h->err, 0, sizeof(int)) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->items_evt, cudaEventDisableTiming) == cudaSuccess;
     if (ok && h->has_bias) ok = cudaMalloc(&h->bias, sizeof(float) * E) == cudaSuccess;
+    h->Kp32 = (int)((K + 31) / 32 * 32);
+    if (ok) ok = cudaMalloc(&h->wpack32, sizeof(uint32_t) * (size_t)E * h->Kp32) == cudaSuccess;
     if (ok && tp == 2) ok = cudaMalloc(&h->wpack_t, sizeof(uint16_t) * (size_t)E * 2 * h->Kh) == cudaSuccess &&
                             cudaMalloc(&h->wpack_fold, sizeof(uint16_t) * (size_t)E * h->Kh) == cudaSuccess;
     if (ok) {
@@ -665,7 +675,9 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
                  (!h->wpack_t || make_tmap_bf16(&h->tmap_wt[i], h->wpack_t, (uint64_t)E, (uint64_t)(2 * h->Kh),
                                                 (uint64_t)(2 * h->Kh), boxes[i])) &&
                  (!h->wpack_fold || make_tmap_bf16(&h->tmap_wfold[i], h->wpack_fold, (uint64_t)E, (uint64_t)h->Kh,
-                                                   (uint64_t)h->Kh, boxes[i]));
+                                                   (uint64_t)h->Kh, boxes[i])) &&
+                 make_tmap(&h->tmap_w32[i], h->wpack32, true, (uint64_t)E, (uint64_t)h->Kp32, (uint64_t)h->Kp32,
+                           boxes[i], 32, CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (!ok) { pe_destroy(h); return PE_ERR_CUDA; }
     *out = h;
@@ -680,6 +692,7 @@ void pe_destroy(pe_handle *h) {
     if (h->wpack_f) cudaFree(h->wpack_f);
     if (h->wpack_t) cudaFree(h->wpack_t);
     if (h->wpack_fold) cudaFree(h->wpack_fold);
+    if (h->wpack32) cudaFree(h->wpack32);
     if (h->bias) cudaFree(h->bias);
     if (h->err) cudaFree(h->err);
     if (h->items_dev) cudaFree(h->items_dev);
@@ -718,7 +731,16 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
                                                           nullptr, h->E, h->C, h->tp, h->p, h->Kh, 3, h->Kh);
         if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
     }
+    pe_pack_weight_tf32_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, h->wpack32, h->E, h->K, h->Kp32);
+    if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
     h->weight_set = true;
+    return PE_OK;
+}
+
+pe_status pe_set_tf32(pe_handle *h, int enable) {
+    if (!h) return PE_ERR_INVALID_ARG;
+    if (enable && (h->K % 4) != 0) return PE_ERR_UNSUPPORTED;
+    h->tf32 = enable != 0;
     return PE_OK;
 }
 
@@ -772,6 +794,44 @@ pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
     // fp32 rows with K % 8 == 0: cast them to bf16 once into the workspace and
     // run the TMA-fed contraction (PE_PATCHES_PATH=threads keeps the producer
     // warps converting inside the contraction kernel).
+    if (x_dt == PE_F32 && h->tf32) {
+        // tf32 contraction: rows rounded to tf32 once into the workspace, then
+        // kind::tf32 pair MMAs against the tf32-rounded weight (K % 4 == 0).
+        const size_t need = (size_t)N * h->K * 4;
+        cudaStream_t st = (cudaStream_t)stream;
+        if (need > h->stage_bytes) {
+            if (h->stage_rows) {
+                if (cudaStreamSynchronize(st) != cudaSuccess) return PE_ERR_CUDA;
+                cudaFree(h->stage_rows);
+            }
+            h->stage_rows = nullptr;
+            h->stage_bytes = 0;
+            if (cudaMalloc(&h->stage_rows, need) != cudaSuccess) return PE_ERR_CUDA;
+            h->stage_bytes = need;
+        }
+        int grid = 0;
+        bool ok = true;
+        plan_tiles(h, P, N, false, grid, ok);
+        if (!ok) return PE_ERR_UNSUPPORTED;
+        const size_t smem = plan_pipeline(h, P, kAModeTmaTf32);
+        CUtensorMap tx, to;
+        if (!make_tmap(&tx, h->stage_rows, true, (uint64_t)N, (uint64_t)h->K, (uint64_t)h->K, kBM, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return PE_ERR_CUDA;
+        if (!make_out_tmap(&to, out, P.out_f32, N, h->E)) return PE_ERR_CUDA;
+        const int64_t n4 = (int64_t)N * h->K / 4;
+        const int cb = (int)std::min<int64_t>((n4 + 255) / 256, (int64_t)h->num_sms * 8);
+        pe_round_tf32_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(x),
+                                                 reinterpret_cast<uint32_t *>(h->stage_rows), n4);
+        if (h->prof_on) ++h->prof_launches;
+        if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+        FwdParams G = P;
+        G.x = h->stage_rows;
+        G.x_f32 = 1;
+        G.x_vec = 1;
+        return finish(
+            launch_fwd<kAModeTmaTf32, 0, false>(h->tmap_w32[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
+    }
     const char *pp = std::getenv("PE_PATCHES_PATH");
     if (x_dt == PE_F32 && (h->K % 8) == 0 && !(pp && std::strcmp(pp, "threads") == 0)) {
         const size_t need = (size_t)N * h->K * 2;

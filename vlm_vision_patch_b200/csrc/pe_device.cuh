@@ -308,6 +308,18 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, 
         : "memory");
 }
 
+// Pair MMA of kind::tf32: A and B are fp32 words read as tf32, K = 8 per
+// instruction (32 bytes of a K-major row, the same descriptor step as bf16).
+__device__ __forceinline__ void mma_tf32_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on the barrier at this shared offset in every CTA of `mask`
 // when all pair MMAs issued so far are done.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
@@ -370,11 +382,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::tf32: D fp32, A and B tf32 (format 2), both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+    return (1u << 4)            // D format: fp32
+           | (2u << 7)          // A format: tf32
+           | (2u << 10)         // B format: tf32
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // ------------------------------------------------------ numerics helpers
 
 // bf16 x 2 packed in a 32-bit word -> two fp32 (exact).
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// fp32 -> the nearest tf32 value (ties away from zero), as an fp32 word whose
+// 13 low mantissa bits are zero.
+__device__ __forceinline__ uint32_t round_tf32(float v) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
+    return r;
+}
 
 // Two fp32 -> bf16 x 2 (round to nearest even), `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -32,7 +32,9 @@ namespace pe {
 
 constexpr int kThreads = 640;       // 20 warps (A produced by threads)
 constexpr int kThreadsTma = 320;    // 10 warps (A fetched by TMA)
-__host__ __device__ constexpr int threads_for(int amode) { return (amode == 0 || amode == 3) ? kThreadsTma : kThreads; }
+__host__ __device__ constexpr int threads_for(int amode) {
+    return (amode == 0 || amode == 3 || amode == 5) ? kThreadsTma : kThreads;
+}
 constexpr int kStreamProdWarp0 = 8;   // kAModeTmaStream: warps 8..15 produce rows
 constexpr int kStreamProdWarps = 8;
 constexpr int kBM = 128;           // rows per CTA (pair tile: 256 rows)
@@ -55,9 +57,14 @@ constexpr int kBStageBytes = (kMaxBN / 2) * kBK * 2;   // 16 KB: this CTA's half
 //                      back by TMA once their M-block is complete: single-frame
 //                      rows as in kAModeTmaShared (DUPALL), otherwise both
 //                      slices per row against the slice-major weight.
-enum AMode : int { kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2, kAModeTmaShared = 3, kAModeTmaStream = 4 };
+//   kAModeTmaTf32      TMA tiles of fp32 rows (tf32-rounded) against the
+//                      tf32-rounded fp32 weight, kind::tf32 MMAs (K = 8 each)
+enum AMode : int {
+    kAModeTma = 0, kAModePatchThreads = 1, kAModeFrames = 2, kAModeTmaShared = 3, kAModeTmaStream = 4,
+    kAModeTmaTf32 = 5
+};
 __host__ __device__ constexpr bool tma_fed(int amode) {
-    return amode == kAModeTma || amode == kAModeTmaShared || amode == kAModeTmaStream;
+    return amode == kAModeTma || amode == kAModeTmaShared || amode == kAModeTmaStream || amode == kAModeTmaTf32;
 }
 
 struct ItemDesc {
@@ -835,14 +842,14 @@ __device__ __forceinline__ void produce_rows_stream(const FwdParams &P, int pw, 
 //   also holds the weight tiles of slice 0 and slice 1 at the same k, so the
 //   rows are fetched once for the two temporal slices they stand for.
 //   KSUB == 2: 128 k per stage (8 MMAs per barrier round trip).
-template <int SLICES, int KSUB>
+template <int SLICES, int KSUB, bool TF32 = false>
 __device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring, uint64_t *full_b,
                                               uint64_t *empty_b, uint64_t *tfull, uint64_t *tempty,
                                               uint64_t *mma_done, uint32_t tmem_base, volatile int *abort) {
     constexpr uint16_t kPair = 0x3;
     constexpr uint32_t kTile = (uint32_t)kBStageBytes >> 4;   // one 16 KB tile, descriptor units
     constexpr int KS = 4 * KSUB;                               // k-steps per stage
-    const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
+    const uint32_t idesc = TF32 ? idesc_tf32_f32(2 * kBM, P.bn) : idesc_bf16_f32(2 * kBM, P.bn);
     const uint64_t a0 = smem_desc(smem_addr(a_ring), 16, 1024, kLayoutSw128);
     const uint64_t b0 = smem_desc(smem_addr(b_ring), 16, 1024, kLayoutSw128);
     const uint32_t a_lo0 = (uint32_t)a0, b_lo0 = (uint32_t)b0;
@@ -854,8 +861,12 @@ __device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_rin
         const int sub = ks / 4, j = ks % 4;
         const uint64_t ad = desc_with_lo(a0, a_lo + (uint32_t)sub * kTile + 2u * j);
         const uint32_t bl = b_lo + (uint32_t)(sub * SLICES) * kTile + 2u * j;
-        mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, bl), idesc, first ? 0u : 1u);
-        if constexpr (SLICES == 2) mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, bl + kTile), idesc, 1u);
+        if constexpr (TF32) {
+            mma_tf32_pair(d_tmem, ad, desc_with_lo(b0, bl), idesc, first ? 0u : 1u);
+        } else {
+            mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, bl), idesc, first ? 0u : 1u);
+            if constexpr (SLICES == 2) mma_bf16_pair(d_tmem, ad, desc_with_lo(b0, bl + kTile), idesc, 1u);
+        }
     };
     for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
         if (!mbar_wait(smem_addr(&tempty[acc]), accph ^ 1, abort)) return;
@@ -1029,8 +1040,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     const uint32_t adst = smem_addr(a_ring + (size_t)bs * P.a_stage_bytes);
                     const uint32_t bdst = smem_addr(b_ring + (size_t)bs * P.b_slot_bytes);
                     const int wrow = n_blk * P.bn + (int)rank * (P.bn / 2);
+                    // k columns per 128-byte tile row: 64 bf16 or 32 fp32 (tf32)
+                    constexpr int kBKe = (AMODE == kAModeTmaTf32) ? kBK / 2 : kBK;
                     for (int sub = 0; sub < ksub; ++sub) {
-                        const int kx = (kb * ksub + sub) * kBK;
+                        const int kx = (kb * ksub + sub) * kBKe;
                         if (kTmaA)
                             tma_load_2d_pair(adst + (uint32_t)sub * kBStageBytes, &tmap_x, fb0 + 8u * bs, kx,
                                              m_blk * (2 * kBM) + (int)rank * kBM, pol_x);
@@ -1048,7 +1061,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             constexpr int KSA = (AMODE == kAModeFrames) ? (PT ? PT / 2 : 0) : 4;
             if constexpr (kTmaA) {
                 constexpr int kSl = (AMODE == kAModeTmaShared || (AMODE == kAModeTmaStream && DUPALL)) ? 2 : 1;
-                if (kSl == 1 && P.ksub == 2)
+                if constexpr (AMODE == kAModeTmaTf32)
+                    mma_issue_tma<1, 2, true>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base,
+                                              abort);
+                else if (kSl == 1 && P.ksub == 2)
                     mma_issue_tma<kSl, 2>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
                 else
                     mma_issue_tma<kSl, 1>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
@@ -1393,6 +1409,33 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
         bulk_store(A + m0 * row_elems, smem_addr(prep_smem), (uint32_t)(rows * row_elems * 2));
         bulk_commit();
         bulk_wait<0>();
+    }
+}
+
+// fp32 patch rows -> tf32-rounded fp32 rows (nearest, ties away from zero)
+// for the tf32 contraction.  4 elements per thread.
+__global__ void pe_round_tf32_kernel(const float *__restrict__ x, uint32_t *__restrict__ A, int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(x) + i);
+        *(reinterpret_cast<uint4 *>(A) + i) = make_uint4(round_tf32(a.x), round_tf32(a.y), round_tf32(a.z), round_tf32(a.w));
+    }
+}
+
+// The weight for the tf32 contraction: W[e, k] (view order) rounded to tf32,
+// as fp32 words, zero for K <= k < ld.
+__global__ void pe_pack_weight_tf32_kernel(const void *w, int w_f32, uint32_t *wpack, int E, int K, int ld) {
+    const int64_t total = (int64_t)E * ld;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = idx / ld;
+        const int k = (int)(idx - e * ld);
+        uint32_t v = 0u;
+        if (k < K) {
+            const float f = w_f32 ? reinterpret_cast<const float *>(w)[e * K + k]
+                                  : __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(w)[e * K + k] << 16);
+            v = round_tf32(f);
+        }
+        wpack[idx] = v;
     }
 }
 
