@@ -68,6 +68,9 @@ def _load():
             f32p, ctypes.c_int64, f32p, f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, u8p, f64p, f64p]
         lib.oracle_conv3d_patches_fp32.argtypes = lib.oracle_conv3d_patches.argtypes
+        lib.oracle_patch_merger.argtypes = [
+            f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, f32p, f32p, ctypes.c_double, f32p, f32p, f32p, f32p,
+            ctypes.c_int, u8p, f64p, f64p]
         lib.oracle_conv3d_frames.argtypes = [
             f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, f32p, f32p, f32p, f32p, ctypes.c_int, ctypes.c_int,
@@ -160,6 +163,33 @@ def conv3d_patches_fp32(x, w, bias, C: int, tp: int, p: int, row_mask=None
                                        _p(b, ctypes.c_float), E, C, tp, p,
                                        _p(m, ctypes.c_uint8), _p(out, ctypes.c_double),
                                        _p(mag, ctypes.c_double))
+    return out, mag
+
+
+def patch_merger(x, m2: int, gamma, beta, eps: float, w1, b1, w2, b2, v_mask=None
+                 ) -> Tuple[np.ndarray, np.ndarray]:
+    """PatchMerger on rows in merge order: x [V*m2, E] -> (out [V, H], absdot [V, H])
+    fp64 (LayerNorm, concat of m2 rows, fc1 + exact GELU, fc2; the LayerNorm and
+    GELU outputs and the weights rounded to bf16).  Masked-out rows are NaN."""
+    x = _f32(x)
+    E = int(x.shape[1])
+    assert x.shape[0] % m2 == 0
+    V = x.shape[0] // m2
+    D = E * m2
+    w1 = _f32(w1)
+    w2 = _f32(w2)
+    H = int(w2.shape[0])
+    assert w1.shape == (D, D) and w2.shape == (H, D)
+    gm, bt = _f32(gamma), _f32(beta)                 # held for the duration of the call
+    b1a = None if b1 is None else _f32(b1)
+    b2a = None if b2 is None else _f32(b2)
+    out = np.full((V, H), np.nan)
+    mag = np.full((V, H), np.nan)
+    m = _mask(v_mask, V)
+    _load().oracle_patch_merger(_p(x, ctypes.c_float), V, E, m2, _p(gm, ctypes.c_float), _p(bt, ctypes.c_float),
+                                float(eps), _p(w1, ctypes.c_float), _p(b1a, ctypes.c_float), _p(w2, ctypes.c_float),
+                                _p(b2a, ctypes.c_float), H, _p(m, ctypes.c_uint8), _p(out, ctypes.c_double),
+                                _p(mag, ctypes.c_double))
     return out, mag
 
 

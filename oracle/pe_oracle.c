@@ -287,3 +287,66 @@ int oracle_patchify(const float *frames, int T, int H, int W, int gt, int gh, in
     free(vol);
     return 0;
 }
+
+/* PatchMerger (mytransformer README §3.2 and §4.1: LayerNorm, then the 2x2
+ * neighbouring patch rows concatenated, 1280 x 4 = 5120, then a GELU MLP
+ * 5120 -> 5120 -> hidden).  x: [N, E] fp32 rows in merge order (N = V * m*m),
+ * so rows 4v .. 4v+3 form merged row v.  Compute precision mirrors a bf16
+ * pipeline: the LayerNorm output and the GELU output are rounded to bf16,
+ * weights are rounded to bf16, everything else is fp64.  LayerNorm:
+ * (x - mean) / sqrt(var + eps) * gamma + beta with the biased variance over
+ * the E features.  GELU: the exact form 0.5 * y * (1 + erf(y / sqrt(2))).
+ * out: [V, H] fp64; absdot: [V, H] sum over k of |g_k * w2_k| (g = the bf16
+ * GELU output), for tolerance scaling.  v_mask: optional [V] row selector. */
+void oracle_patch_merger(const float *x, int64_t V, int E, int m2, const float *gamma, const float *beta,
+                         double eps, const float *w1, const float *b1, const float *w2, const float *b2,
+                         int H, const uint8_t *v_mask, double *out, double *absdot)
+{
+    const int64_t D = (int64_t)E * m2;
+    float *w1b = (float *)malloc(sizeof(float) * (size_t)(D * D));
+    float *w2b = (float *)malloc(sizeof(float) * (size_t)(H * D));
+    oracle_bf16_round_array(w1, w1b, D * D);
+    oracle_bf16_round_array(w2, w2b, (int64_t)H * D);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t v = 0; v < V; ++v) {
+        if (v_mask && !v_mask[v])
+            continue;
+        double *hln = (double *)malloc(sizeof(double) * (size_t)D);
+        double *g = (double *)malloc(sizeof(double) * (size_t)D);
+        for (int q = 0; q < m2; ++q) {                 /* LayerNorm of each of the m*m rows */
+            const float *row = x + (v * m2 + q) * (int64_t)E;
+            double mean = 0.0, var = 0.0;
+            for (int e = 0; e < E; ++e) mean += (double)row[e];
+            mean /= E;
+            for (int e = 0; e < E; ++e) var += ((double)row[e] - mean) * ((double)row[e] - mean);
+            var /= E;
+            const double inv = 1.0 / sqrt(var + eps);
+            for (int e = 0; e < E; ++e) {
+                const double y = ((double)row[e] - mean) * inv * (double)gamma[e] + (double)beta[e];
+                hln[(int64_t)q * E + e] = (double)oracle_bf16_round((float)y);
+            }
+        }
+        for (int64_t j = 0; j < D; ++j) {              /* fc1 + GELU */
+            double acc = 0.0;
+            for (int64_t k = 0; k < D; ++k) acc += hln[k] * (double)w1b[j * D + k];
+            const double y = acc + (b1 ? (double)b1[j] : 0.0);
+            const double gl = 0.5 * y * (1.0 + erf(y / sqrt(2.0)));
+            g[j] = (double)oracle_bf16_round((float)gl);
+        }
+        for (int h = 0; h < H; ++h) {                  /* fc2 */
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < D; ++k) {
+                const double t = g[k] * (double)w2b[(int64_t)h * D + k];
+                acc += t;
+                mag += fabs(t);
+            }
+            out[v * H + h] = acc + (b2 ? (double)b2[h] : 0.0);
+            if (absdot)
+                absdot[v * H + h] = mag;
+        }
+        free(hln);
+        free(g);
+    }
+    free(w1b);
+    free(w2b);
+}

@@ -44,6 +44,12 @@ MUTANTS = {
                                "const double xv = (double)oracle_bf16_round(x[n * K + k]);"),
     "fp32_form_neighbour_column": ("const double xv = (double)x[n * K + k];",
                                    "const double xv = (double)x[n * K + (k ^ 1)];"),
+    "merger_window_columns_transposed": ("hln[(int64_t)q * E + e] = (double)oracle_bf16_round((float)y);",
+                                         "hln[(int64_t)e * m2 + q] = (double)oracle_bf16_round((float)y);"),
+    "merger_unbiased_variance": ("            var /= E;\n", "            var /= (E - 1);\n"),
+    "merger_gelu_without_half": ("const double gl = 0.5 * y * (1.0 + erf(y / sqrt(2.0)));",
+                                 "const double gl = y * (1.0 + erf(y / sqrt(2.0)));"),
+    "merger_ln_drops_beta": ("* (double)gamma[e] + (double)beta[e];", "* (double)gamma[e];"),
     "patchify_drops_time_offset": ("const int64_t tau = g_t * tp + t;\n                        rows",
                                    "const int64_t tau = g_t * tp;\n                        rows"),
 }

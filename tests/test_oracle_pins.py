@@ -8,6 +8,7 @@ None of these re-types the oracle's own formula.  Each pin is one of
     linearity, exact integer arithmetic, the duplicated-frame identity).
 """
 import json
+import math
 import os
 
 import numpy as np
@@ -342,3 +343,58 @@ def test_patches_fp32_equals_rounded_form_on_bf16_values():
     a, ma = oracle.conv3d_patches_fp32(x, w, None, C, tp, p)
     b, mb = oracle.conv3d_patches(x, w, None, C, tp, p)
     assert np.array_equal(a, b) and np.array_equal(ma, mb)
+
+
+# ------------------------------------------------------------- PatchMerger
+
+def _bf16(t):
+    return t.to(torch.bfloat16).double()
+
+
+@pytest.mark.parametrize("E,m2,H,with_bias", [(8, 4, 5, True), (12, 4, 3, False), (6, 1, 4, True)])
+def test_patch_merger_matches_torch(E, m2, H, with_bias):
+    """LayerNorm -> concat of m2 rows -> fc1 -> exact GELU -> fc2, against torch's
+    fp64 layer_norm / linear / gelu library routines with the same bf16 roundings
+    of the LayerNorm output, the GELU output and the weights (mytransformer
+    README §3.2 and §4.1)."""
+    g = torch.Generator().manual_seed(400 + E + m2)
+    V = 5
+    D = E * m2
+    x = torch.randn(V * m2, E, generator=g) * 2.0 + 0.5
+    gamma = torch.randn(E, generator=g) * 0.5 + 1.0
+    beta = torch.randn(E, generator=g) * 0.1
+    w1 = torch.randn(D, D, generator=g) * 0.2
+    w2 = torch.randn(H, D, generator=g) * 0.2
+    b1 = torch.randn(D, generator=g) * 0.1 if with_bias else None
+    b2 = torch.randn(H, generator=g) * 0.1 if with_bias else None
+    eps = 1e-6
+    out, mag = oracle.patch_merger(x, m2, gamma, beta, eps, w1, b1, w2, b2)
+    ln = torch.nn.functional.layer_norm(x.double(), (E,), gamma.double(), beta.double(), eps)
+    h = _bf16(ln.float()).view(V, D)
+    y = torch.nn.functional.linear(h, _bf16(w1), None if b1 is None else b1.double())
+    gl = _bf16(torch.nn.functional.gelu(y).float())
+    ref = torch.nn.functional.linear(gl, _bf16(w2), None if b2 is None else b2.double())
+    assert np.allclose(out, ref.numpy(), rtol=1e-9, atol=1e-9)
+    refmag = torch.nn.functional.linear(gl.abs(), _bf16(w2).abs())
+    assert np.allclose(mag, refmag.numpy(), rtol=1e-9, atol=1e-9)
+
+
+def test_patch_merger_concatenates_the_window_rows_in_order():
+    """With fc1 = identity and fc2 selecting one input column, the output is that
+    column of the (bf16) LayerNorm of the right row: row q of a window lands at
+    columns q*E .. q*E+E-1 of the merged row."""
+    E, m2, V = 4, 4, 3
+    D = E * m2
+    x = workloads.normal((V * m2, E), 410)
+    gamma, beta = torch.ones(E), torch.zeros(E)
+    w1 = torch.eye(D) * 64.0      # fc1 passes each merged column through, scaled
+    ln = torch.nn.functional.layer_norm(x.double(), (E,), None, None, 1e-6)
+    for col in (0, E + 1, 2 * E + 3, 3 * E + 2):
+        w2 = torch.zeros(1, D)
+        w2[0, col] = 1.0
+        out, _ = oracle.patch_merger(x, m2, gamma, beta, 1e-6, w1, None, w2, None)
+        q, e = divmod(col, E)
+        for v in range(V):
+            y = 64.0 * float(_bf16(ln[v * m2 + q, e].float()))
+            gl = 0.5 * y * (1.0 + math.erf(y / math.sqrt(2.0)))
+            assert out[v, 0] == float(torch.tensor(gl, dtype=torch.float32).to(torch.bfloat16).double())
