@@ -432,6 +432,97 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def run_merger(args, rank, world, local):
+    """--merger: the PatchMerger (LayerNorm, 2x2 concat, GELU MLP 5120 -> 5120 ->
+    1536, synthetic N(0, 1/sqrt(D)) weights) on the workload's PatchEmbed output
+    (computed once, untimed).  A step is one merger forward; the roofline
+    object describes its dominant kernel, fc1."""
+    import vlm_vision_patch_b200 as vp
+    from vlm_vision_patch_b200 import _binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    wl = workloads.ALL[args.workload]()
+    pe = vp.PatchEmbed(wl.E, wl.C, wl.tp, wl.p, wl.bias is not None)
+    pe.set_weight(wl.weight.to(dev), None if wl.bias is None else wl.bias.to(dev))
+    pe.set_norm(wl.mean, wl.std)
+    if wl.patches is not None:
+        x = pe.forward_patches(wl.patches.to(dev))
+    else:
+        x = pe.forward_frames_grouped([it.frames.to(dev) for it in wl.items], [it.grid for it in wl.items], wl.merge)
+    m, H = 2, 1536
+    E, D = wl.E, wl.E * 4
+    V = x.shape[0] // 4
+    x = x[: V * 4]
+    gen = torch.Generator().manual_seed(77)
+    mk = lambda *shape, std: (torch.randn(*shape, generator=gen) * std).to(torch.bfloat16).to(dev)
+    gamma = (1.0 + torch.randn(E, generator=gen) * 0.1).to(torch.bfloat16).to(dev)
+    beta, b1, b2 = mk(E, std=0.05), mk(D, std=0.02), mk(H, std=0.02)
+    w1, w2 = mk(D, D, std=D ** -0.5), mk(H, D, std=D ** -0.5)
+    pm = vp.PatchMerger(E, m, H, 1e-6)
+    pm.set_weights(gamma, beta, w1, b1, w2, b2)
+    out = torch.empty((V, H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        pm.forward(x, out=out)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    B.pe_merger_profile_begin(pm.h, 2 * args.steps)
+    with ClockSampler(local) as clk:
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        for a, b in evs:
+            flush_buf.zero_()
+            a.record(stream)
+            pm.forward(x, out=out)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+    times = [a.elapsed_time(b) for a, b in evs]
+    lin, launches = B.pe_merger_profile_end(pm.h, 2 * args.steps)
+    if pm.last_error() != 0:
+        raise RuntimeError("device pipeline timeout in the merger")
+    total_max_ms = max_over_ranks(sum(times), pg, dev)
+    value = weak_scaling_value(x.shape[0], args.steps, world, total_max_ms)
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        flop = 2.0 * V * (D * D + D * H)
+        mean_ms = statistics.mean(times)
+        fc1 = [lin[i] for i in range(0, len(lin), 2)]
+        fc1_ms = statistics.mean(fc1)
+        achieved = 2.0 * V * D * D / (fc1_ms / 1e3) / 1e12
+        print(json.dumps({
+            "metric": "PatchMerger patches/s and TFLOP/s (% of B200 dense bf16 peak), 1 GPU", "value": value,
+            "unit": "patches/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (PatchEmbed output of the workload, "
+            "seeded N(0, 1/sqrt(D)) merger weights)",
+            "config": {"workload": "patch_merger_" + wl.name, "rows_in": int(x.shape[0]), "rows_out": V, "E": E,
+                       "D": D, "H": H, "l2": "flushed before every timed step"},
+            "tflops": flop / (mean_ms / 1e3) / 1e12,
+            "kernel_ms": {"fc1_mean": fc1_ms, "fc2_mean": statistics.mean(lin[1::2]) if len(lin) > 1 else None},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "pe_fwd_kernel (merger fc1 + GELU)",
+                         "peak_source": f"{src} bf16 dense (burst)"},
+            "cpu_baseline": None,
+            "e2e": None, "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
+    if pg:
+        pg.destroy_process_group()
+    pm.close()
+    pe.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -444,6 +535,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the cuBLAS context timing")
+    ap.add_argument("--merger", action="store_true",
+                    help="time the PatchMerger on the workload's PatchEmbed output instead of the PatchEmbed")
     ap.add_argument("--tf32", action="store_true",
                     help="opt-in tf32 contraction of fp32 patch rows (the fp32 workloads); dtype reads tf32")
     ap.add_argument("--fold", action="store_true",
@@ -455,6 +548,8 @@ def main(argv=None):
     rank, world, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.merger:
+        return run_merger(args, rank, world, local)
     return run_ours(args, rank, world, local)
 
 

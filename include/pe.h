@@ -322,6 +322,63 @@ void pe_destroy(pe_handle *h);
 /* Device this handle was created on, or -1 for NULL. */
 int pe_device(const pe_handle *h);
 
+/* ------------------------------------------------------------------------
+ * PatchMerger -- the step that consumes the PatchEmbed rows in merge order
+ * (mytransformer README §3.2 and §4.1): LayerNorm of each row, the m*m rows of
+ * a merge window concatenated (1280 x 4 = 5120 for Qwen2-VL), then a GELU MLP
+ * D -> D -> H (D = E*m*m; 5120 -> 5120 -> 1536).  Readings where the page is
+ * silent: an affine LayerNorm (gamma, beta) with the biased variance and the
+ * given eps (1e-6 for Qwen2-VL), the exact erf GELU, bias on both linear
+ * layers optional.  Compute: bf16 operands on the tensor cores with fp32
+ * accumulation; the LayerNorm output and the GELU output are stored as bf16.
+ */
+typedef struct pe_merger pe_merger;
+
+/*
+ * pe_merger_create -- E: rows' width (multiple of 8); m: merge size (1..4);
+ * H: output width (multiple of 8, >= 16); eps > 0.  D = E*m*m must be a
+ * multiple of 64 and at most 65536.  Binds to the current CUDA device.
+ * Errors: PE_ERR_INVALID_ARG, PE_ERR_UNSUPPORTED, PE_ERR_CUDA.
+ */
+pe_status pe_merger_create(int E, int m, int H, float eps, pe_merger **out);
+
+/*
+ * pe_merger_set_weights -- device pointers, all of dtype dt (copied and packed;
+ * the caller keeps ownership): gamma, beta [E]; w1 [D, D] and w2 [H, D] in the
+ * nn.Linear [out, in] layout; b1 [D] and b2 [H] or NULL.  16-byte aligned.
+ * Asynchronous on stream.  Errors: PE_ERR_INVALID_ARG, PE_ERR_DTYPE,
+ * PE_ERR_ALIGN, PE_ERR_CUDA.
+ */
+pe_status pe_merger_set_weights(pe_merger *pm, const void *gamma, const void *beta, const void *w1,
+                                const void *b1, const void *w2, const void *b2, pe_dtype dt,
+                                pe_stream_t stream);
+
+/*
+ * pe_merger_forward -- x: dev [N, E] bf16 rows in merge order (the PatchEmbed
+ * output); N a multiple of m*m (N = 0: nothing is launched).  out: dev
+ * [N / (m*m), H] of dtype out_dt.  Three launches on stream: LayerNorm, fc1
+ * with the GELU in its epilogue, fc2.  The intermediate rows live in the
+ * merger's grow-only workspace, so calls must be serialised on one stream.
+ * Errors: PE_ERR_INVALID_ARG, PE_ERR_DTYPE, PE_ERR_ALIGN, PE_ERR_NO_WEIGHT,
+ * PE_ERR_SHAPE, PE_ERR_CUDA.
+ */
+pe_status pe_merger_forward(pe_merger *pm, const void *x, int64_t N, void *out, pe_dtype out_dt,
+                            pe_stream_t stream);
+
+/*
+ * pe_merger_profile_begin / pe_merger_profile_end -- as pe_profile_begin /
+ * pe_profile_end, around each of the two linear layers of every forward call
+ * (so the times alternate fc1, fc2); launches counts all three kernels.
+ */
+pe_status pe_merger_profile_begin(pe_merger *pm, int max_calls);
+pe_status pe_merger_profile_end(pe_merger *pm, float *ms, int *n, int64_t *launches);
+
+/* pe_merger_last_error -- as pe_last_error, for the merger's kernels. */
+pe_status pe_merger_last_error(pe_merger *pm);
+
+/* pe_merger_destroy -- waits for the device, frees everything; NULL is a no-op. */
+void pe_merger_destroy(pe_merger *pm);
+
 #ifdef __cplusplus
 }
 #endif

@@ -594,3 +594,79 @@ def test_tf32_switch_is_per_handle_and_reversible():
     v = pe.forward_patches(xb, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(u, v)
+
+
+# ------------------------------------------------------------- PatchMerger
+
+from vlm_vision_patch_b200 import PatchMerger  # noqa: E402
+
+
+def _merger_case(E, m, H, V, bias, wdt, seed):
+    m2 = m * m
+    D = E * m2
+    x = (workloads.normal((V * m2, E), seed) * 0.7 + 0.05).to(torch.bfloat16)
+    gamma = (1.0 + workloads.normal((E,), seed + 1, std=0.1)).to(wdt)
+    beta = workloads.normal((E,), seed + 2, std=0.05).to(wdt)
+    w1 = workloads.normal((D, D), seed + 3, std=D ** -0.5).to(wdt)
+    w2 = workloads.normal((H, D), seed + 4, std=D ** -0.5).to(wdt)
+    b1 = workloads.normal((D,), seed + 5, std=0.02).to(wdt) if bias else None
+    b2 = workloads.normal((H,), seed + 6, std=0.02).to(wdt) if bias else None
+    return x, gamma, beta, w1, b1, w2, b2
+
+
+@pytest.mark.parametrize("E,m,H,V,bias,wdt,out_dtype", [
+    (1280, 2, 1536, 64, True, torch.bfloat16, torch.bfloat16),    # Qwen2-VL: 5120 -> 5120 -> 1536
+    (1152, 2, 1024, 37, False, torch.float32, torch.float32),     # ragged V, fp32 weights
+    (64, 1, 128, 300, True, torch.bfloat16, torch.float32),       # m = 1
+])
+def test_patch_merger(E, m, H, V, bias, wdt, out_dtype):
+    """GPU PatchMerger vs the oracle.  Tolerance: the GPU rounds the LayerNorm
+    and GELU outputs to bf16 like the oracle, but from fp32 rather than fp64
+    values, so an element of either may land one bf16 ulp away; through fc2
+    that is at most 2^-8 * sum|g w2| per output, doubled for the fc1 stage and
+    widened for fp32 accumulation: |err| <= 1e-2 * sum|g w2| (+ 1 bf16 ulp for
+    bf16 output).  The typical error must also stay well inside it."""
+    x, gamma, beta, w1, b1, w2, b2 = _merger_case(E, m, H, V, bias, wdt, 500 + E + V)
+    pm = PatchMerger(E, m, H, 1e-6)
+    dev = lambda t: None if t is None else t.to(DEV).contiguous()
+    pm.set_weights(dev(gamma), dev(beta), dev(w1), dev(b1), dev(w2), dev(b2))
+    out = pm.forward(x.to(DEV), out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert pm.last_error() == 0
+    ref, mag = oracle.patch_merger(x, m * m, gamma, beta, 1e-6, w1, b1, w2, b2)
+    r = assert_within_tolerance(out, ref, mag, what=f"merger {E},{m},{H},{V}", rel=1e-2)
+    err = np.abs(out.detach().cpu().double().numpy() - ref) / np.maximum(mag, 1e-30)
+    assert np.median(err) < 1e-3, np.median(err)
+    assert r <= 1.0
+    pm.close()
+
+
+def test_patch_merger_full_size_sampled():
+    """The merger on config-4-sized input (59204 patch rows -> 14801 merged rows,
+    5120 -> 5120 -> 1536), sampled merged rows incl. the first and last."""
+    E, m, H = 1280, 2, 1536
+    V = 14801
+    x, gamma, beta, w1, b1, w2, b2 = _merger_case(E, m, H, V, True, torch.bfloat16, 600)
+    pm = PatchMerger(E, m, H, 1e-6)
+    pm.set_weights(*(None if t is None else t.to(DEV) for t in (gamma, beta, w1, b1, w2, b2)))
+    out = pm.forward(x.to(DEV))
+    torch.cuda.synchronize()
+    assert pm.last_error() == 0
+    rows = sample_rows(V, 24, 601)
+    ref, mag = oracle.patch_merger(x, 4, gamma, beta, 1e-6, w1, b1, w2, b2, v_mask=mask_of(rows, V))
+    assert_within_tolerance(out, ref, mag, rows=rows, what="merger full size", rel=1e-2)
+    pm.close()
+
+
+def test_patch_merger_errors():
+    pm = PatchMerger(64, 2, 128)
+    x = torch.zeros(8, 64, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(PEError) as e:
+        pm.forward(x)
+    assert e.value.status == "PE_ERR_NO_WEIGHT"
+    z = lambda *s: torch.zeros(*s, dtype=torch.bfloat16, device=DEV)
+    pm.set_weights(z(64), z(64), z(256, 256), None, z(128, 256), None)
+    with pytest.raises(PEError) as e:
+        pm.forward(torch.zeros(6, 64, dtype=torch.bfloat16, device=DEV))   # 6 rows: not whole 2x2 windows
+    assert e.value.status == "PE_ERR_SHAPE"
+    pm.close()

@@ -14,7 +14,7 @@ import torch
 from . import _binding as B
 from ._binding import PE_BF16, PE_F32, PEError, load  # noqa: F401
 
-__all__ = ["PatchEmbed", "PEError", "PE_F32", "PE_BF16", "load", "num_patches"]
+__all__ = ["PatchEmbed", "PatchMerger", "PEError", "PE_F32", "PE_BF16", "load", "num_patches"]
 
 
 def _dt(t: torch.dtype) -> int:
@@ -146,3 +146,46 @@ class PatchEmbed:
                       [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames], grid_thw, merge,
                       _dev(rows, "rows"), _dt(rows.dtype), _stream(stream))
         return rows
+
+
+class PatchMerger:
+    """LayerNorm -> concat of the m*m rows of each merge window -> GELU MLP
+    D -> D -> H on rows in merge order (the PatchEmbed output).  Thin wrapper
+    over the pe_merger_* C calls."""
+
+    def __init__(self, E: int, m: int, H: int, eps: float = 1e-6):
+        self.E, self.m2, self.H = E, m * m, H
+        self.h = B.pe_merger_create(E, m, H, eps)
+
+    def set_weights(self, gamma: torch.Tensor, beta: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor],
+                    w2: torch.Tensor, b2: Optional[torch.Tensor], stream=None) -> None:
+        ts = [gamma, beta, w1, w2] + [t for t in (b1, b2) if t is not None]
+        if len({t.dtype for t in ts}) != 1:
+            raise TypeError("all merger weights must share one dtype")
+        self._keep = ts
+        B.pe_merger_set_weights(self.h, _dev(gamma, "gamma"), _dev(beta, "beta"), _dev(w1, "w1"),
+                                None if b1 is None else _dev(b1, "b1"), _dev(w2, "w2"),
+                                None if b2 is None else _dev(b2, "b2"), _dt(w1.dtype), _stream(stream))
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
+                stream=None) -> torch.Tensor:
+        V = x.shape[0] // self.m2
+        if out is None:
+            out = torch.empty((V, self.H), dtype=out_dtype, device=x.device)
+        B.pe_merger_forward(self.h, _dev(x, "x"), x.shape[0], _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        return out
+
+    def last_error(self) -> int:
+        return B.pe_merger_last_error(self.h)
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            B.pe_merger_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+

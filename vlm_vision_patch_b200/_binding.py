@@ -30,6 +30,8 @@ EXPORTS = (
     "pe_forward_frames_grouped", "pe_forward_frames_grouped_noalloc", "pe_patchify", "pe_num_patches", "pe_last_error",
     "pe_status_string", "pe_destroy", "pe_device", "pe_profile_begin", "pe_profile_end",
     "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos", "pe_set_tf32",
+    "pe_merger_create", "pe_merger_set_weights", "pe_merger_forward", "pe_merger_last_error", "pe_merger_destroy",
+    "pe_merger_profile_begin", "pe_merger_profile_end",
 )
 
 
@@ -62,6 +64,14 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_set_norm": ([vp, f32p, f32p], i32),
         "pe_set_temporal_fold": ([vp, i32], i32),
         "pe_set_tf32": ([vp, i32], i32),
+        "pe_merger_create": ([i32, i32, i32, ctypes.c_float, ctypes.POINTER(vp)], i32),
+        "pe_merger_set_weights": ([vp, vp, vp, vp, vp, vp, vp, i32, vp], i32),
+        "pe_merger_forward": ([vp, vp, i64, vp, i32, vp], i32),
+        "pe_merger_last_error": ([vp], i32),
+        "pe_merger_destroy": ([vp], None),
+        "pe_merger_profile_begin": ([vp, i32], i32),
+        "pe_merger_profile_end": ([vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(i32),
+                                   ctypes.POINTER(ctypes.c_int64)], i32),
         "pe_forward_patches": ([vp, vp, i32, i64, vp, i32, vp], i32),
         "pe_forward_patches_pos": ([vp, vp, i32, i64, vp, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped_pos": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp, i32, vp],
@@ -209,6 +219,42 @@ def pe_profile_end(h: int, max_calls: int):
     launches = ctypes.c_int64(0)
     _check("pe_profile_end", load().pe_profile_end(h, ms, ctypes.byref(n), ctypes.byref(launches)))
     return [float(ms[i]) for i in range(n.value)], int(launches.value)
+
+
+def pe_merger_create(E: int, m: int, H: int, eps: float) -> int:
+    h = ctypes.c_void_p()
+    _check("pe_merger_create", load().pe_merger_create(E, m, H, eps, ctypes.byref(h)))
+    return h.value
+
+
+def pe_merger_set_weights(pm: int, gamma: int, beta: int, w1: int, b1: Optional[int], w2: int, b2: Optional[int],
+                          dt: int, stream: int) -> None:
+    _check("pe_merger_set_weights", load().pe_merger_set_weights(pm, gamma, beta, w1, b1, w2, b2, dt, stream))
+
+
+def pe_merger_forward(pm: int, x_ptr: int, N: int, out_ptr: int, out_dt: int, stream: int) -> None:
+    _check("pe_merger_forward", load().pe_merger_forward(pm, x_ptr, N, out_ptr, out_dt, stream))
+
+
+def pe_merger_profile_begin(pm: int, max_calls: int) -> None:
+    _check("pe_merger_profile_begin", load().pe_merger_profile_begin(pm, max_calls))
+
+
+def pe_merger_profile_end(pm: int, max_calls: int):
+    """Returns (per-linear-layer ms, alternating fc1/fc2; kernels launched)."""
+    ms = (ctypes.c_float * max(1, max_calls))()
+    n = ctypes.c_int(max_calls)
+    launches = ctypes.c_int64(0)
+    _check("pe_merger_profile_end", load().pe_merger_profile_end(pm, ms, ctypes.byref(n), ctypes.byref(launches)))
+    return [float(ms[i]) for i in range(n.value)], int(launches.value)
+
+
+def pe_merger_last_error(pm: int) -> int:
+    return int(load().pe_merger_last_error(pm))
+
+
+def pe_merger_destroy(pm: int) -> None:
+    load().pe_merger_destroy(pm)
 
 
 def pe_last_error(h: int) -> int:

@@ -1091,4 +1091,197 @@ pe_status pe_last_error(pe_handle *h) {
     return v == 0 ? PE_OK : (pe_status)v;
 }
 
+// ---------------------------------------------------------------------------
+// PatchMerger: LayerNorm, the m*m neighbouring rows of a merge window
+// concatenated (they are adjacent in merge order, so [N, E] is [V, m*m*E]
+// without a copy), then fc1 + exact GELU and fc2 on the TMA-fed pair GEMM.
+}  // extern "C"
+
+struct pe_merger {
+    pe_handle core;              // device properties for the shared planners (owns nothing)
+    int E = 0, m2 = 0, H = 0, D = 0;
+    float eps = 1e-6f;
+    bool weights_set = false;
+    uint16_t *w1 = nullptr;      // [D, D] bf16
+    uint16_t *w2 = nullptr;      // [H, D] bf16
+    float *b1 = nullptr, *b2 = nullptr, *gamma = nullptr, *beta = nullptr;
+    bool has_b1 = false, has_b2 = false;
+    int *err = nullptr;
+    CUtensorMap tmap_w1[3], tmap_w2[3];
+    uint16_t *ln_rows = nullptr;  // [N, E] bf16 workspace
+    size_t ln_bytes = 0;
+    uint16_t *hid = nullptr;      // [V, D] bf16 workspace
+    size_t hid_bytes = 0;
+};
+
+namespace {
+
+bool grow(uint16_t **buf, size_t *cap, size_t need, cudaStream_t st) {
+    if (need <= *cap) return true;
+    if (*buf) {
+        if (cudaStreamSynchronize(st) != cudaSuccess) return false;
+        cudaFree(*buf);
+    }
+    *buf = nullptr;
+    *cap = 0;
+    if (cudaMalloc(buf, need) != cudaSuccess) return false;
+    *cap = need;
+    return true;
+}
+
+// One linear layer of the merger on the pair GEMM: out[V, nout] = act(A[V, D] W^T + b).
+pe_status merger_linear(pe_merger *pm, const uint16_t *A, int64_t V, const CUtensorMap *tw3, int nout,
+                        const float *bias, int act, void *out, int out_dt, cudaStream_t st) {
+    FwdParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.E = nout;
+    G.K = pm->D;
+    G.Kpad = pm->D;
+    G.C = 1;
+    G.TP = 1;
+    G.P = 1;
+    G.N = V;
+    G.x = A;
+    G.x_vec = 1;
+    G.bias = bias;
+    G.act = act;
+    G.out_f32 = out_dt == PE_F32;
+    G.err = pm->err;
+    int grid = 0;
+    bool ok = true;
+    plan_tiles(&pm->core, G, V, false, grid, ok);
+    if (!ok) return PE_ERR_UNSUPPORTED;
+    const size_t smem = plan_pipeline(&pm->core, G, kAModeTma, pm->D);
+    CUtensorMap tx, to;
+    if (!make_tmap_bf16(&tx, A, (uint64_t)V, (uint64_t)pm->D, (uint64_t)pm->D, kBM)) return PE_ERR_CUDA;
+    if (!make_out_tmap(&to, out, G.out_f32, V, nout)) return PE_ERR_CUDA;
+    return finish(launch_fwd<kAModeTma, 0, false>(tw3[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
+}
+
+}  // namespace
+
+extern "C" {
+
+pe_status pe_merger_create(int E, int m, int H, float eps, pe_merger **out) {
+    if (!out) return PE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (E < 8 || (E % 8) != 0 || m < 1 || m > 4 || H < 16 || (H % 8) != 0 || !(eps > 0.f)) return PE_ERR_INVALID_ARG;
+    const int64_t D = (int64_t)E * m * m;
+    if ((D % 64) != 0 || D > 65536) return PE_ERR_UNSUPPORTED;
+    pe_merger *pm = new (std::nothrow) pe_merger();
+    if (!pm) return PE_ERR_CUDA;
+    if (cudaGetDevice(&pm->core.dev) != cudaSuccess) { delete pm; return PE_ERR_CUDA; }
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, pm->core.dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, pm->core.dev);
+    if (major != 10 || minor != 0) { delete pm; return PE_ERR_UNSUPPORTED; }
+    cudaDeviceGetAttribute(&pm->core.num_sms, cudaDevAttrMultiProcessorCount, pm->core.dev);
+    cudaDeviceGetAttribute(&pm->core.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, pm->core.dev);
+    pm->E = E;
+    pm->m2 = m * m;
+    pm->H = H;
+    pm->D = (int)D;
+    pm->eps = eps;
+    bool ok = cudaMalloc(&pm->w1, sizeof(uint16_t) * (size_t)(D * D)) == cudaSuccess &&
+              cudaMalloc(&pm->w2, sizeof(uint16_t) * (size_t)H * D) == cudaSuccess &&
+              cudaMalloc(&pm->b1, sizeof(float) * (size_t)D) == cudaSuccess &&
+              cudaMalloc(&pm->b2, sizeof(float) * (size_t)H) == cudaSuccess &&
+              cudaMalloc(&pm->gamma, sizeof(float) * (size_t)E) == cudaSuccess &&
+              cudaMalloc(&pm->beta, sizeof(float) * (size_t)E) == cudaSuccess &&
+              cudaMalloc(&pm->err, sizeof(int)) == cudaSuccess && cudaMemset(pm->err, 0, sizeof(int)) == cudaSuccess;
+    const uint32_t boxes[3] = {32, 64, 128};
+    for (int i = 0; i < 3 && ok; ++i)
+        ok = make_tmap_bf16(&pm->tmap_w1[i], pm->w1, (uint64_t)D, (uint64_t)D, (uint64_t)D, boxes[i]) &&
+             make_tmap_bf16(&pm->tmap_w2[i], pm->w2, (uint64_t)H, (uint64_t)D, (uint64_t)D, boxes[i]);
+    if (!ok) { pe_merger_destroy(pm); return PE_ERR_CUDA; }
+    *out = pm;
+    return PE_OK;
+}
+
+void pe_merger_destroy(pe_merger *pm) {
+    if (!pm) return;
+    DeviceGuard g(pm->core.dev);
+    cudaDeviceSynchronize();
+    for (void *p : {(void *)pm->w1, (void *)pm->w2, (void *)pm->b1, (void *)pm->b2, (void *)pm->gamma,
+                    (void *)pm->beta, (void *)pm->err, (void *)pm->ln_rows, (void *)pm->hid})
+        if (p) cudaFree(p);
+    delete pm;
+}
+
+pe_status pe_merger_set_weights(pe_merger *pm, const void *gamma, const void *beta, const void *w1, const void *b1,
+                                const void *w2, const void *b2, pe_dtype dt, pe_stream_t stream) {
+    if (!pm || !gamma || !beta || !w1 || !w2) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(dt)) return PE_ERR_DTYPE;
+    for (const void *p : {gamma, beta, w1, w2, b1, b2})
+        if (p && !aligned16(p)) return PE_ERR_ALIGN;
+    DeviceGuard g(pm->core.dev);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t D = pm->D, H = pm->H;
+    auto to_bf16 = [&](const void *src, uint16_t *dst, int64_t n) -> bool {
+        if (dt == PE_BF16) return cudaMemcpyAsync(dst, src, sizeof(uint16_t) * n, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+        const int64_t n8 = n / 8;   // D % 64 == 0: whole 8-element groups
+        const int cb = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)pm->core.num_sms * 8);
+        pe_cast_rows_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(src), dst, n8);
+        return cudaGetLastError() == cudaSuccess;
+    };
+    auto to_f32 = [&](const void *src, float *dst, int64_t n) -> bool {
+        const int cb = (int)std::min<int64_t>((n + 255) / 256, 1024);
+        pe_to_f32_kernel<<<cb, 256, 0, st>>>(src, dt == PE_F32, dst, n);
+        return cudaGetLastError() == cudaSuccess;
+    };
+    if (!to_bf16(w1, pm->w1, D * D) || !to_bf16(w2, pm->w2, H * D) || !to_f32(gamma, pm->gamma, pm->E) ||
+        !to_f32(beta, pm->beta, pm->E))
+        return PE_ERR_CUDA;
+    pm->has_b1 = b1 != nullptr;
+    pm->has_b2 = b2 != nullptr;
+    if ((b1 && !to_f32(b1, pm->b1, D)) || (b2 && !to_f32(b2, pm->b2, H))) return PE_ERR_CUDA;
+    pm->weights_set = true;
+    return PE_OK;
+}
+
+pe_status pe_merger_forward(pe_merger *pm, const void *x, int64_t N, void *out, pe_dtype out_dt, pe_stream_t stream) {
+    if (!pm || N < 0) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(out_dt)) return PE_ERR_DTYPE;
+    if (!pm->weights_set) return PE_ERR_NO_WEIGHT;
+    if (N % pm->m2 != 0) return PE_ERR_SHAPE;
+    if (N == 0) return PE_OK;
+    if (!x || !out) return PE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return PE_ERR_ALIGN;
+    DeviceGuard g(pm->core.dev);
+    ProfScope ps(&pm->core);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t V = N / pm->m2;
+    if (!grow(&pm->ln_rows, &pm->ln_bytes, sizeof(uint16_t) * (size_t)N * pm->E, st) ||
+        !grow(&pm->hid, &pm->hid_bytes, sizeof(uint16_t) * (size_t)V * pm->D, st))
+        return PE_ERR_CUDA;
+    const int64_t blocks = (N + 7) / 8;
+    pe_layernorm_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint16_t *>(x), N, pm->E, pm->gamma,
+                                                         pm->beta, pm->eps, pm->ln_rows);
+    if (pm->core.prof_on) ++pm->core.prof_launches;
+    if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    pe_status s = merger_linear(pm, pm->ln_rows, V, pm->tmap_w1, pm->D, pm->has_b1 ? pm->b1 : nullptr, 1, pm->hid,
+                                PE_BF16, st);
+    if (s != PE_OK) return s;
+    return merger_linear(pm, pm->hid, V, pm->tmap_w2, pm->H, pm->has_b2 ? pm->b2 : nullptr, 0, out, out_dt, st);
+}
+
+pe_status pe_merger_profile_begin(pe_merger *pm, int max_calls) {
+    if (!pm) return PE_ERR_INVALID_ARG;
+    return pe_profile_begin(&pm->core, max_calls);
+}
+
+pe_status pe_merger_profile_end(pe_merger *pm, float *ms, int *n, int64_t *launches) {
+    if (!pm) return PE_ERR_INVALID_ARG;
+    return pe_profile_end(&pm->core, ms, n, launches);
+}
+
+pe_status pe_merger_last_error(pe_merger *pm) {
+    if (!pm) return PE_ERR_INVALID_ARG;
+    DeviceGuard g(pm->core.dev);
+    int v = 0;
+    if (cudaMemcpy(&v, pm->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PE_ERR_CUDA;
+    if (v != 0 && cudaMemset(pm->err, 0, sizeof(int)) != cudaSuccess) return PE_ERR_CUDA;
+    return v == 0 ? PE_OK : (pe_status)v;
+}
+
 }  // extern "C"

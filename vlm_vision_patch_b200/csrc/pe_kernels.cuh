@@ -100,6 +100,7 @@ struct FwdParams {
     const float *bias;                // fp32 [E] or nullptr
     const void *pos;                  // [N, E] added in the epilogue, or nullptr
     int32_t pos_f32;                  // pos dtype is fp32 (else bf16)
+    int32_t act;                      // epilogue activation after bias: 0 none, 1 exact GELU
     int *err;                         // device error word
     // kAModeTmaStream
     uint16_t *a_rows;                 // [N, row_elems] rows written by the producers
@@ -1125,6 +1126,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 if (nbufs == 4) bulk_wait_read<3>(); else bulk_wait_read<1>();
             }
             __syncwarp();
+            if (P.act) {   // exact GELU, 0.5 x (1 + erf(x / sqrt 2)), in fp32
+#pragma unroll
+                for (int e = 0; e < 32; ++e) f[e] = 0.5f * f[e] * (1.0f + erff(f[e] * 0.70710678118654752f));
+            }
             if constexpr (has_pos) {   // out = acc + bias + pos, in fp32, before the output cast
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -1410,6 +1415,63 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
         bulk_commit();
         bulk_wait<0>();
     }
+}
+
+// LayerNorm of bf16 rows [N, E] (E % 8 == 0) into bf16 rows: one warp per row,
+// fp32 statistics over the E features (mean, then the biased variance of the
+// deviations), y = (x - mean) * rsqrt(var + eps) * gamma + beta, rounded to
+// bf16.  The PatchMerger's first step (mytransformer README §3.2, §4.1).
+__global__ void pe_layernorm_kernel(const uint16_t *__restrict__ x, int64_t N, int E, const float *__restrict__ gamma,
+                                    const float *__restrict__ beta, float eps, uint16_t *__restrict__ y) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= N) return;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * E);
+    const int nv = E / 8;
+    float s = 0.f;
+    for (int i = lane; i < nv; i += 32) {
+        const uint4 v = __ldg(xr + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s += bf16lo_to_f32(w[u]) + bf16hi_to_f32(w[u]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / (float)E;
+    float q = 0.f;
+    for (int i = lane; i < nv; i += 32) {
+        const uint4 v = __ldg(xr + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float d0 = bf16lo_to_f32(w[u]) - mean, d1 = bf16hi_to_f32(w[u]) - mean;
+            q += d0 * d0 + d1 * d1;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float inv = rsqrtf(q / (float)E + eps);
+    uint4 *yr = reinterpret_cast<uint4 *>(y + row * E);
+    for (int i = lane; i < nv; i += 32) {
+        const uint4 v = __ldg(xr + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = 8 * i + 2 * u;
+            const float a = (bf16lo_to_f32(w[u]) - mean) * inv * __ldg(gamma + e) + __ldg(beta + e);
+            const float b = (bf16hi_to_f32(w[u]) - mean) * inv * __ldg(gamma + e + 1) + __ldg(beta + e + 1);
+            o4[u] = pack_bf16x2(a, b);
+        }
+        yr[i] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+}
+
+// bf16 or fp32 values -> fp32 (exact).
+__global__ void pe_to_f32_kernel(const void *src, int src_f32, float *dst, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = src_f32 ? reinterpret_cast<const float *>(src)[i]
+                         : __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(src)[i] << 16);
 }
 
 // fp32 patch rows -> tf32-rounded fp32 rows (nearest, ties away from zero)
