@@ -64,8 +64,8 @@ def load_peaks():
 # the figure (reported as null) until it is captured again.
 TRAFFIC = {
     # profiles/pe_fwd_kernel_grouped_16_images.md, profiles/pe_fwd_kernel_long_video_64x896.md
-    ("grouped_16_images", "staged"): {"bytes": 115302656 + 97552896, "kernel_sha": "35f1cefad9cf5a2a"},
-    ("long_video_64x896", "staged"): {"bytes": 507656192 + 281458176, "kernel_sha": "35f1cefad9cf5a2a"},
+    ("grouped_16_images", "staged"): {"bytes": 97596160 + 98053888, "kernel_sha": "aff60e535f2c6447"},
+    ("long_video_64x896", "staged"): {"bytes": 425094656 + 282965760, "kernel_sha": "aff60e535f2c6447"},
 }
 KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh")
 
