@@ -1,26 +1,35 @@
-// sm_100a kernels of the vision PatchEmbed.
+// sm_100a kernels of the vision PatchEmbed (and of the PatchMerger that
+// consumes its rows).
 //
 // The PatchEmbed is a Conv3d whose kernel equals its stride, i.e. one dense
 // contraction out[N, E] = A[N, K] * W[E, K]^T (+ bias) with K = C*tp*p*p
 // (Qwen2.5VL-Vision Encode-PatchEmbed: the conv is a dot product of the
 // flattened input and weight; mytransformer README §4.1: F.linear(x,
-// w.reshape(1280, 1176))).  One persistent kernel runs the whole path on CTA
-// pairs (thread-block clusters of 2) that share each 256 x BN output tile
-// through the pair form of the 5th-generation MMA (tcgen05 cta_group::2):
-// every CTA stages its own 128 rows of A and BN/2 rows of the weight, the
-// leader CTA issues the MMAs, and each CTA accumulates its 128 rows x BN fp32
-// in its own tensor memory.
+// w.reshape(1280, 1176))).  One persistent kernel, pe_fwd_kernel, runs the
+// contraction on CTA pairs (thread-block clusters of 2) that share each
+// 256 x BN output tile through the pair form of the 5th-generation MMA
+// (tcgen05 cta_group::2): every CTA stages its own 128 rows of A and BN/2 rows
+// of the weight, the leader CTA issues the MMAs, and each CTA accumulates its
+// 128 rows x BN fp32 in its own tensor memory.
 //
-//   warp 0      TMA producer: weight tiles (and A tiles of bf16 patch rows)
+//   warps 0, 2, 3 (+ 8, 9 when A is TMA-fed; + 16, 17 in the streamed mode)
+//               TMA issuers: weight tiles, and A tiles in the TMA-fed modes
 //   warp 1      TMEM owner; in the leader CTA one thread issues the MMAs
-//   warps 4-7   epilogue: TMEM -> registers, + bias, cast, TMA stores
-//   warps 8-15  A producers for the thread-fed modes: fp32 / unaligned patch
+//   warps 4-7   epilogue: TMEM -> registers, + bias (+ position table, GELU),
+//               cast, TMA stores
+//   warps 8-19  A producers of the thread-fed modes: fp32 / unaligned patch
 //               rows converted to bf16, or the fused frames gather that builds
 //               each patch row from raw [T, C, H, W] frames, normalises it and
-//               places it in merge order, straight into shared memory.
+//               places it in merge order, straight into shared memory
+//               (warps 8-15 write rows to global memory in the streamed mode).
 //
-// The accumulator is double buffered (2 x 256 TMEM columns) so the epilogue of
-// one tile overlaps the MMAs of the next.  Every pipeline wait is bounded.
+// The A modes (AMode below) select how A reaches shared memory.  The
+// accumulator is double buffered (2 x 256 TMEM columns) so the epilogue of one
+// tile overlaps the MMAs of the next.  Every pipeline wait is bounded.
+//
+// Around it: the staged prepare kernel (pe_prep_rows_kernel), the fp32 casts
+// (pe_cast_rows_kernel, pe_round_tf32_kernel), the weight packers, the
+// patchify test hook and the PatchMerger's LayerNorm (pe_layernorm_kernel).
 #pragma once
 
 #include <type_traits>
@@ -650,22 +659,22 @@ __device__ __forceinline__ void produce_patches(const FwdParams &P, const ProdCt
 
 // ------------------------------------------------------------- MMA issue
 
-// The single MMA-issuing thread must keep pace with the tensor core (one pair
-// MMA of 256 x 256 x 16 every 128 cycles), so the loop is unrolled over a
-// super-stage of lcm(KSA, 4) k-steps: waits, commits and descriptor offsets
-// sit at compile-time positions, descriptors advance by constant adds, and
-// nothing divides.  A stages hold KSA k-steps, weight stages 4.
+// Issue loop of the thread-fed modes (A written into shared memory by
+// producer warps, no-swizzle K-major layout, own full barriers).  The single
+// MMA-issuing thread must keep pace with the tensor core (one pair MMA of
+// 256 x 256 x 16 every 128 cycles), so the loop is unrolled over a super-stage
+// of lcm(KSA, 4) k-steps: waits, commits and descriptor offsets sit at
+// compile-time positions, descriptors advance by constant adds, and nothing
+// divides.  A stages hold KSA k-steps, weight stages 4.
 //   SEP_A_COMMIT  A stages have their own empty barriers (frames path);
 //                 otherwise A and weight stages coincide and share one.
-//   SEP_A_WAIT    A stages have their own full barriers (thread-produced A);
-//                 otherwise the A TMA bytes land on the weight stage's barrier.
 __host__ __device__ constexpr int lcm4(int a) { return (a % 4 == 0) ? a : (a % 2 == 0 ? 2 * a : 4 * a); }
 
 __device__ __forceinline__ uint64_t desc_with_lo(uint64_t d, uint32_t lo) {
     return (d & 0xFFFFFFFF00000000ull) | lo;
 }
 
-template <int KSA, bool SEP_A_COMMIT, bool SEP_A_WAIT>
+template <int KSA, bool SEP_A_COMMIT>
 __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, uint8_t *b_ring, uint64_t *full_a,
                                           uint64_t *empty_a, uint64_t *full_b, uint64_t *empty_b, uint64_t *tfull,
                                           uint64_t *tempty, uint64_t *mma_done, uint32_t tmem_base,
@@ -674,13 +683,12 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
     constexpr int L = lcm4(KSA);
     constexpr uint16_t kPair = 0x3;
     const uint32_t idesc = idesc_bf16_f32(2 * kBM, P.bn);
-    // Descriptor templates (address field of slot 0); a k-step inside a stage
-    // adds 32 bytes (128-byte swizzle) or 4096 bytes (no-swizzle, 2 core-matrix columns).
-    const uint64_t a0 = (SEP_A_COMMIT) ? smem_desc(smem_addr(a_ring), 2048, 128, kLayoutInterleave)
-                        : (SEP_A_WAIT) ? smem_desc(smem_addr(a_ring), 2048, 128, kLayoutInterleave)
-                                       : smem_desc(smem_addr(a_ring), 16, 1024, kLayoutSw128);
+    // Descriptor templates (address field of slot 0); an A k-step adds 4096
+    // bytes (no-swizzle, 2 core-matrix columns), a weight k-step 32 bytes
+    // (128-byte swizzle).
+    const uint64_t a0 = smem_desc(smem_addr(a_ring), 2048, 128, kLayoutInterleave);
     const uint64_t b0 = smem_desc(smem_addr(b_ring), 16, 1024, kLayoutSw128);
-    constexpr uint32_t kAStep = (SEP_A_WAIT) ? (4096u >> 4) : (32u >> 4);
+    constexpr uint32_t kAStep = 4096u >> 4;
     const uint32_t a_slot_step = (uint32_t)P.a_stage_bytes >> 4;
     constexpr uint32_t kBSlotStep = (uint32_t)kBStageBytes >> 4;
     const uint32_t a_lo0 = (uint32_t)a0, b_lo0 = (uint32_t)b0;
@@ -701,9 +709,8 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
                     if (j % KSB == 0) {
                         if (!mbar_wait(smem_addr(&full_b[bs]), bph, abort)) return;
                         b_lo = b_lo0 + (uint32_t)bs * kBSlotStep;
-                        if (!SEP_A_WAIT) a_lo = a_lo0 + (uint32_t)bs * a_slot_step;
                     }
-                    if (SEP_A_WAIT && j % KSA == 0) {
+                    if (j % KSA == 0) {
                         if (!mbar_wait(smem_addr(&full_a[as]), aph, abort)) return;
                         a_lo = a_lo0 + (uint32_t)(SEP_A_COMMIT ? as : bs) * a_slot_step;
                     }
@@ -719,7 +726,7 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
                         mma_commit_pair(smem_addr(&empty_a[as]), kPair);
                         if (++as == P.na) { as = 0; aph ^= 1; }
                     }
-                    if (SEP_A_WAIT && !SEP_A_COMMIT && (j % KSA == KSA - 1 || last)) {
+                    if (!SEP_A_COMMIT && (j % KSA == KSA - 1 || last)) {
                         if (++as == P.na) { as = 0; aph ^= 1; }
                     }
                 }
@@ -1071,7 +1078,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     mma_issue_tma<kSl, 1>(P, a_ring, b_ring, full_b, empty_b, tfull, tempty, mma_done, tmem_base, abort);
             }
             else if constexpr (KSA > 0)
-                mma_issue<KSA, AMODE == kAModeFrames, AMODE != kAModeTma>(P, a_ring, b_ring, full_a, empty_a, full_b,
+                mma_issue<KSA, AMODE == kAModeFrames>(P, a_ring, b_ring, full_a, empty_a, full_b,
                                                                           empty_b, tfull, tempty, mma_done, tmem_base,
                                                                           abort);
             else
