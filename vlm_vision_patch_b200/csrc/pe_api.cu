@@ -396,19 +396,17 @@ bool staged_eligible(const pe_handle *h, int f_dt) {
 }
 
 // bf16 frames with tp = 2 and p in {14, 16}: 0 = fused kernel, 1 = staged
-// pair (the default), 2 = streamed kernel.  PE_FRAMES_PATH=fused|staged|streamed
-// overrides.  The
+// pair (the default), 2 = streamed kernel; PE_FRAMES_PATH=fused|staged|streamed
+// overrides.  Every other frames call takes the fused kernel.  The
 // streamed kernel overlaps row production with the contraction but its
 // producer warps' scattered loads and stores slow the contraction down more
 // than the separate prepare kernel costs (measured on B200), so it is not the
 // default.
-int large_path(const pe_handle *h, const FwdParams &P, int f_dt) {
+int frames_path(const pe_handle *h, int f_dt) {
     if (!staged_eligible(h, f_dt)) return 0;
     const char *e = std::getenv("PE_FRAMES_PATH");
     if (e && std::strcmp(e, "fused") == 0) return 0;
-    if (e && std::strcmp(e, "staged") == 0) return 1;
     if (e && std::strcmp(e, "streamed") == 0) return 2;
-    (void)P;
     return 1;
 }
 
@@ -553,7 +551,7 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
         return run_frames_staged(h, P, out, all_scaled, true, st, true);
     }
-    const int lp = allow_staged ? large_path(h, P, f_dt) : 0;
+    const int lp = allow_staged ? frames_path(h, f_dt) : 0;
     if (lp != 0) {
         bool all_scaled = true;
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
