@@ -64,8 +64,8 @@ def load_peaks():
 # the figure (reported as null) until it is captured again.
 TRAFFIC = {
     # profiles/pe_fwd_kernel_grouped_16_images.md, profiles/pe_fwd_kernel_long_video_64x896.md
-    ("grouped_16_images", "staged"): {"bytes": 97596160 + 98053888, "kernel_sha": "6ac25972a2d12b41"},
-    ("long_video_64x896", "staged"): {"bytes": 425094656 + 282965760, "kernel_sha": "6ac25972a2d12b41"},
+    ("grouped_16_images", "staged"): {"bytes": 94770944 + 97856256, "kernel_sha": "2d0b9a5fb46fd12c"},
+    ("long_video_64x896", "staged"): {"bytes": 381790464 + 282007296, "kernel_sha": "2d0b9a5fb46fd12c"},
 }
 KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh")
 
