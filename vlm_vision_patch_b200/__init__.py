@@ -46,7 +46,7 @@ def num_patches(grid_thw: Sequence[Sequence[int]]) -> int:
 
 
 class PatchEmbed:
-    """Conv3d(C, E, kernel=stride=(tp, p, p)) as one fused sm_100a kernel."""
+    """Conv3d(C, E, kernel=stride=(tp, p, p)) on sm_100a kernels (C ABI in include/pe.h)."""
 
     def __init__(self, E: int, C: int = 3, tp: int = 2, p: int = 14, bias: bool = False):
         self.E, self.C, self.tp, self.p, self.has_bias = E, C, tp, p, bias
