@@ -670,3 +670,54 @@ def test_patch_merger_errors():
         pm.forward(torch.zeros(6, 64, dtype=torch.bfloat16, device=DEV))   # 6 rows: not whole 2x2 windows
     assert e.value.status == "PE_ERR_SHAPE"
     pm.close()
+
+
+# ------------------------------------------------------ more path/shape cases
+
+@pytest.mark.parametrize("case", ["staged_E200_bias_f32", "staged_merge1_odd_gw_p16", "fold_with_pos",
+                                  "tf32_with_pos"])
+def test_more_path_combinations(case, monkeypatch):
+    """Combinations of options and ragged shapes on the default paths, each
+    against the oracle at the parity tolerance (the folded case at the folding
+    bound, the tf32 case against the unrounded oracle at the tf32 bound)."""
+    C, tp = 3, 2
+    if case.startswith("tf32"):
+        p, E, N = 14, 256, 200
+        K = C * tp * p * p
+        x = workloads.normal((N, K), 700)
+        w = workloads.normal((E, C, tp, p, p), 701, std=0.03)
+        pos = workloads.normal((N, E), 702, std=0.5)
+        pe = _pe((E, C, tp, p), w, None)
+        pe.set_tf32(True)
+        out = pe.forward_patches(x.to(DEV), out_dtype=torch.float32, pos=pos.to(DEV))
+        torch.cuda.synchronize()
+        ref, mag = oracle.conv3d_patches_fp32(x, w, None, C, tp, p)
+        pv = pos.double().numpy()
+        assert_within_tolerance(out, ref + pv, mag + np.abs(pv), what=case, rel=2.0 ** -10 + 2.0 ** -13)
+        return
+    if case == "staged_E200_bias_f32":
+        p, E, merge, grids, Ts, od = 14, 200, 2, [(2, 6, 8), (1, 4, 10)], [3, 1], torch.float32
+    elif case == "staged_merge1_odd_gw_p16":
+        p, E, merge, grids, Ts, od = 16, 384, 1, [(1, 5, 7), (2, 3, 9)], [1, 4], torch.bfloat16
+    else:
+        p, E, merge, grids, Ts, od = 14, 512, 2, [(1, 8, 12), (1, 6, 6)], [1, 1], torch.bfloat16
+    items = [(workloads.uniform01((T, C, g[1] * p, g[2] * p), 710 + i), g) for i, (T, g) in enumerate(zip(Ts, grids))]
+    w = workloads.normal((E, C, tp, p, p), 720, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 721, std=0.02, dtype=torch.bfloat16)
+    pe = _pe((E, C, tp, p), w, b, workloads.CLIP_MEAN, workloads.CLIP_STD)
+    N = sum(g[0] * g[1] * g[2] for g in grids)
+    pos = None
+    if case == "fold_with_pos":
+        pe.set_temporal_fold(True)
+        pos = workloads.normal((N, E), 722, std=0.5, dtype=torch.bfloat16)
+    out = pe.forward_frames_grouped([f.to(DEV) for f, _ in items], grids, merge, out_dtype=od,
+                                    pos=None if pos is None else pos.to(DEV))
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    ref, mag = oracle.conv3d_grouped(items, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
+    rel = 1e-3
+    if pos is not None:
+        pv = pos.double().numpy()
+        ref, mag = ref + pv, mag + np.abs(pv)
+        rel = 2.0 ** -8 + 1e-3
+    assert_within_tolerance(out, ref, mag, what=case, rel=rel)

@@ -398,3 +398,25 @@ def test_patch_merger_concatenates_the_window_rows_in_order():
             y = 64.0 * float(_bf16(ln[v * m2 + q, e].float()))
             gl = 0.5 * y * (1.0 + math.erf(y / math.sqrt(2.0)))
             assert out[v, 0] == float(torch.tensor(gl, dtype=torch.float32).to(torch.bfloat16).double())
+
+
+def test_frames_form_is_translation_invariant():
+    """Patches that an image and its crop share (the crop drops the first patch
+    column and the first patch row) must embed identically: the frames form
+    locates every patch at (g_h * p, g_w * p) of its own image.  Raster order
+    (merge 1) so that the shared rows are easy to pair up."""
+    C, tp, p, E = 3, 2, 4, 6
+    T, gh, gw = 3, 4, 5
+    img = workloads.normal((T, C, gh * p, gw * p), 420)
+    crop = img[:, :, p:, p:].contiguous()
+    w = workloads.normal((E, C, tp, p, p), 421, std=0.3)
+    gt = -(-T // tp)
+    full, _ = oracle.conv3d_frames(img, (gt, gh, gw), 1, (0.1, 0.2, 0.3), (0.5, 0.7, 0.9), w, None, C, tp, p)
+    part, _ = oracle.conv3d_frames(crop, (gt, gh - 1, gw - 1), 1, (0.1, 0.2, 0.3), (0.5, 0.7, 0.9), w, None,
+                                   C, tp, p)
+    for t in range(gt):
+        for y in range(gh - 1):
+            for x in range(gw - 1):
+                a = full[(t * gh + (y + 1)) * gw + (x + 1)]
+                b = part[(t * (gh - 1) + y) * (gw - 1) + x]
+                assert np.array_equal(a, b), (t, y, x)
