@@ -136,23 +136,18 @@ int bn_override() {
     return (v == 64 || v == 128 || v == 256) ? v : 0;
 }
 
-// Tile width: frames tiles pay the gather once per tile whatever BN is, so use
-// the widest BN unless the problem is too small to fill the GPU in one wave;
-// TMA-fed patch tiles are cheap to refill, so prefer enough tiles for all SMs.
-int choose_bn(int64_t N, int E, int num_pairs, bool gather_fed) {
+// Tile width: the widest BN (256: the pair MMA at full rate) unless the problem
+// is too small to fill the GPU in one wave at 256; then every pair runs at most
+// one tile, so the narrowest BN that still fits one wave finishes first (a
+// second round of narrow tiles costs more than the narrow MMAs save).
+int choose_bn(int64_t N, int E, int num_pairs) {
     if (const int o = bn_override()) return o;
     const int64_t mt = (N + 2 * kBM - 1) / (2 * kBM);
     auto tiles = [&](int bn) { return mt * ((E + bn - 1) / bn); };
     if (tiles(256) >= num_pairs) return 256;
-    if (gather_fed) {
-        // Less than one wave even at BN=256: every pair runs one tile, so the
-        // narrowest BN that still fits one wave finishes first.
-        if (tiles(64) <= num_pairs) return 64;
-        if (tiles(128) <= num_pairs) return 128;
-        return 256;
-    }
-    if (tiles(128) >= num_pairs) return 128;
-    return 64;
+    if (tiles(64) <= num_pairs) return 64;
+    if (tiles(128) <= num_pairs) return 128;
+    return 256;
 }
 
 thread_local pe_handle *t_prof_handle = nullptr;   // handle of the call being launched
@@ -214,9 +209,9 @@ struct ProfScope {   // makes the handle's profiling events visible to launch_fw
 int bn_index(int bn) { return bn == 64 ? 0 : (bn == 128 ? 1 : 2); }
 
 // Pair tiles, grid (two CTAs per pair, at most one pair per two SMs).
-void plan_tiles(const pe_handle *h, FwdParams &P, int64_t N, bool gather_fed, int &grid, bool &ok) {
+void plan_tiles(const pe_handle *h, FwdParams &P, int64_t N, int &grid, bool &ok) {
     const int num_pairs = h->num_sms / 2;
-    P.bn = choose_bn(N, P.E, num_pairs, gather_fed);
+    P.bn = choose_bn(N, P.E, num_pairs);
     P.n_tiles_n = (P.E + P.bn - 1) / P.bn;
     const int64_t mt = (N + 2 * kBM - 1) / (2 * kBM);
     ok = mt * P.n_tiles_n <= INT32_MAX;
@@ -456,7 +451,7 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     G.x_vec = 1;
     int grid = 0;
     bool ok = true;
-    plan_tiles(h, G, G.N, false, grid, ok);
+    plan_tiles(h, G, G.N, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
     const int amode = (shared && !fold) ? kAModeTmaShared : kAModeTma;
     const size_t smem = plan_pipeline(h, G, amode, row_elems);
@@ -516,7 +511,7 @@ pe_status run_frames_streamed(pe_handle *h, FwdParams &P, void *out, bool all_sc
     G.n_mblocks = (int)mt;
     int grid = 0;
     bool ok = true;
-    plan_tiles(h, G, G.N, false, grid, ok);
+    plan_tiles(h, G, G.N, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
     G.ready_target = (uint32_t)(kStreamProdWarps * 2 * G.n_tiles_n);
     // single-frame rows: one slice against both weight slices; otherwise both
@@ -561,7 +556,7 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
     }
     int grid = 0;
     bool ok = true;
-    plan_tiles(h, P, P.N, true, grid, ok);
+    plan_tiles(h, P, P.N, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
     const size_t smem = plan_pipeline(h, P, kAModeFrames);
     CUtensorMap dummy, to;
@@ -809,7 +804,7 @@ pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
         }
         int grid = 0;
         bool ok = true;
-        plan_tiles(h, P, N, false, grid, ok);
+        plan_tiles(h, P, N, grid, ok);
         if (!ok) return PE_ERR_UNSUPPORTED;
         const size_t smem = plan_pipeline(h, P, kAModeTmaTf32);
         CUtensorMap tx, to;
@@ -846,7 +841,7 @@ pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
         }
         int grid = 0;
         bool ok = true;
-        plan_tiles(h, P, N, false, grid, ok);
+        plan_tiles(h, P, N, grid, ok);
         if (!ok) return PE_ERR_UNSUPPORTED;
         const size_t smem = plan_pipeline(h, P, kAModeTma);
         CUtensorMap tx, to;
@@ -865,7 +860,7 @@ pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
     }
     int grid = 0;
     bool ok = true;
-    plan_tiles(h, P, N, !tma, grid, ok);
+    plan_tiles(h, P, N, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
     const size_t smem = plan_pipeline(h, P, tma ? kAModeTma : kAModePatchThreads);
     cudaStream_t st = (cudaStream_t)stream;
@@ -1147,7 +1142,7 @@ pe_status merger_linear(pe_merger *pm, const uint16_t *A, int64_t V, const CUten
     G.err = pm->err;
     int grid = 0;
     bool ok = true;
-    plan_tiles(&pm->core, G, V, false, grid, ok);
+    plan_tiles(&pm->core, G, V, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
     const size_t smem = plan_pipeline(&pm->core, G, kAModeTma, pm->D);
     CUtensorMap tx, to;
