@@ -24,17 +24,20 @@
  *     every input and output buffer; the library owns only what a handle holds
  *     (packed weight, fp32 bias, normalisation constants, tensor-map
  *     descriptors, a small device workspace and a device error word).
- *   - Calls that take a stream are asynchronous on that stream and never
- *     synchronise it.  Argument and shape errors are detected on the host and
- *     returned before anything is launched or written.
+ *   - Calls that take a stream are asynchronous on that stream.  They do not
+ *     synchronise it, except when a grow-only workspace has to be enlarged
+ *     (the old buffer is freed only after the stream drains).  Argument and
+ *     shape errors are detected on the host and returned before anything is
+ *     launched or written.
  *   - Dense row-major layouts only.  Device pointers must be 16-byte aligned.
  *   - No C++ exception crosses this interface.  A CUDA error maps to
  *     PE_ERR_CUDA.
  *   - Forward calls that use a handle's workspace must be serialised on one
  *     stream: grouped calls with more than PE_INLINE_ITEMS items (item table),
- *     and frames calls large enough to take the staged path (see
- *     pe_forward_frames).  pe_set_weight / pe_set_norm must not run
- *     concurrently with anything else on the same handle.
+ *     frames calls on the staged or streamed path (see pe_forward_frames), and
+ *     pe_forward_patches on fp32 rows.  pe_set_weight, pe_set_norm,
+ *     pe_set_temporal_fold and pe_set_tf32 must not run concurrently with
+ *     anything else on the same handle.
  */
 #ifndef PE_H_
 #define PE_H_
@@ -175,7 +178,7 @@ pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int
                                  pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream);
 
 /*
- * pe_forward_frames -- fused patchify + normalise + embed of one image/video.
+ * pe_forward_frames -- patchify + normalise + embed of one image/video.
  *   frames   : dev [T, C, H, W] of dtype f_dt (PE_BF16 or PE_F32), dense.
  *   grid_thw : host [3] = (gt, gh, gw) in patch units.  Requires H == gh*p,
  *              W == gw*p and ceil(T / tp) == gt (patch详解 §4.5).  When T is not
@@ -286,15 +289,16 @@ int64_t pe_num_patches(const int32_t *grid_thw, int n);
 
 /*
  * pe_profile_begin / pe_profile_end -- device time of each forward call's
- * contraction kernel (the fused kernel, or the GEMM of the staged path),
- * recorded with a CUDA event pair on the call's stream around that launch.
- * pe_profile_begin creates event pairs for up to max_calls calls (0..1e6; 0
- * records no events and only counts launches) and starts recording; pe_profile_end waits for the recorded events, writes the
+ * contraction kernel (the fused kernel, or the GEMM that follows the prepare
+ * or cast kernel), recorded with a CUDA event pair on the call's stream
+ * around that launch.  pe_profile_begin creates event pairs for up to
+ * max_calls calls (0..1e6; 0 records no events and only counts launches) and
+ * starts recording; pe_profile_end waits for the recorded events, writes the
  * elapsed milliseconds of the first min(*n, recorded) calls to host ms[] and
  * that count to *n, writes to *launches (if not NULL) how many kernels the
- * forward calls launched in the window (the staged frames path launches two
- * per call, every other forward one), then frees the events and stops
- * recording.  Profiling is a measurement aid: it allocates events and must not
+ * forward calls launched in the window (two per call on the staged frames
+ * path and for fp32 patch rows, one otherwise), then frees the events and
+ * stops recording.  Profiling is a measurement aid: it allocates events and must not
  * overlap another profiling window on the same handle.  An event recorded
  * between two kernels of one call serialises them, so a window with events
  * runs the staged path a few microseconds slower than a window without.
