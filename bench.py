@@ -66,6 +66,8 @@ TRAFFIC = {
     # profiles/pe_fwd_kernel_grouped_16_images.md, profiles/pe_fwd_kernel_long_video_64x896.md
     ("grouped_16_images", "staged"): {"bytes": 94770944 + 97856256, "kernel_sha": "2d0b9a5fb46fd12c"},
     ("long_video_64x896", "staged"): {"bytes": 381790464 + 282007296, "kernel_sha": "2d0b9a5fb46fd12c"},
+    # profiles/pe_fwd_kernel_merger_fc1_grouped_16_images.md (the PatchMerger's fc1 + GELU)
+    ("patch_merger_grouped_16_images", "fc1"): {"bytes": 614624768 + 134967040, "kernel_sha": "2d0b9a5fb46fd12c"},
 }
 KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh")
 
@@ -524,7 +526,8 @@ def run_merger(args, rank, world, local):
             "tflops": flop / (mean_ms / 1e3) / 1e12,
             "kernel_ms": {"fc1_mean": fc1_ms, "fc2_mean": statistics.mean(lin[1::2]) if len(lin) > 1 else None},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "pe_fwd_kernel (merger fc1 + GELU)",
+                         "frac": achieved / peak, "traffic": measured_traffic("patch_merger_" + wl.name, "fc1"),
+                         "kernel": "pe_fwd_kernel (merger fc1 + GELU)",
                          "peak_source": f"{src} bf16 dense (burst)"},
             "cpu_baseline": None,
             "e2e": None, "gpu_launches": launches, "clocks": clk.summary()}), flush=True)
