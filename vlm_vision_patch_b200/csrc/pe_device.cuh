@@ -271,6 +271,17 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
         : "memory");
 }
 
+// Commit every pair MMA issued so far to `bar` (leader CTA only) and wait for
+// it, bounded by time alone: after an abort the MMAs already in flight must
+// still finish before the TMEM they write is freed.
+__device__ __forceinline__ void mma_drain(uint32_t bar) {
+    mma_commit_pair(bar, 0x1);
+    if (mbar_try_wait(bar, 0)) return;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, 0))
+        if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
+}
+
 // 32 lanes x 32 consecutive fp32 columns: thread t of the warp gets lane
 // (base lane + t), columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {

@@ -735,8 +735,6 @@ __device__ __forceinline__ void mma_issue(const FwdParams &P, uint8_t *a_ring, u
         mma_commit_pair(smem_addr(&tfull[acc]), kPair);
         if (++acc == 2) { acc = 0; accph ^= 1; }
     }
-    mma_commit_pair(smem_addr(mma_done), 0x1);
-    mbar_wait(smem_addr(mma_done), 0, abort);
 }
 
 // Streamed frames producer (kAModeTmaStream), warps 8..15 of every CTA.
@@ -897,8 +895,6 @@ __device__ __forceinline__ void mma_issue_tma(const FwdParams &P, uint8_t *a_rin
         mma_commit_pair(smem_addr(&tfull[acc]), kPair);
         if (++acc == 2) { acc = 0; accph ^= 1; }
     }
-    mma_commit_pair(smem_addr(mma_done), 0x1);
-    mbar_wait(smem_addr(mma_done), 0, abort);
 }
 
 // Runtime-p frames path (p not 14 or 16): the same protocol, not unrolled.
@@ -940,8 +936,6 @@ __device__ __noinline__ void mma_issue_generic(const FwdParams &P, uint8_t *a_ri
         mma_commit_pair(smem_addr(&tfull[acc]), kPair);
         if (++acc == 2) { acc = 0; accph ^= 1; }
     }
-    mma_commit_pair(smem_addr(mma_done), 0x1);
-    mbar_wait(smem_addr(mma_done), 0, abort);
 }
 
 // ------------------------------------------------------------- the kernel
@@ -1084,6 +1078,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             else
                 mma_issue_generic(P, a_ring, b_ring, full_a, empty_a, full_b, empty_b, tfull, tempty, mma_done,
                                   tmem_base, abort);
+            // Every MMA issued so far completes before the pair frees its TMEM, also
+            // when an issue loop returned early because a wait gave up.
+            mma_drain(smem_addr(mma_done));
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         // ---------------- epilogue (both CTAs)
@@ -1097,8 +1094,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         const int nch = P.bn / 32;   // 2, 4 or 8
         int acc = 0, nbuf = 0;
         uint32_t accph = 0;
-        auto emit = [&](auto kPos, const uint32_t (&v)[32], int cc, int64_t row0, int n_blk) {
+        auto emit = [&](auto kPos, auto kAct, const uint32_t (&v)[32], int cc, int64_t row0, int n_blk) {
             constexpr bool has_pos = decltype(kPos)::value;
+            constexpr bool has_act = decltype(kAct)::value;
             const int col0 = n_blk * P.bn + cc * 32;
             if (row0 >= P.N || col0 >= P.E) return;   // whole box outside: nothing to store
             // position-embedding row segment of this lane's row (E % 8 == 0, so a
@@ -1133,7 +1131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 if (nbufs == 4) bulk_wait_read<3>(); else bulk_wait_read<1>();
             }
             __syncwarp();
-            if (P.act) {   // exact GELU, 0.5 x (1 + erf(x / sqrt 2)), in fp32
+            if constexpr (has_act) {   // exact GELU, 0.5 x (1 + erf(x / sqrt 2)), in fp32
 #pragma unroll
                 for (int e = 0; e < 32; ++e) f[e] = 0.5f * f[e] * (1.0f + erff(f[e] * 0.70710678118654752f));
             }
@@ -1176,8 +1174,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
             }
             if (++nbuf == nbufs) nbuf = 0;
         };
-        // the tile loop, compiled with and without the position-embedding add
-        auto tiles = [&](auto kPos) {
+        // the tile loop, compiled without options, with the position-embedding
+        // add, and with the GELU (the PatchMerger's fc1)
+        auto tiles = [&](auto kPos, auto kAct) {
             for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
                 const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
                 if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
@@ -1191,17 +1190,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     for (int cc = 0; cc < nch; cc += 2) {
                         tmem_ld_wait();
                         tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 1) * 32, vb);
-                        emit(kPos, va, cc, row0, n_blk);
+                        emit(kPos, kAct, va, cc, row0, n_blk);
                         tmem_ld_wait();
                         if (cc + 2 < nch) tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 2) * 32, va);
-                        emit(kPos, vb, cc + 1, row0, n_blk);
+                        emit(kPos, kAct, vb, cc + 1, row0, n_blk);
                     }
                 } else {
                     uint32_t va[32];
                     for (int cc = 0; cc < nch; ++cc) {
                         tmem_ld_32x32b_x32(tbase + (uint32_t)cc * 32, va);
                         tmem_ld_wait();
-                        emit(kPos, va, cc, row0, n_blk);
+                        emit(kPos, kAct, va, cc, row0, n_blk);
                     }
                 }
                 tc_fence_before();
@@ -1210,8 +1209,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 if (++acc == 2) { acc = 0; accph ^= 1; }
             }
         };
-        if (P.pos) tiles(std::true_type{});
-        else tiles(std::false_type{});
+        if (P.pos) tiles(std::true_type{}, std::false_type{});
+        else if (P.act) tiles(std::false_type{}, std::true_type{});
+        else tiles(std::false_type{}, std::false_type{});
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
     } else if (AMODE == kAModeTmaStream && warp >= kStreamProdWarp0 && warp < kStreamProdWarp0 + kStreamProdWarps) {
