@@ -282,8 +282,8 @@ pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f
 
 /*
  * pe_num_patches -- sum_i gt_i * gh_i * gw_i over host grid_thw [n, 3];
- * 0 for n == 0; -1 on a NULL pointer with n > 0, negative n or a
- * non-positive entry.
+ * 0 for n == 0; -1 on a NULL pointer with n > 0, negative n, a
+ * non-positive entry or a sum that does not fit in int64_t.
  */
 int64_t pe_num_patches(const int32_t *grid_thw, int n);
 

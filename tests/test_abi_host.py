@@ -68,6 +68,11 @@ def test_num_patches(lib):
     assert _binding.pe_num_patches([]) == 0
     assert _binding.pe_num_patches([(1, 0, 4)]) == -1
     assert lib.pe_num_patches(None, 1) == -1
+    big = 2**31 - 1
+    assert _binding.pe_num_patches([(big, big, 2)]) == big * big * 2      # < 2^63: exact
+    assert _binding.pe_num_patches([(big, big, 3)]) == -1                 # product beyond int64
+    assert _binding.pe_num_patches([(big, big, 2), (big, big, 2)]) == -1  # sum beyond int64
+    assert _binding.pe_num_patches([(big, big, 2), (1, 1, 1)]) == big * big * 2 + 1
 
 
 def test_null_handle_calls_are_rejected(lib):

@@ -312,7 +312,7 @@ pe_status make_item(const pe_handle *h, const void *frames, int T, int H, int W,
     if (!aligned16(frames)) return PE_ERR_ALIGN;
     if (T < 1 || H < 1 || W < 1 || g[0] < 1 || g[1] < 1 || g[2] < 1) return PE_ERR_SHAPE;
     if ((int64_t)H != (int64_t)g[1] * h->p || (int64_t)W != (int64_t)g[2] * h->p) return PE_ERR_SHAPE;
-    if ((T + h->tp - 1) / h->tp != g[0]) return PE_ERR_SHAPE;
+    if (((int64_t)T + h->tp - 1) / h->tp != g[0]) return PE_ERR_SHAPE;
     if (merge == 2 && ((g[1] & 1) || (g[2] & 1))) return PE_ERR_SHAPE;
     if ((int64_t)T * h->C * H * W >= (int64_t)1 << 40) return PE_ERR_UNSUPPORTED;
     if ((int64_t)h->C * H * W > INT32_MAX) return PE_ERR_UNSUPPORTED;
@@ -617,7 +617,11 @@ int64_t pe_num_patches(const int32_t *grid_thw, int n) {
     for (int i = 0; i < n; ++i) {
         const int32_t *g = grid_thw + 3 * i;
         if (g[0] < 1 || g[1] < 1 || g[2] < 1) return -1;
-        s += (int64_t)g[0] * g[1] * g[2];
+        const int64_t th = (int64_t)g[0] * g[1];           // < 2^62: no overflow
+        if (th > INT64_MAX / g[2]) return -1;
+        const int64_t rows = th * g[2];
+        if (s > INT64_MAX - rows) return -1;
+        s += rows;
     }
     return s;
 }
@@ -1198,6 +1202,7 @@ void pe_merger_destroy(pe_merger *pm) {
     for (void *p : {(void *)pm->w1, (void *)pm->w2, (void *)pm->b1, (void *)pm->b2, (void *)pm->gamma,
                     (void *)pm->beta, (void *)pm->err, (void *)pm->ln_rows, (void *)pm->hid})
         if (p) cudaFree(p);
+    for (cudaEvent_t e : pm->core.prof_ev) cudaEventDestroy(e);   // profiling window left open
     delete pm;
 }
 
