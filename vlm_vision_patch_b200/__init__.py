@@ -25,12 +25,27 @@ def _dt(t: torch.dtype) -> int:
     raise TypeError(f"unsupported dtype {t}; use torch.float32 or torch.bfloat16")
 
 
-def _dev(t: torch.Tensor, name: str) -> int:
+def _dev(t: torch.Tensor, name: str, device: Optional[int] = None) -> int:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device.index != device:
+        raise ValueError(f"{name} is on cuda:{t.device.index}, the handle on cuda:{device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def _need(t: torch.Tensor, shape: Sequence[int], name: str) -> None:
+    """The C ABI takes raw pointers and trusts the documented layout, so a tensor
+    of the wrong shape would be read or written past its end: refuse it here."""
+    if tuple(t.shape) != tuple(int(v) for v in shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {tuple(int(v) for v in shape)}")
+
+
+def _need_frames(frames: Sequence[torch.Tensor], C: int) -> None:
+    for f in frames:
+        if f.dim() != 4 or f.shape[1] != C:
+            raise ValueError(f"frames must be [T, {C}, H, W]; got {tuple(f.shape)}")
 
 
 def _stream(stream) -> int:
@@ -52,6 +67,7 @@ class PatchEmbed:
         self.E, self.C, self.tp, self.p, self.has_bias = E, C, tp, p, bias
         self.K = C * tp * p * p
         self.h = B.pe_create(E, C, tp, p, bias)
+        self.dev = B.pe_device(self.h)
 
     # ------------------------------------------------------------ lifetime
     def close(self) -> None:
@@ -67,8 +83,14 @@ class PatchEmbed:
 
     # ------------------------------------------------------------ state
     def set_weight(self, w: torch.Tensor, bias: Optional[torch.Tensor] = None, stream=None) -> None:
-        B.pe_set_weight(self.h, _dev(w, "weight"), _dt(w.dtype),
-                        None if bias is None else _dev(bias, "bias"),
+        """w: [E, C, tp, p, p] (or [E, K] flattened in that order); bias: [E]."""
+        if w.shape[:1] != (self.E,) or w.numel() != self.E * self.K:
+            raise ValueError(f"weight has shape {tuple(w.shape)}; expected "
+                             f"{(self.E, self.C, self.tp, self.p, self.p)}")
+        if bias is not None and bias.numel() != self.E:
+            raise ValueError(f"bias has shape {tuple(bias.shape)}; expected {(self.E,)}")
+        B.pe_set_weight(self.h, _dev(w, "weight", self.dev), _dt(w.dtype),
+                        None if bias is None else _dev(bias, "bias", self.dev),
                         _dt(bias.dtype) if bias is not None else PE_F32, _stream(stream))
 
     def set_norm(self, mean: Sequence[float], std: Sequence[float]) -> None:
@@ -91,30 +113,49 @@ class PatchEmbed:
     def _out(self, n: int, out, out_dtype, device):
         if out is None:
             out = torch.empty((n, self.E), dtype=out_dtype, device=device)
+        _need(out, (n, self.E), "out")
         return out
 
     def forward_patches(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
                         out_dtype: torch.dtype = torch.bfloat16, stream=None,
                         pos: Optional[torch.Tensor] = None) -> torch.Tensor:
         """out = x @ W^T (+ bias) (+ pos, a [N, E] table added in the same epilogue)."""
+        if x.dim() != 2 or x.shape[1] != self.K:
+            raise ValueError(f"x must be [N, {self.K}]; got {tuple(x.shape)}")
         out = self._out(x.shape[0], out, out_dtype, x.device)
+        if pos is not None:
+            _need(pos, (x.shape[0], self.E), "pos")
+        d = self.dev
         if pos is None:
-            B.pe_forward_patches(self.h, _dev(x, "x"), _dt(x.dtype), x.shape[0], _dev(out, "out"),
+            B.pe_forward_patches(self.h, _dev(x, "x", d), _dt(x.dtype), x.shape[0], _dev(out, "out", d),
                                  _dt(out.dtype), _stream(stream))
         else:
-            B.pe_forward_patches_pos(self.h, _dev(x, "x"), _dt(x.dtype), x.shape[0], _dev(pos, "pos"),
-                                     _dt(pos.dtype), _dev(out, "out"), _dt(out.dtype), _stream(stream))
+            B.pe_forward_patches_pos(self.h, _dev(x, "x", d), _dt(x.dtype), x.shape[0], _dev(pos, "pos", d),
+                                     _dt(pos.dtype), _dev(out, "out", d), _dt(out.dtype), _stream(stream))
         return out
 
     def forward_frames(self, frames: torch.Tensor, grid_thw: Sequence[int], merge: int = 2,
                        out: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
                        stream=None) -> torch.Tensor:
+        _need_frames([frames], self.C)
+        if len(grid_thw) != 3:
+            raise ValueError("grid_thw must be (t, h, w)")
         T, C, H, W = frames.shape
         n = int(grid_thw[0]) * int(grid_thw[1]) * int(grid_thw[2])
         out = self._out(n, out, out_dtype, frames.device)
-        B.pe_forward_frames(self.h, _dev(frames, "frames"), _dt(frames.dtype), T, H, W, grid_thw, merge,
-                            _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        B.pe_forward_frames(self.h, _dev(frames, "frames", self.dev), _dt(frames.dtype), T, H, W, grid_thw, merge,
+                            _dev(out, "out", self.dev), _dt(out.dtype), _stream(stream))
         return out
+
+    def _items(self, frames, grid_thw):
+        if len(frames) == 0 or len(frames) != len(grid_thw):
+            raise ValueError(f"{len(frames)} frame tensors for {len(grid_thw)} grids; need one per item, at least one")
+        if any(len(g) != 3 for g in grid_thw):
+            raise ValueError("every grid_thw entry must be (t, h, w)")
+        _need_frames(frames, self.C)
+        if len({f.dtype for f in frames}) != 1:
+            raise TypeError("all items must share one dtype")
+        return sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
 
     def forward_frames_grouped(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]],
                                merge: int = 2, out: Optional[torch.Tensor] = None,
@@ -122,27 +163,27 @@ class PatchEmbed:
                                pos: Optional[torch.Tensor] = None) -> torch.Tensor:
         """All items in one launch; `pos`, if given, is a [N, E] table in output row
         order added in the same epilogue."""
-        n = sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
+        n = self._items(frames, grid_thw)
         out = self._out(n, out, out_dtype, frames[0].device)
-        dts = {f.dtype for f in frames}
-        if len(dts) != 1:
-            raise TypeError("all items must share one dtype")
-        ptrs = [_dev(f, "frames") for f in frames]
+        if pos is not None:
+            _need(pos, (n, self.E), "pos")
+        d = self.dev
+        ptrs = [_dev(f, "frames", d) for f in frames]
         thw = [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames]
         if pos is None:
             B.pe_forward_frames_grouped(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
-                                        _dev(out, "out"), _dt(out.dtype), _stream(stream))
+                                        _dev(out, "out", d), _dt(out.dtype), _stream(stream))
         else:
             B.pe_forward_frames_grouped_pos(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
-                                            _dev(pos, "pos"), _dt(pos.dtype), _dev(out, "out"), _dt(out.dtype),
-                                            _stream(stream))
+                                            _dev(pos, "pos", d), _dt(pos.dtype), _dev(out, "out", d),
+                                            _dt(out.dtype), _stream(stream))
         return out
 
     def patchify(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]], merge: int = 2,
                  rows_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
-        n = sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
+        n = self._items(frames, grid_thw)
         rows = torch.empty((n, self.K), dtype=rows_dtype, device=frames[0].device)
-        B.pe_patchify(self.h, [_dev(f, "frames") for f in frames], _dt(frames[0].dtype),
+        B.pe_patchify(self.h, [_dev(f, "frames", self.dev) for f in frames], _dt(frames[0].dtype),
                       [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames], grid_thw, merge,
                       _dev(rows, "rows"), _dt(rows.dtype), _stream(stream))
         return rows
@@ -155,24 +196,37 @@ class PatchMerger:
 
     def __init__(self, E: int, m: int, H: int, eps: float = 1e-6):
         self.E, self.m2, self.H = E, m * m, H
+        self.D = E * m * m
         self.h = B.pe_merger_create(E, m, H, eps)
+        self.dev = torch.cuda.current_device()   # the device pe_merger_create bound the handle to
 
     def set_weights(self, gamma: torch.Tensor, beta: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor],
                     w2: torch.Tensor, b2: Optional[torch.Tensor], stream=None) -> None:
+        """gamma, beta: [E]; w1: [D, D], b1: [D]; w2: [H, D], b2: [H] (D = m*m*E)."""
+        E, D, H = self.E, self.D, self.H
+        for t, shape, name in ((gamma, (E,), "gamma"), (beta, (E,), "beta"), (w1, (D, D), "w1"),
+                               (b1, (D,), "b1"), (w2, (H, D), "w2"), (b2, (H,), "b2")):
+            if t is not None:
+                _need(t, shape, name)
         ts = [gamma, beta, w1, w2] + [t for t in (b1, b2) if t is not None]
         if len({t.dtype for t in ts}) != 1:
             raise TypeError("all merger weights must share one dtype")
         self._keep = ts
-        B.pe_merger_set_weights(self.h, _dev(gamma, "gamma"), _dev(beta, "beta"), _dev(w1, "w1"),
-                                None if b1 is None else _dev(b1, "b1"), _dev(w2, "w2"),
-                                None if b2 is None else _dev(b2, "b2"), _dt(w1.dtype), _stream(stream))
+        d = self.dev
+        B.pe_merger_set_weights(self.h, _dev(gamma, "gamma", d), _dev(beta, "beta", d), _dev(w1, "w1", d),
+                                None if b1 is None else _dev(b1, "b1", d), _dev(w2, "w2", d),
+                                None if b2 is None else _dev(b2, "b2", d), _dt(w1.dtype), _stream(stream))
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
                 stream=None) -> torch.Tensor:
+        if x.dim() != 2 or x.shape[1] != self.E:
+            raise ValueError(f"x must be [N, {self.E}]; got {tuple(x.shape)}")
         V = x.shape[0] // self.m2
         if out is None:
             out = torch.empty((V, self.H), dtype=out_dtype, device=x.device)
-        B.pe_merger_forward(self.h, _dev(x, "x"), x.shape[0], _dev(out, "out"), _dt(out.dtype), _stream(stream))
+        _need(out, (V, self.H), "out")
+        B.pe_merger_forward(self.h, _dev(x, "x", self.dev), x.shape[0], _dev(out, "out", self.dev), _dt(out.dtype),
+                            _stream(stream))
         return out
 
     def last_error(self) -> int:
