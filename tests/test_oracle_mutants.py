@@ -52,6 +52,23 @@ MUTANTS = {
     "merger_ln_drops_beta": ("* (double)gamma[e] + (double)beta[e];", "* (double)gamma[e];"),
     "patchify_drops_time_offset": ("const int64_t tau = g_t * tp + t;\n                        rows",
                                    "const int64_t tau = g_t * tp;\n                        rows"),
+    "norm_uses_first_channel_constants": ("oracle_normalize_pixel(s[q], mean[c], std[c])",
+                                          "oracle_normalize_pixel(s[q], mean[0], std[0])"),
+    "frames_temporal_slices_reversed": ("const int64_t tau = g_t * tp + t;\n                            const int64_t y",
+                                        "const int64_t tau = g_t * tp + (tp - 1 - t);\n"
+                                        "                            const int64_t y"),
+    "patches_weight_transposed": ("const double wv = (double)wb[(int64_t)e * K + k];",
+                                  "const double wv = (double)wb[k * E + e];"),
+    "accumulates_in_fp32": ("double acc = 0.0, mag = 0.0;", "float acc = 0.0f; double mag = 0.0;"),
+    "raster_order_w_major": ("return (g_t * h + g_h) * w + g_w;", "return (g_t * w + g_w) * h + g_h;"),
+    "merger_gelu_tanh_form": ("const double gl = 0.5 * y * (1.0 + erf(y / sqrt(2.0)));",
+                              "const double gl = 0.5 * y * (1.0 + tanh(0.7978845608028654 * (y + 0.044715 * y * y * y)));"),
+    "merger_eps_outside_sqrt": ("const double inv = 1.0 / sqrt(var + eps);",
+                                "const double inv = 1.0 / (sqrt(var) + eps);"),
+    "merger_second_moment_as_variance": ("var += ((double)row[e] - mean) * ((double)row[e] - mean);",
+                                         "var += (double)row[e] * (double)row[e];"),
+    "merger_fc2_takes_fc1_bias": ("out[v * H + h] = acc + (b2 ? (double)b2[h] : 0.0);",
+                                  "out[v * H + h] = acc + (b2 ? (double)b1[h] : 0.0);"),
 }
 
 

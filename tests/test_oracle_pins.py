@@ -351,12 +351,14 @@ def _bf16(t):
     return t.to(torch.bfloat16).double()
 
 
-@pytest.mark.parametrize("E,m2,H,with_bias", [(8, 4, 5, True), (12, 4, 3, False), (6, 1, 4, True)])
-def test_patch_merger_matches_torch(E, m2, H, with_bias):
+@pytest.mark.parametrize("E,m2,H,with_bias,eps", [(8, 4, 5, True, 1e-6), (12, 4, 3, False, 1e-6),
+                                                  (6, 1, 4, True, 1e-6), (8, 4, 5, True, 0.5)])
+def test_patch_merger_matches_torch(E, m2, H, with_bias, eps):
     """LayerNorm -> concat of m2 rows -> fc1 -> exact GELU -> fc2, against torch's
     fp64 layer_norm / linear / gelu library routines with the same bf16 roundings
     of the LayerNorm output, the GELU output and the weights (mytransformer
-    README §3.2 and §4.1)."""
+    README §3.2 and §4.1).  The large eps makes the place of eps visible: it is
+    added to the variance under the square root."""
     g = torch.Generator().manual_seed(400 + E + m2)
     V = 5
     D = E * m2
@@ -367,7 +369,6 @@ def test_patch_merger_matches_torch(E, m2, H, with_bias):
     w2 = torch.randn(H, D, generator=g) * 0.2
     b1 = torch.randn(D, generator=g) * 0.1 if with_bias else None
     b2 = torch.randn(H, generator=g) * 0.1 if with_bias else None
-    eps = 1e-6
     out, mag = oracle.patch_merger(x, m2, gamma, beta, eps, w1, b1, w2, b2)
     ln = torch.nn.functional.layer_norm(x.double(), (E,), gamma.double(), beta.double(), eps)
     h = _bf16(ln.float()).view(V, D)
