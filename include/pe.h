@@ -270,6 +270,53 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
                                             void *out, pe_dtype out_dt, pe_stream_t stream);
 
 /*
+ * pe_forward_frames_grouped_host -- pe_forward_frames_grouped with the frames
+ * and the output in HOST memory: the call copies the frames in, embeds them
+ * and copies the rows out.  It is the call for a caller whose decoded frames
+ * sit in host memory and who wants the embeddings back there.  The pages have
+ * no counterpart; the arithmetic is exactly that of the device-pointer call.
+ *   frames_host : host array of n host pointers, item i is
+ *                 [THW[3i], C, THW[3i+1], THW[3i+2]] of dtype f_dt, dense
+ *   out_host    : host [sum_i gt_i*gh_i*gw_i, E] of dtype out_dt, dense
+ *   Other arguments as pe_forward_frames_grouped.
+ * The items are cut into chunks of about an eighth of the rows (at least 8192
+ * rows; whole items, and whole temporal patches of a video, which are
+ * contiguous output rows).  Each chunk is copied into one of two device input
+ * slots on the handle's copy-in stream, computed on `stream` by the
+ * device-pointer path, and copied out of one of two output slots on the
+ * handle's copy-out stream; so one chunk's copy in, another's contraction and
+ * a third's copy out overlap.  The environment variable PE_HOST_CHUNK_ROWS
+ * overrides the chunk size.
+ * Ordering: the copies start after the work already queued on `stream`, and
+ * `stream` waits for the last copy out, so out_host is complete once `stream`
+ * has drained (cudaStreamSynchronize, or an event recorded after the call).
+ * The host buffers must stay valid and unchanged until then.  Pinned host
+ * memory (cudaMallocHost / cudaHostRegister) gives the overlap; with pageable
+ * memory the copies are staged by the CUDA driver and the call blocks the host
+ * on each copy.
+ * Workspace: the handle's grow-only device slots and two streams, created on
+ * first use; calls on one handle must be serialised on one stream.
+ * Errors: as pe_forward_frames_grouped; every item is validated before
+ * anything is copied or launched.  A CUDA error after work was queued returns
+ * PE_ERR_CUDA with the earlier chunks possibly done.
+ */
+pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const *frames_host, pe_dtype f_dt,
+                                         const int32_t *THW, const int32_t *grid_thw, int merge, void *out_host,
+                                         pe_dtype out_dt, pe_stream_t stream);
+
+/*
+ * pe_forward_patches_host -- pe_forward_patches with x and out in HOST memory,
+ * pipelined over row chunks exactly as pe_forward_frames_grouped_host.
+ *   x_host   : host [N, K] of dtype x_dt, dense, rows as in pe_forward_patches
+ *   out_host : host [N, E] of dtype out_dt, dense
+ * Ordering, workspace and pinned-memory notes as for
+ * pe_forward_frames_grouped_host.  N may be 0 (nothing is queued).
+ * Errors: PE_ERR_INVALID_ARG, PE_ERR_DTYPE, PE_ERR_NO_WEIGHT, PE_ERR_CUDA.
+ */
+pe_status pe_forward_patches_host(pe_handle *h, const void *x_host, pe_dtype x_dt, int64_t N, void *out_host,
+                                  pe_dtype out_dt, pe_stream_t stream);
+
+/*
  * pe_patchify -- test hook: the fused producer's gather and normalisation
  * written out to memory instead of feeding the tensor cores.
  *   rows : dev [sum_i N_i, K] of dtype rows_dt (PE_BF16 or PE_F32; values are

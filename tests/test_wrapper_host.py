@@ -3,7 +3,9 @@
 The C ABI takes raw device pointers and trusts the documented layouts, so the
 wrapper must refuse a tensor whose shape does not match before any pointer is
 handed over.  The objects are built without a handle (no pe_create), so every
-case here has to be refused before the wrapper reaches the C library."""
+case here has to be refused before the wrapper reaches the C library, except
+the well-formed host-buffer calls, which reach it and are refused there for the
+missing handle."""
 from __future__ import annotations
 
 import pytest
@@ -112,3 +114,25 @@ def test_merger_shapes():
         kw = dict(good, **{name: bad})
         with pytest.raises(ValueError, match=f"{name} has shape"):
             pm.set_weights(**kw)
+
+
+def test_host_buffer_calls_check_shapes_then_reach_the_library():
+    from vlm_vision_patch_b200 import PEError
+    pe = _pe()
+    with pytest.raises(ValueError, match="x must be"):
+        pe.forward_patches_host(z(4, K + 2))
+    with pytest.raises(ValueError, match="out has shape"):
+        pe.forward_patches_host(z(4, K), out=z(4, E + 8))
+    f = z(1, C, 28, 28)
+    with pytest.raises(ValueError, match="one per item"):
+        pe.forward_frames_grouped_host([f], [(1, 2, 2), (1, 2, 2)])
+    with pytest.raises(ValueError, match="out has shape"):
+        pe.forward_frames_grouped_host([f], [(1, 2, 2)], out=z(3, E))
+    # well-formed host tensors reach the C call (raw stream handle 0: no CUDA
+    # query on the way), which refuses the missing handle
+    with pytest.raises(PEError) as e:
+        pe.forward_patches_host(z(4, K), stream=0, blocking=False)
+    assert e.value.status == "PE_ERR_INVALID_ARG"
+    with pytest.raises(PEError) as e:
+        pe.forward_frames_grouped_host([f], [(1, 2, 2)], stream=0, blocking=False)
+    assert e.value.status == "PE_ERR_INVALID_ARG"

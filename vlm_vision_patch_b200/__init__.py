@@ -35,6 +35,21 @@ def _dev(t: torch.Tensor, name: str, device: Optional[int] = None) -> int:
     return t.data_ptr()
 
 
+def _host(t: torch.Tensor, name: str) -> int:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _host_out(shape, out, out_dtype) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, pin_memory=torch.cuda.is_available())
+    _need(out, shape, "out")
+    return out
+
+
 def _need(t: torch.Tensor, shape: Sequence[int], name: str) -> None:
     """The C ABI takes raw pointers and trusts the documented layout, so a tensor
     of the wrong shape would be read or written past its end: refuse it here."""
@@ -54,6 +69,16 @@ def _stream(stream) -> int:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def _sync(stream) -> None:
+    """Wait for `stream` (None: the current stream; a raw handle: the device)."""
+    if stream is None:
+        torch.cuda.current_stream().synchronize()
+    elif isinstance(stream, torch.cuda.Stream):
+        stream.synchronize()
+    else:
+        torch.cuda.synchronize()
 
 
 def num_patches(grid_thw: Sequence[Sequence[int]]) -> int:
@@ -177,6 +202,41 @@ class PatchEmbed:
             B.pe_forward_frames_grouped_pos(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
                                             _dev(pos, "pos", d), _dt(pos.dtype), _dev(out, "out", d),
                                             _dt(out.dtype), _stream(stream))
+        return out
+
+    def forward_frames_grouped_host(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]],
+                                    merge: int = 2, out: Optional[torch.Tensor] = None,
+                                    out_dtype: torch.dtype = torch.bfloat16, stream=None,
+                                    blocking: bool = True) -> torch.Tensor:
+        """forward_frames_grouped with host (CPU) frames and a host output: the
+        library copies the frames in and the rows out in pipelined chunks.  Pinned
+        tensors (``pin_memory()``) overlap the copies; the default output is
+        pinned.  With ``blocking=False`` the output is complete only once the
+        stream has drained."""
+        n = self._items(frames, grid_thw)
+        out = _host_out((n, self.E), out, out_dtype)
+        ptrs = [_host(f, "frames") for f in frames]
+        thw = [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames]
+        st = _stream(stream)
+        B.pe_forward_frames_grouped_host(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
+                                         _host(out, "out"), _dt(out.dtype), st)
+        if blocking:
+            _sync(stream)
+        return out
+
+    def forward_patches_host(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                             out_dtype: torch.dtype = torch.bfloat16, stream=None,
+                             blocking: bool = True) -> torch.Tensor:
+        """forward_patches with host (CPU) rows in and out, pipelined in chunks
+        (see forward_frames_grouped_host)."""
+        if x.dim() != 2 or x.shape[1] != self.K:
+            raise ValueError(f"x must be [N, {self.K}]; got {tuple(x.shape)}")
+        out = _host_out((x.shape[0], self.E), out, out_dtype)
+        st = _stream(stream)
+        B.pe_forward_patches_host(self.h, _host(x, "x"), _dt(x.dtype), x.shape[0], _host(out, "out"),
+                                  _dt(out.dtype), st)
+        if blocking:
+            _sync(stream)
         return out
 
     def patchify(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]], merge: int = 2,

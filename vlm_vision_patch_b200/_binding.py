@@ -31,7 +31,7 @@ EXPORTS = (
     "pe_status_string", "pe_destroy", "pe_device", "pe_profile_begin", "pe_profile_end",
     "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos", "pe_set_tf32",
     "pe_merger_create", "pe_merger_set_weights", "pe_merger_forward", "pe_merger_last_error", "pe_merger_destroy",
-    "pe_merger_profile_begin", "pe_merger_profile_end",
+    "pe_merger_profile_begin", "pe_merger_profile_end", "pe_forward_frames_grouped_host", "pe_forward_patches_host",
 )
 
 
@@ -80,6 +80,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_forward_frames_grouped": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
         "pe_forward_frames_grouped_noalloc": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
         "pe_patchify": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
+        "pe_forward_frames_grouped_host": ([vp, i32, ctypes.POINTER(vp), i32, i32p, i32p, i32, vp, i32, vp], i32),
+        "pe_forward_patches_host": ([vp, vp, i32, i64, vp, i32, vp], i32),
         "pe_num_patches": ([i32p, i32], i64),
         "pe_last_error": ([vp], i32),
         "pe_status_string": ([i32], ctypes.c_char_p),
@@ -192,6 +194,20 @@ def pe_forward_frames_grouped_noalloc(h: int, f_ptrs: Sequence[int], f_dt: int, 
     _check("pe_forward_frames_grouped_noalloc", load().pe_forward_frames_grouped_noalloc(
         h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
         _i32arr([v for g in grid_thw for v in g]), merge, out_ptr, out_dt, stream))
+
+
+def pe_forward_frames_grouped_host(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence[int]],
+                                   grid_thw: Sequence[Sequence[int]], merge: int, out_ptr: int, out_dt: int,
+                                   stream: int) -> None:
+    """Host pointers in and out (see include/pe.h)."""
+    n = len(f_ptrs)
+    _check("pe_forward_frames_grouped_host", load().pe_forward_frames_grouped_host(
+        h, n, _ptrs(f_ptrs), f_dt, _i32arr([v for t in THW for v in t]),
+        _i32arr([v for g in grid_thw for v in g]), merge, out_ptr, out_dt, stream))
+
+
+def pe_forward_patches_host(h: int, x_ptr: int, x_dt: int, N: int, out_ptr: int, out_dt: int, stream: int) -> None:
+    _check("pe_forward_patches_host", load().pe_forward_patches_host(h, x_ptr, x_dt, N, out_ptr, out_dt, stream))
 
 
 def pe_patchify(h: int, f_ptrs: Sequence[int], f_dt: int, THW: Sequence[Sequence[int]],

@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "../../include/pe.h"
+#include "pe_host_plan.h"
 #include "pe_kernels.cuh"
 
 using namespace pe;
@@ -64,6 +65,12 @@ struct pe_handle {
     bool prof_on = false;
     cudaEvent_t items_evt = nullptr;
     bool items_evt_pending = false;
+    // host-buffer calls: two input and two output slots in one device buffer,
+    // a copy-in and a copy-out stream, and per-slot events (created on first use)
+    uint8_t *host_ws = nullptr;
+    size_t host_ws_in = 0, host_ws_out = 0;   // bytes of one input / one output slot
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
 };
 
 namespace {
@@ -698,6 +705,12 @@ void pe_destroy(pe_handle *h) {
     if (h->ready) cudaFree(h->ready);
     if (h->items_evt) cudaEventDestroy(h->items_evt);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
+    if (h->host_ws) cudaFree(h->host_ws);
+    for (cudaStream_t s : {h->s_in, h->s_out})
+        if (s) cudaStreamDestroy(s);
+    for (cudaEvent_t e : {h->ev_start, h->ev_in[0], h->ev_in[1], h->ev_comp[0], h->ev_comp[1], h->ev_out[0],
+                          h->ev_out[1]})
+        if (e) cudaEventDestroy(e);
     delete h;
 }
 
@@ -1086,6 +1099,202 @@ pe_status pe_last_error(pe_handle *h) {
     if (cudaMemcpy(&v, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PE_ERR_CUDA;
     if (v != 0 && cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return PE_ERR_CUDA;
     return v == 0 ? PE_OK : (pe_status)v;
+}
+
+// ---------------------------------------------------------------------------
+// Host-buffer calls: the call's inputs and outputs live in host memory.  The
+// work is cut into chunks (pe_host_plan.h); chunk c uses input and output slot
+// c % 2 of the handle's device buffer.  Its inputs are copied in on the
+// handle's copy-in stream, its rows computed on the caller's stream by the
+// device-pointer path, and copied out on the handle's copy-out stream, so
+// that (with pinned host memory) the copies in both directions and the
+// contraction of neighbouring chunks overlap.  Events order the slots:
+//   copy-in of c  waits for the contraction of c - 2 (input slot free),
+//   contraction of c  waits for copy-in of c and copy-out of c - 2,
+//   copy-out of c  waits for the contraction of c.
+// The caller's stream waits for the last copy-out before the call returns.
+}  // extern "C"
+
+namespace {
+
+pe_status host_pipe_init(pe_handle *h) {
+    bool ok = true;
+    for (cudaStream_t *s : {&h->s_in, &h->s_out})
+        if (ok && !*s) ok = cudaStreamCreateWithFlags(s, cudaStreamNonBlocking) == cudaSuccess;
+    for (cudaEvent_t *e : {&h->ev_start, &h->ev_in[0], &h->ev_in[1], &h->ev_comp[0], &h->ev_comp[1], &h->ev_out[0],
+                           &h->ev_out[1]})
+        if (ok && !*e) ok = cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+    return ok ? PE_OK : PE_ERR_CUDA;   // objects already created are kept and released by pe_destroy
+}
+
+// Grow-only slots; the old buffer is freed only after every stream that may
+// still use it has drained.
+pe_status host_slots(pe_handle *h, int64_t in_bytes, int64_t out_bytes, cudaStream_t st) {
+    const size_t in = (size_t)pe_plan::align_up(std::max<int64_t>(in_bytes, 1), pe_plan::kSlotAlign);
+    const size_t out = (size_t)pe_plan::align_up(std::max<int64_t>(out_bytes, 1), pe_plan::kSlotAlign);
+    if (in <= h->host_ws_in && out <= h->host_ws_out) return PE_OK;
+    const size_t new_in = std::max(in, h->host_ws_in), new_out = std::max(out, h->host_ws_out);
+    if (h->host_ws) {
+        if (cudaStreamSynchronize(st) != cudaSuccess || cudaStreamSynchronize(h->s_in) != cudaSuccess ||
+            cudaStreamSynchronize(h->s_out) != cudaSuccess)
+            return PE_ERR_CUDA;
+        cudaFree(h->host_ws);
+    }
+    h->host_ws = nullptr;
+    h->host_ws_in = h->host_ws_out = 0;
+    if (cudaMalloc(&h->host_ws, 2 * (new_in + new_out)) != cudaSuccess) return PE_ERR_CUDA;
+    h->host_ws_in = new_in;
+    h->host_ws_out = new_out;
+    return PE_OK;
+}
+
+uint8_t *slot_in(const pe_handle *h, int s) { return h->host_ws + (size_t)s * h->host_ws_in; }
+uint8_t *slot_out(const pe_handle *h, int s) { return h->host_ws + 2 * h->host_ws_in + (size_t)s * h->host_ws_out; }
+
+// Chunk rows: PE_HOST_CHUNK_ROWS overrides the planner's choice (tests use it
+// to force many small chunks).
+int64_t host_chunk_rows(int64_t N) {
+    if (const char *s = std::getenv("PE_HOST_CHUNK_ROWS")) {
+        const long long v = std::atoll(s);
+        if (v > 0) return (int64_t)v;
+    }
+    return pe_plan::chunk_rows(N);
+}
+
+template <class CopyIn, class Compute, class CopyOut>
+pe_status run_host_pipeline(pe_handle *h, int nchunks, cudaStream_t st, CopyIn copy_in, Compute compute,
+                            CopyOut copy_out) {
+    if (cudaEventRecord(h->ev_start, st) != cudaSuccess || cudaStreamWaitEvent(h->s_in, h->ev_start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(h->s_out, h->ev_start, 0) != cudaSuccess)
+        return PE_ERR_CUDA;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        if (c >= 2 && cudaStreamWaitEvent(h->s_in, h->ev_comp[s], 0) != cudaSuccess) return PE_ERR_CUDA;
+        pe_status r = copy_in(c, slot_in(h, s), h->s_in);
+        if (r != PE_OK) return r;
+        if (cudaEventRecord(h->ev_in[s], h->s_in) != cudaSuccess || cudaStreamWaitEvent(st, h->ev_in[s], 0) != cudaSuccess)
+            return PE_ERR_CUDA;
+        if (c >= 2 && cudaStreamWaitEvent(st, h->ev_out[s], 0) != cudaSuccess) return PE_ERR_CUDA;
+        r = compute(c, slot_in(h, s), slot_out(h, s), st);
+        if (r != PE_OK) return r;
+        if (cudaEventRecord(h->ev_comp[s], st) != cudaSuccess || cudaStreamWaitEvent(h->s_out, h->ev_comp[s], 0) != cudaSuccess)
+            return PE_ERR_CUDA;
+        r = copy_out(c, slot_out(h, s), h->s_out);
+        if (r != PE_OK) return r;
+        if (cudaEventRecord(h->ev_out[s], h->s_out) != cudaSuccess) return PE_ERR_CUDA;
+    }
+    // the copy-out stream is in order: its last event covers every chunk
+    if (cudaEventRecord(h->ev_start, h->s_out) != cudaSuccess || cudaStreamWaitEvent(st, h->ev_start, 0) != cudaSuccess)
+        return PE_ERR_CUDA;
+    return PE_OK;
+}
+
+alignas(16) const unsigned char kStandIn[16] = {};   // validation stand-in for a frames pointer
+
+}  // namespace
+
+extern "C" {
+
+pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const *frames_host, pe_dtype f_dt,
+                                         const int32_t *THW, const int32_t *grid_thw, int merge, void *out_host,
+                                         pe_dtype out_dt, pe_stream_t stream) {
+    if (!h || n < 1 || !frames_host || !THW || !grid_thw || !out_host) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(f_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
+    if (merge != 1 && merge != 2) return PE_ERR_INVALID_ARG;
+    if (!h->weight_set) return PE_ERR_NO_WEIGHT;
+    if ((h->p & 1) || h->p > PE_MAX_PATCH) return PE_ERR_UNSUPPORTED;
+    // Every item is validated as the device-pointer call validates it, before
+    // anything is allocated, copied or launched.
+    const int64_t es = f_dt == PE_F32 ? 4 : 2;
+    std::vector<int64_t> frame_bytes((size_t)n);
+    int64_t N = 0;
+    for (int i = 0; i < n; ++i) {
+        if (!frames_host[i]) return PE_ERR_INVALID_ARG;
+        ItemDesc d;
+        const pe_status s = make_item(h, kStandIn, THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid_thw + 3 * i, merge,
+                                      N, d);
+        if (s != PE_OK) return s;
+        frame_bytes[(size_t)i] = (int64_t)h->C * THW[3 * i + 1] * THW[3 * i + 2] * es;
+        N += (int64_t)grid_thw[3 * i] * grid_thw[3 * i + 1] * grid_thw[3 * i + 2];
+    }
+    DeviceGuard g(h->dev);
+    cudaStream_t st = (cudaStream_t)stream;
+    const pe_plan::Plan pl = pe_plan::plan_frames(n, THW, grid_thw, h->tp, frame_bytes.data(), host_chunk_rows(N));
+    const int64_t row_bytes = (int64_t)h->E * (out_dt == PE_F32 ? 4 : 2);
+    pe_status r = host_pipe_init(h);
+    if (r == PE_OK) r = host_slots(h, pl.max_in, pl.max_rows * row_bytes, st);
+    if (r != PE_OK) return r;
+    std::vector<const void *> ptrs;
+    std::vector<int32_t> thw, grid;
+    auto copy_in = [&](int c, uint8_t *slot, cudaStream_t s) -> pe_status {
+        const pe_plan::Chunk &ch = pl.chunks[(size_t)c];
+        for (int j = ch.first; j < ch.first + ch.count; ++j) {
+            const pe_plan::SubItem &sb = pl.subs[(size_t)j];
+            const char *src = static_cast<const char *>(frames_host[sb.item]) + (int64_t)sb.f0 * frame_bytes[(size_t)sb.item];
+            if (cudaMemcpyAsync(slot + sb.in_off, src, (size_t)sb.in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return PE_ERR_CUDA;
+        }
+        return PE_OK;
+    };
+    auto compute = [&](int c, uint8_t *in, uint8_t *out, cudaStream_t s) -> pe_status {
+        const pe_plan::Chunk &ch = pl.chunks[(size_t)c];
+        ptrs.clear();
+        thw.clear();
+        grid.clear();
+        for (int j = ch.first; j < ch.first + ch.count; ++j) {
+            const pe_plan::SubItem &sb = pl.subs[(size_t)j];
+            const int32_t *it = THW + 3 * sb.item, *gr = grid_thw + 3 * sb.item;
+            ptrs.push_back(in + sb.in_off);
+            thw.insert(thw.end(), {sb.T, it[1], it[2]});
+            grid.insert(grid.end(), {sb.gt, gr[1], gr[2]});
+        }
+        return forward_frames_grouped(h, ch.count, ptrs.data(), f_dt, thw.data(), grid.data(), merge, nullptr, PE_BF16,
+                                      out, out_dt, s);
+    };
+    auto copy_out = [&](int c, uint8_t *slot, cudaStream_t s) -> pe_status {
+        const pe_plan::Chunk &ch = pl.chunks[(size_t)c];
+        return cudaMemcpyAsync(static_cast<char *>(out_host) + ch.row0 * row_bytes, slot, (size_t)(ch.rows * row_bytes),
+                               cudaMemcpyDeviceToHost, s) == cudaSuccess
+                   ? PE_OK
+                   : PE_ERR_CUDA;
+    };
+    return run_host_pipeline(h, (int)pl.chunks.size(), st, copy_in, compute, copy_out);
+}
+
+pe_status pe_forward_patches_host(pe_handle *h, const void *x_host, pe_dtype x_dt, int64_t N, void *out_host,
+                                  pe_dtype out_dt, pe_stream_t stream) {
+    if (!h || N < 0) return PE_ERR_INVALID_ARG;
+    if (!valid_dtype(x_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
+    if (!h->weight_set) return PE_ERR_NO_WEIGHT;
+    if (N == 0) return PE_OK;
+    if (!x_host || !out_host) return PE_ERR_INVALID_ARG;
+    DeviceGuard g(h->dev);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t per = std::min(host_chunk_rows(N), N);
+    const int64_t nch = (N + per - 1) / per;
+    if (nch > INT32_MAX) return PE_ERR_UNSUPPORTED;
+    const int64_t in_row = (int64_t)h->K * (x_dt == PE_F32 ? 4 : 2);
+    const int64_t out_row = (int64_t)h->E * (out_dt == PE_F32 ? 4 : 2);
+    pe_status r = host_pipe_init(h);
+    if (r == PE_OK) r = host_slots(h, per * in_row, per * out_row, st);
+    if (r != PE_OK) return r;
+    auto rows_of = [&](int c) { return std::min(per, N - (int64_t)c * per); };
+    auto copy_in = [&](int c, uint8_t *slot, cudaStream_t s) -> pe_status {
+        const char *src = static_cast<const char *>(x_host) + (int64_t)c * per * in_row;
+        return cudaMemcpyAsync(slot, src, (size_t)(rows_of(c) * in_row), cudaMemcpyHostToDevice, s) == cudaSuccess
+                   ? PE_OK
+                   : PE_ERR_CUDA;
+    };
+    auto compute = [&](int c, uint8_t *in, uint8_t *out, cudaStream_t s) -> pe_status {
+        return forward_patches(h, in, x_dt, rows_of(c), nullptr, PE_BF16, out, out_dt, s);
+    };
+    auto copy_out = [&](int c, uint8_t *slot, cudaStream_t s) -> pe_status {
+        char *dst = static_cast<char *>(out_host) + (int64_t)c * per * out_row;
+        return cudaMemcpyAsync(dst, slot, (size_t)(rows_of(c) * out_row), cudaMemcpyDeviceToHost, s) == cudaSuccess
+                   ? PE_OK
+                   : PE_ERR_CUDA;
+    };
+    return run_host_pipeline(h, (int)nch, st, copy_in, compute, copy_out);
 }
 
 // ---------------------------------------------------------------------------
