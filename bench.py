@@ -123,8 +123,30 @@ def dist_env():
 
 # ------------------------------------------------------------------ clocks
 
+def nvml_handle_for(nv, props):
+    """NVML handle of the CUDA device with properties `props`.  NVML numbers
+    every GPU of the machine and ignores CUDA_VISIBLE_DEVICES, so the device is
+    found by its PCI location (then by UUID).  Returns (handle, how) or
+    (None, None)."""
+    want = (int(props.pci_domain_id), int(props.pci_bus_id), int(props.pci_device_id))
+    handles = [nv.nvmlDeviceGetHandleByIndex(i) for i in range(nv.nvmlDeviceGetCount())]
+    for h in handles:
+        pci = nv.nvmlDeviceGetPciInfo(h)
+        if (int(pci.domain), int(pci.bus), int(pci.device)) == want:
+            return h, "pci"
+    uid = str(getattr(props, "uuid", "") or "")
+    if uid:
+        for h in handles:
+            u = nv.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else str(u)
+            if uid in u:
+                return h, "uuid"
+    return None, None
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while running."""
+    """Samples SM clock and clock-event reasons through NVML while running,
+    on the GPU that CUDA device `index` is."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -139,13 +161,19 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = None
         self.ok = False
+        self.match = None
 
     def __enter__(self):
         try:
             import pynvml
             pynvml.nvmlInit()
             self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            try:
+                self._h, self.match = nvml_handle_for(pynvml, torch.cuda.get_device_properties(self.index))
+            except Exception:
+                self._h, self.match = None, None
+            if self._h is None:   # no PCI or UUID match: NVML's own numbering, flagged as such
+                self._h, self.match = pynvml.nvmlDeviceGetHandleByIndex(self.index), "index (unverified)"
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -176,14 +204,14 @@ class ClockSampler:
 
     def summary(self):
         if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "gpu_match": self.match}
         mhz = [s[0] for s in self.samples]
         bits = 0
         for s in self.samples:
             bits |= s[1]
         names = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
         return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+                "reasons": names, "samples": len(self.samples), "gpu_match": self.match}
 
 
 # ------------------------------------------------------------------ oracle arm

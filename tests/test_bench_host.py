@@ -73,3 +73,40 @@ def test_reference_arm_prints_one_line_on_rank0():
     line = json.loads(buf.getvalue().strip())
     assert line["impl"] == "reference" and line["unit"] == "patches/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+class _FakeNVML:
+    """Three GPUs of a machine, as NVML numbers them (PCI order)."""
+
+    class _Pci:
+        def __init__(self, domain, bus, device):
+            self.domain, self.bus, self.device = domain, bus, device
+
+    def __init__(self):
+        self.gpus = [(0, 0x1B, 0, b"GPU-aaaa"), (0, 0x43, 0, b"GPU-bbbb"), (0, 0x52, 0, b"GPU-cccc")]
+
+    def nvmlDeviceGetCount(self):
+        return len(self.gpus)
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetPciInfo(self, h):
+        return self._Pci(*self.gpus[h][:3])
+
+    def nvmlDeviceGetUUID(self, h):
+        return self.gpus[h][3]
+
+
+def _props(domain, bus, device, uuid=""):
+    return type("P", (), dict(pci_domain_id=domain, pci_bus_id=bus, pci_device_id=device, uuid=uuid))()
+
+
+def test_clock_sampler_finds_the_cuda_device_among_all_gpus():
+    """With CUDA_VISIBLE_DEVICES picking one GPU of several, CUDA device 0 is
+    not NVML's GPU 0: the sampler must read the GPU at the same PCI location."""
+    nv = _FakeNVML()
+    assert bench.nvml_handle_for(nv, _props(0, 0x43, 0)) == (1, "pci")
+    assert bench.nvml_handle_for(nv, _props(0, 0x52, 0)) == (2, "pci")
+    assert bench.nvml_handle_for(nv, _props(0, 0x99, 0, "cccc")) == (2, "uuid")
+    assert bench.nvml_handle_for(nv, _props(0, 0x99, 0)) == (None, None)
