@@ -1161,32 +1161,37 @@ int64_t host_chunk_rows(int64_t N) {
     return pe_plan::chunk_rows(N);
 }
 
+// pe_plan::run_pipeline's stream/event interface on CUDA: the caller's
+// stream and the handle's copy streams and events.
+template <class CopyIn, class Compute, class CopyOut>
+struct CudaPipeOps {
+    pe_handle *h;
+    cudaStream_t st;
+    CopyIn &copy_in_fn;
+    Compute &compute_fn;
+    CopyOut &copy_out_fn;
+    cudaStream_t stream(int id) const {
+        return id == pe_plan::kCaller ? st : (id == pe_plan::kCopyIn ? h->s_in : h->s_out);
+    }
+    cudaEvent_t event(int id) const {
+        if (id == pe_plan::kEvStart) return h->ev_start;
+        if (id < pe_plan::kEvComp0) return h->ev_in[id - pe_plan::kEvIn0];
+        if (id < pe_plan::kEvOut0) return h->ev_comp[id - pe_plan::kEvComp0];
+        return h->ev_out[id - pe_plan::kEvOut0];
+    }
+    bool record(int e, int s) { return cudaEventRecord(event(e), stream(s)) == cudaSuccess; }
+    bool wait(int s, int e) { return cudaStreamWaitEvent(stream(s), event(e), 0) == cudaSuccess; }
+    int copy_in(int c, int s) { return (int)copy_in_fn(c, slot_in(h, s), h->s_in); }
+    int compute(int c, int s) { return (int)compute_fn(c, slot_in(h, s), slot_out(h, s), st); }
+    int copy_out(int c, int s) { return (int)copy_out_fn(c, slot_out(h, s), h->s_out); }
+};
+
 template <class CopyIn, class Compute, class CopyOut>
 pe_status run_host_pipeline(pe_handle *h, int nchunks, cudaStream_t st, CopyIn copy_in, Compute compute,
                             CopyOut copy_out) {
-    if (cudaEventRecord(h->ev_start, st) != cudaSuccess || cudaStreamWaitEvent(h->s_in, h->ev_start, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(h->s_out, h->ev_start, 0) != cudaSuccess)
-        return PE_ERR_CUDA;
-    for (int c = 0; c < nchunks; ++c) {
-        const int s = c & 1;
-        if (c >= 2 && cudaStreamWaitEvent(h->s_in, h->ev_comp[s], 0) != cudaSuccess) return PE_ERR_CUDA;
-        pe_status r = copy_in(c, slot_in(h, s), h->s_in);
-        if (r != PE_OK) return r;
-        if (cudaEventRecord(h->ev_in[s], h->s_in) != cudaSuccess || cudaStreamWaitEvent(st, h->ev_in[s], 0) != cudaSuccess)
-            return PE_ERR_CUDA;
-        if (c >= 2 && cudaStreamWaitEvent(st, h->ev_out[s], 0) != cudaSuccess) return PE_ERR_CUDA;
-        r = compute(c, slot_in(h, s), slot_out(h, s), st);
-        if (r != PE_OK) return r;
-        if (cudaEventRecord(h->ev_comp[s], st) != cudaSuccess || cudaStreamWaitEvent(h->s_out, h->ev_comp[s], 0) != cudaSuccess)
-            return PE_ERR_CUDA;
-        r = copy_out(c, slot_out(h, s), h->s_out);
-        if (r != PE_OK) return r;
-        if (cudaEventRecord(h->ev_out[s], h->s_out) != cudaSuccess) return PE_ERR_CUDA;
-    }
-    // the copy-out stream is in order: its last event covers every chunk
-    if (cudaEventRecord(h->ev_start, h->s_out) != cudaSuccess || cudaStreamWaitEvent(st, h->ev_start, 0) != cudaSuccess)
-        return PE_ERR_CUDA;
-    return PE_OK;
+    CudaPipeOps<CopyIn, Compute, CopyOut> ops{h, st, copy_in, compute, copy_out};
+    const int r = pe_plan::run_pipeline(ops, nchunks);
+    return r == 0 ? PE_OK : (r < 0 ? PE_ERR_CUDA : (pe_status)r);
 }
 
 alignas(16) const unsigned char kStandIn[16] = {};   // validation stand-in for a frames pointer

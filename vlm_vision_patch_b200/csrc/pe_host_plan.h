@@ -103,4 +103,44 @@ inline int64_t chunk_rows(int64_t N, int64_t min_rows = 8192) {
     return align_up(r, 256);
 }
 
+// The event protocol of the host-buffer calls, written once over an abstract
+// stream/event interface so that the same code runs on CUDA and in a model
+// that checks it for races.  Three streams: the caller's (contractions), a
+// copy-in and a copy-out stream.  Chunk c uses input and output slot c % 2.
+//   copy-in of c      waits for the contraction of c - 2 (input slot free)
+//   contraction of c  waits for copy-in of c and copy-out of c - 2 (output slot free)
+//   copy-out of c     waits for the contraction of c
+// Both copy streams first wait for the work queued on the caller's stream, and
+// the caller's stream finally waits for the last copy-out (the copy-out stream
+// is in order).  `ops` provides
+//   bool record(int event, int stream)   capture the stream's queued work
+//   bool wait(int stream, int event)     later work on `stream` waits for it
+//   int copy_in(int chunk, int slot), compute(int chunk, int slot),
+//   int copy_out(int chunk, int slot)    queue the chunk's work (0: ok)
+// Returns 0, the first non-zero status of a queueing call, or -1 when a record
+// or wait fails.
+enum PipeStream { kCaller = 0, kCopyIn = 1, kCopyOut = 2 };
+enum PipeEvent { kEvStart = 0, kEvIn0 = 1, kEvComp0 = 3, kEvOut0 = 5, kNumPipeEvents = 7 };
+
+template <class Ops>
+int run_pipeline(Ops &ops, int nchunks) {
+    if (!ops.record(kEvStart, kCaller) || !ops.wait(kCopyIn, kEvStart) || !ops.wait(kCopyOut, kEvStart)) return -1;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        if (c >= 2 && !ops.wait(kCopyIn, kEvComp0 + s)) return -1;
+        int r = ops.copy_in(c, s);
+        if (r != 0) return r;
+        if (!ops.record(kEvIn0 + s, kCopyIn) || !ops.wait(kCaller, kEvIn0 + s)) return -1;
+        if (c >= 2 && !ops.wait(kCaller, kEvOut0 + s)) return -1;
+        r = ops.compute(c, s);
+        if (r != 0) return r;
+        if (!ops.record(kEvComp0 + s, kCaller) || !ops.wait(kCopyOut, kEvComp0 + s)) return -1;
+        r = ops.copy_out(c, s);
+        if (r != 0) return r;
+        if (!ops.record(kEvOut0 + s, kCopyOut)) return -1;
+    }
+    if (!ops.record(kEvStart, kCopyOut) || !ops.wait(kCaller, kEvStart)) return -1;
+    return 0;
+}
+
 }  // namespace pe_plan
