@@ -355,6 +355,18 @@ pe_status pe_profile_begin(pe_handle *h, int max_calls);
 pe_status pe_profile_end(pe_handle *h, float *ms, int *n, int64_t *launches);
 
 /*
+ * pe_selftest_wait_timeout -- test hook for failure detection: one warp waits,
+ * through the bounded wait every pipeline uses, on a shared-memory barrier
+ * phase that nothing completes.  The wait gives up after its limit (2 s), and
+ * the kernel records PE_ERR_DEVICE_TIMEOUT in the handle's error word exactly
+ * as a contraction kernel whose pipeline stalled does; pe_last_error then
+ * reports and clears it, and the handle stays usable.  Nothing faults, traps
+ * or hangs.  Asynchronous on `stream`.
+ * Errors: PE_ERR_INVALID_ARG (NULL handle), PE_ERR_CUDA (launch failed).
+ */
+pe_status pe_selftest_wait_timeout(pe_handle *h, pe_stream_t stream);
+
+/*
  * pe_last_error -- read and clear the handle's device error word.  Call after
  * synchronising the streams the handle ran on.  Returns PE_OK, or
  * PE_ERR_DEVICE_TIMEOUT if a kernel stopped waiting on its pipeline (it then

@@ -32,6 +32,7 @@ EXPORTS = (
     "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos", "pe_set_tf32",
     "pe_merger_create", "pe_merger_set_weights", "pe_merger_forward", "pe_merger_last_error", "pe_merger_destroy",
     "pe_merger_profile_begin", "pe_merger_profile_end", "pe_forward_frames_grouped_host", "pe_forward_patches_host",
+    "pe_selftest_wait_timeout",
 )
 
 
@@ -84,6 +85,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_forward_patches_host": ([vp, vp, i32, i64, vp, i32, vp], i32),
         "pe_num_patches": ([i32p, i32], i64),
         "pe_last_error": ([vp], i32),
+        "pe_selftest_wait_timeout": ([vp, vp], i32),
         "pe_status_string": ([i32], ctypes.c_char_p),
         "pe_destroy": ([vp], None),
         "pe_device": ([vp], i32),
@@ -271,6 +273,10 @@ def pe_merger_last_error(pm: int) -> int:
 
 def pe_merger_destroy(pm: int) -> None:
     load().pe_merger_destroy(pm)
+
+
+def pe_selftest_wait_timeout(h: int, stream: int) -> None:
+    _check("pe_selftest_wait_timeout", load().pe_selftest_wait_timeout(h, stream))
 
 
 def pe_last_error(h: int) -> int:

@@ -1092,6 +1092,13 @@ pe_status pe_profile_end(pe_handle *h, float *ms, int *n, int64_t *launches) {
     return st;
 }
 
+pe_status pe_selftest_wait_timeout(pe_handle *h, pe_stream_t stream) {
+    if (!h) return PE_ERR_INVALID_ARG;
+    DeviceGuard g(h->dev);
+    pe_wait_timeout_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(h->err);
+    return finish(cudaGetLastError());
+}
+
 pe_status pe_last_error(pe_handle *h) {
     if (!h) return PE_ERR_INVALID_ARG;
     DeviceGuard g(h->dev);

@@ -1552,4 +1552,24 @@ __global__ void pe_patchify_kernel(const __grid_constant__ FwdParams P, void *ro
     }
 }
 
+// Failure-path self-test.  One warp waits, through the same bounded wait the
+// pipelines use (mbar_wait, kWaitTimeoutNs), on the first phase of a freshly
+// initialised shared-memory barrier that nothing ever completes.  The wait
+// gives up, sets the abort flag, and the kernel records PE_ERR_DEVICE_TIMEOUT
+// in the error word as pe_fwd_kernel does after an aborted wait.  The error
+// word is the only global memory it touches.
+__global__ void pe_wait_timeout_probe_kernel(int *err) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, &abort_flag);
+    __syncthreads();
+    if (threadIdx.x == 0 && abort_flag) atomicExch(err, (int)PE_ERR_DEVICE_TIMEOUT);
+}
+
 }  // namespace pe
