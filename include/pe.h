@@ -32,6 +32,9 @@
  *   - Dense row-major layouts only.  Device pointers must be 16-byte aligned.
  *   - No C++ exception crosses this interface.  A CUDA error maps to
  *     PE_ERR_CUDA.
+ *   - The forward calls, pe_set_weight and pe_patchify each open an NVTX
+ *     range named after the call (Nsight timelines; ncu --nvtx filters);
+ *     without a tool attached it costs nothing measurable.
  *   - Forward calls that use a handle's workspace must be serialised on one
  *     stream: grouped calls with more than PE_INLINE_ITEMS items (item table),
  *     frames calls on the staged or streamed path (see pe_forward_frames), and

@@ -5,6 +5,7 @@
 // pe_kernels.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -119,6 +120,16 @@ bool make_out_tmap(CUtensorMap *m, void *out, bool f32, int64_t N, int E) {
     return make_tmap(m, out, f32, (uint64_t)N, (uint64_t)E, (uint64_t)E, 32, 32,
                      f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
+
+// One NVTX range per public call, named after it: visible on Nsight timelines
+// and usable as an ncu filter (--nvtx --nvtx-include); without a tool attached
+// the push and pop return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -716,6 +727,7 @@ void pe_destroy(pe_handle *h) {
 
 pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *bias, pe_dtype b_dt,
                         pe_stream_t stream) {
+    NvtxRange nvtx("pe_set_weight");
     if (!h || !w) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(w_dt) || (bias && !valid_dtype(b_dt))) return PE_ERR_DTYPE;
     if ((bias != nullptr) != h->has_bias) return PE_ERR_INVALID_ARG;
@@ -922,11 +934,13 @@ extern "C" {
 
 pe_status pe_forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, void *out,
                              pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_patches");
     return forward_patches(h, x, x_dt, N, nullptr, PE_BF16, out, out_dt, stream);
 }
 
 pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N, const void *pos,
                                  pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_patches_pos");
     if (N > 0) {
         const pe_status s = check_pos(pos, pos_dt);
         if (s != PE_OK) return s;
@@ -937,12 +951,14 @@ pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int
 pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
                                     const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
                                     pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_frames_grouped");
     return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, nullptr, PE_BF16, out, out_dt, stream);
 }
 
 pe_status pe_forward_frames_grouped_pos(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
                                         const int32_t *THW, const int32_t *grid_thw, int merge, const void *pos,
                                         pe_dtype pos_dt, void *out, pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_frames_grouped_pos");
     const pe_status s = check_pos(pos, pos_dt);
     if (s != PE_OK) return s;
     return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, pos, pos_dt, out, out_dt, stream);
@@ -958,6 +974,7 @@ pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int
 
 pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt, const int32_t *THW,
                       const int32_t *grid_thw, int merge, void *rows, pe_dtype rows_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_patchify");
     if (!h) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(rows_dt)) return PE_ERR_DTYPE;
     DeviceGuard g(h->dev);
@@ -1008,6 +1025,7 @@ cudaError_t noalloc_table(int dev, ItemDesc **out) {
 pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
                                             const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
                                             pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_frames_grouped_noalloc");
     if (!h || n < 1 || !frames || !THW || !grid_thw || !out) return PE_ERR_INVALID_ARG;
     if (n > PE_NOALLOC_MAX_ITEMS) return PE_ERR_UNSUPPORTED;
     if (!valid_dtype(f_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
@@ -1210,6 +1228,7 @@ extern "C" {
 pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const *frames_host, pe_dtype f_dt,
                                          const int32_t *THW, const int32_t *grid_thw, int merge, void *out_host,
                                          pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_frames_grouped_host");
     if (!h || n < 1 || !frames_host || !THW || !grid_thw || !out_host) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(f_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (merge != 1 && merge != 2) return PE_ERR_INVALID_ARG;
@@ -1275,6 +1294,7 @@ pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const 
 
 pe_status pe_forward_patches_host(pe_handle *h, const void *x_host, pe_dtype x_dt, int64_t N, void *out_host,
                                   pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_patches_host");
     if (!h || N < 0) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(x_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (!h->weight_set) return PE_ERR_NO_WEIGHT;
@@ -1459,6 +1479,7 @@ pe_status pe_merger_set_weights(pe_merger *pm, const void *gamma, const void *be
 }
 
 pe_status pe_merger_forward(pe_merger *pm, const void *x, int64_t N, void *out, pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_merger_forward");
     if (!pm || N < 0) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (!pm->weights_set) return PE_ERR_NO_WEIGHT;
