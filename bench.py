@@ -379,7 +379,9 @@ def run_ours(args, rank, world, local):
     value = weak_scaling_value(wl.N, args.steps, world, total_max_ms)
 
     # end to end through the public API with host buffers (pinned), per step:
-    # H2D of the step's frames, the forward, D2H of the embeddings
+    # H2D of the step's frames, the forward, D2H of the embeddings.  "serial":
+    # copy_ in, the device-pointer call, copy_ out, one stream; "host": the
+    # host-buffer call, which pipelines the copies and the contraction in chunks.
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
     if wl.patches is not None:
         host_in = [wl.patches.pin_memory()]
@@ -388,21 +390,28 @@ def run_ours(args, rank, world, local):
         host_in = [it.frames.pin_memory() for it in wl.items]
         dev_in = frames_dev
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(2):
+
+    def e2e_step():
+        if args.e2e == "host":
+            if wl.patches is not None:
+                pe.forward_patches_host(host_in[0], out=host_out, stream=stream, blocking=False)
+            else:
+                pe.forward_frames_grouped_host(host_in, grids, wl.merge, out=host_out, stream=stream,
+                                               blocking=False)
+            return
         for h_, d_ in zip(host_in, dev_in):
             d_.copy_(h_, non_blocking=True)
         step()
         host_out.copy_(out, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        e2e_step()
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     e0.record(stream)
     for _ in range(e2e_steps):
-        for h_, d_ in zip(host_in, dev_in):
-            d_.copy_(h_, non_blocking=True)
-        step()
-        host_out.copy_(out, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_value = weak_scaling_value(wl.N, e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), pg, dev))
@@ -462,7 +471,10 @@ def run_ours(args, rank, world, local):
                                         + (" x 1.1/2.25 (nominal tf32/bf16)" if tf32 else "")},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
-                    "d2h_bytes_per_step": out_bytes},
+                    "d2h_bytes_per_step": out_bytes,
+                    "path": ("host-buffer call: chunked copies in both directions pipelined with the contraction"
+                             if args.e2e == "host" else
+                             "serial: pinned copy_ in, the device-pointer call, copy_ out, one stream")},
             "gpu_launches": launches,
             "context": context,
             "clocks": clk.summary(),
@@ -576,6 +588,9 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e", default="serial", choices=["serial", "host"],
+                    help="how the end-to-end number moves host data: serial copies around the device-pointer "
+                         "call, or the library's pipelined host-buffer call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the cuBLAS context timing")
     ap.add_argument("--merger", action="store_true",
