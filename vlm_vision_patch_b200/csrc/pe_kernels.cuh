@@ -29,7 +29,8 @@
 //
 // Around it: the staged prepare kernel (pe_prep_rows_kernel), the fp32 casts
 // (pe_cast_rows_kernel, pe_round_tf32_kernel), the weight packers, the
-// patchify test hook and the PatchMerger's LayerNorm (pe_layernorm_kernel).
+// patchify test hook, the PatchMerger's LayerNorm (pe_layernorm_kernel) and
+// the failure self-test (pe_wait_timeout_probe_kernel).
 #pragma once
 
 #include <type_traits>
