@@ -2,11 +2,13 @@
 
 Each case plants one mistake in a copy of oracle/pe_oracle.c (on the CPU),
 builds it, and runs the pin suite against it in a child process; the suite has
-to fail.  The real oracle is never modified.
+to fail.  The real oracle is never modified.  The children run concurrently
+(one OpenMP thread each), once per module; each case then reads its result.
 """
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -72,16 +74,46 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
-    old, new = MUTANTS[name]
-    src = open(SRC).read()
-    assert src.count(old) >= 1, f"pattern for {name} not found in the oracle source"
-    mut = tmp_path / f"{name}.c"
-    mut.write_text(src.replace(old, new))
-    lib = oracle.compile_source(str(mut), str(tmp_path / f"lib{name}.so"))
-    env = dict(os.environ, PE_ORACLE_LIB=lib)
+CONTROL = "unmodified"   # the real source through the same build and run: must pass
+
+
+def _run_mutant(name, src, workdir):
+    if name == CONTROL:
+        text = src
+    else:
+        old, new = MUTANTS[name]
+        if src.count(old) < 1:
+            return None, f"pattern for {name} not found in the oracle source"
+        text = src.replace(old, new)
+    mut = os.path.join(workdir, f"{name}.c")
+    with open(mut, "w") as f:
+        f.write(text)
+    lib = oracle.compile_source(mut, os.path.join(workdir, f"lib{name}.so"))
+    env = dict(os.environ, PE_ORACLE_LIB=lib, OMP_NUM_THREADS="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    src = open(SRC).read()
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    names = [CONTROL] + sorted(MUTANTS)
+    with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
+        results = list(ex.map(lambda n: _run_mutant(n, src, workdir), names))
+    return dict(zip(names, results))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_results):
+    rc, out = mutant_results[name]
+    assert rc is not None, out
+    assert rc != 0, f"mutant {name} survived the pins:\n{out}"
+
+
+def test_unmodified_oracle_passes_the_same_run(mutant_results):
+    """The control: a failure above means a pin failed, not the harness."""
+    rc, out = mutant_results[CONTROL]
+    assert rc == 0, out
