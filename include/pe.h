@@ -31,7 +31,7 @@
  *     launched or written.
  *   - Dense row-major layouts only.  Device pointers must be 16-byte aligned.
  *   - No C++ exception crosses this interface.  A CUDA error maps to
- *     PE_ERR_CUDA.
+ *     PE_ERR_CUDA, a failed host allocation to PE_ERR_HOST_MEMORY.
  *   - The forward calls, pe_set_weight and pe_patchify each open an NVTX
  *     range named after the call (Nsight timelines; ncu --nvtx filters);
  *     without a tool attached it costs nothing measurable.
@@ -65,7 +65,8 @@ typedef enum {
     PE_ERR_NO_WEIGHT = 5,      /* forward called before pe_set_weight                  */
     PE_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed                    */
     PE_ERR_UNSUPPORTED = 7,    /* valid request outside what the kernels implement     */
-    PE_ERR_DEVICE_TIMEOUT = 8  /* a kernel gave up waiting on its pipeline (bounded wait) */
+    PE_ERR_DEVICE_TIMEOUT = 8, /* a kernel gave up waiting on its pipeline (bounded wait) */
+    PE_ERR_HOST_MEMORY = 9     /* a host allocation (item table, chunk plan) failed    */
 } pe_status;
 
 typedef enum { PE_F32 = 0, PE_BF16 = 1 } pe_dtype;

@@ -42,22 +42,31 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, f)
 
 
-def test_library_is_built_for_sm100a(lib):
-    from vlm_vision_patch_b200 import _binding
-    out = subprocess.run(["cuobjdump", "--list-elf", _binding.LIB_PATH], capture_output=True, text=True)
-    if out.returncode != 0:
-        pytest.skip("cuobjdump unavailable")
-    assert "sm_100a" in out.stdout
+def test_library_is_built_for_sm100a_only():
+    """One -gencode, compute_100a -> sm_100a: machine code for sm_100a and no
+    PTX that a JIT could take to another GPU."""
+    from vlm_vision_patch_b200 import build
+    flags = build.NVCC_FLAGS
+    assert flags.count("-gencode") == 1
+    assert flags[flags.index("-gencode") + 1] == "arch=compute_100a,code=sm_100a"
+
+
+def test_build_tracks_every_source():
+    """A change to any file the build reads makes the library stale."""
+    from vlm_vision_patch_b200 import build
+    csrc = [os.path.join(build.CSRC, f) for f in os.listdir(build.CSRC) if f.endswith((".cu", ".cuh", ".h"))]
+    assert set(csrc) | {os.path.join(ROOT, "include", "pe.h")} <= set(build.DEPS)
 
 
 def test_status_strings(lib):
     from vlm_vision_patch_b200 import _binding
     seen = set()
-    for code in range(9):
+    for code in range(10):
         s = _binding.status_string(code)
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 9
+    assert len(seen) == 10
+    assert set(_binding.STATUS) == set(range(10))
     assert _binding.status_string(99) == "unknown status"
 
 

@@ -18,7 +18,7 @@ PE_F32, PE_BF16 = 0, 1
 STATUS = {
     0: "PE_OK", 1: "PE_ERR_INVALID_ARG", 2: "PE_ERR_SHAPE", 3: "PE_ERR_DTYPE",
     4: "PE_ERR_ALIGN", 5: "PE_ERR_NO_WEIGHT", 6: "PE_ERR_CUDA", 7: "PE_ERR_UNSUPPORTED",
-    8: "PE_ERR_DEVICE_TIMEOUT",
+    8: "PE_ERR_DEVICE_TIMEOUT", 9: "PE_ERR_HOST_MEMORY",
 }
 PE_INLINE_ITEMS = 16
 PE_MAX_PATCH = 32

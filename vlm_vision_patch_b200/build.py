@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpe.so")
 SOURCES = [os.path.join(CSRC, "pe_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pe_kernels.cuh", "pe_device.cuh")] + \
+# every file the build reads: a change to any of them makes the library stale
+DEPS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))) + \
     [os.path.join(os.path.dirname(HERE), "include", "pe.h")]
 
 NVCC_FLAGS = [

@@ -131,6 +131,20 @@ struct NvtxRange {
     NvtxRange &operator=(const NvtxRange &) = delete;
 };
 
+// Runs an entry point's body so that no C++ exception crosses the C ABI: a
+// failed host allocation (the item tables and chunk plans are std::vectors)
+// returns PE_ERR_HOST_MEMORY, anything else PE_ERR_CUDA.
+template <class F>
+pe_status no_throw(F &&body) {
+    try {
+        return body();
+    } catch (const std::bad_alloc &) {
+        return PE_ERR_HOST_MEMORY;
+    } catch (...) {
+        return PE_ERR_CUDA;
+    }
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_dtype(int d) { return d == PE_F32 || d == PE_BF16; }
@@ -624,6 +638,7 @@ const char *pe_status_string(pe_status s) {
         case PE_ERR_CUDA: return "CUDA error";
         case PE_ERR_UNSUPPORTED: return "unsupported configuration";
         case PE_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+        case PE_ERR_HOST_MEMORY: return "host memory allocation failed";
     }
     return "unknown status";
 }
@@ -952,7 +967,9 @@ pe_status pe_forward_frames_grouped(pe_handle *h, int n, const void *const *fram
                                     const int32_t *THW, const int32_t *grid_thw, int merge, void *out,
                                     pe_dtype out_dt, pe_stream_t stream) {
     NvtxRange nvtx("pe_forward_frames_grouped");
-    return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, nullptr, PE_BF16, out, out_dt, stream);
+    return no_throw([&] {
+        return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, nullptr, PE_BF16, out, out_dt, stream);
+    });
 }
 
 pe_status pe_forward_frames_grouped_pos(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
@@ -961,7 +978,9 @@ pe_status pe_forward_frames_grouped_pos(pe_handle *h, int n, const void *const *
     NvtxRange nvtx("pe_forward_frames_grouped_pos");
     const pe_status s = check_pos(pos, pos_dt);
     if (s != PE_OK) return s;
-    return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, pos, pos_dt, out, out_dt, stream);
+    return no_throw([&] {
+        return forward_frames_grouped(h, n, frames, f_dt, THW, grid_thw, merge, pos, pos_dt, out, out_dt, stream);
+    });
 }
 
 pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H, int W,
@@ -980,7 +999,7 @@ pe_status pe_patchify(pe_handle *h, int n, const void *const *frames, pe_dtype f
     DeviceGuard g(h->dev);
     FwdParams P;
     cudaStream_t st = (cudaStream_t)stream;
-    const pe_status s = setup_frames(h, n, frames, f_dt, THW, grid_thw, merge, rows, P, st);
+    const pe_status s = no_throw([&] { return setup_frames(h, n, frames, f_dt, THW, grid_thw, merge, rows, P, st); });
     if (s != PE_OK) return s;
     if (P.N == 0) return PE_OK;
     const int64_t total = P.N * (h->K / 2);
@@ -1081,7 +1100,14 @@ pe_status pe_profile_begin(pe_handle *h, int max_calls) {
     if (!h || max_calls < 0 || max_calls > 1000000) return PE_ERR_INVALID_ARG;
     DeviceGuard g(h->dev);
     for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
-    h->prof_ev.assign((size_t)2 * max_calls, nullptr);
+    h->prof_ev.clear();
+    h->prof_cap = h->prof_n = 0;
+    h->prof_on = false;
+    try {
+        h->prof_ev.assign((size_t)2 * max_calls, nullptr);
+    } catch (const std::bad_alloc &) {
+        return PE_ERR_HOST_MEMORY;
+    }
     for (auto &e : h->prof_ev)
         if (cudaEventCreate(&e) != cudaSuccess) return PE_ERR_CUDA;
     h->prof_cap = max_calls;
@@ -1225,10 +1251,11 @@ alignas(16) const unsigned char kStandIn[16] = {};   // validation stand-in for 
 
 extern "C" {
 
-pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const *frames_host, pe_dtype f_dt,
-                                         const int32_t *THW, const int32_t *grid_thw, int merge, void *out_host,
-                                         pe_dtype out_dt, pe_stream_t stream) {
-    NvtxRange nvtx("pe_forward_frames_grouped_host");
+// Body of pe_forward_frames_grouped_host (internal linkage; the exported
+// call runs it under no_throw).
+static pe_status frames_grouped_host_body(pe_handle *h, int n, const void *const *frames_host, pe_dtype f_dt,
+                                          const int32_t *THW, const int32_t *grid_thw, int merge, void *out_host,
+                                          pe_dtype out_dt, pe_stream_t stream) {
     if (!h || n < 1 || !frames_host || !THW || !grid_thw || !out_host) return PE_ERR_INVALID_ARG;
     if (!valid_dtype(f_dt) || !valid_dtype(out_dt)) return PE_ERR_DTYPE;
     if (merge != 1 && merge != 2) return PE_ERR_INVALID_ARG;
@@ -1290,6 +1317,15 @@ pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const 
                    : PE_ERR_CUDA;
     };
     return run_host_pipeline(h, (int)pl.chunks.size(), st, copy_in, compute, copy_out);
+}
+
+pe_status pe_forward_frames_grouped_host(pe_handle *h, int n, const void *const *frames_host, pe_dtype f_dt,
+                                         const int32_t *THW, const int32_t *grid_thw, int merge, void *out_host,
+                                         pe_dtype out_dt, pe_stream_t stream) {
+    NvtxRange nvtx("pe_forward_frames_grouped_host");
+    return no_throw([&] {
+        return frames_grouped_host_body(h, n, frames_host, f_dt, THW, grid_thw, merge, out_host, out_dt, stream);
+    });
 }
 
 pe_status pe_forward_patches_host(pe_handle *h, const void *x_host, pe_dtype x_dt, int64_t N, void *out_host,
