@@ -592,7 +592,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="grouped_16_images", choices=sorted(workloads.ALL))
-    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--cpu-rows", type=int, default=65536,
+                    help="output rows in the CPU oracle's timed sample (capped at the workload's N): about "
+                         "10-30 s on the host cores")
     ap.add_argument("--ref-rows", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--e2e", default="serial", choices=["serial", "host"],
