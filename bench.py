@@ -447,7 +447,7 @@ def run_ours(args, rank, world, local):
         if world == 1 and not args.no_cpu_baseline:
             r, dt, th = oracle_sample_rate(wl, args.cpu_rows, 7)
             cpu = {"value": r, "unit": UNIT, "cores": th, "kind": "oracle",
-                   "sample": f"{args.cpu_rows} seeded random output rows of {wl.name} (of {wl.N}), "
+                   "sample": f"{min(args.cpu_rows, wl.N)} seeded random output rows of {wl.name} (of {wl.N}), "
                              f"{dt:.1f} s; direct fp64 Conv3d, OpenMP over rows"}
         traffic = measured_traffic(wl.name, "staged" if staged else "single")
         context = None if (args.no_context or world > 1) else library_context(wl, dev, flush_buf)
