@@ -255,7 +255,7 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(wl, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{rows_per_step} seeded random output rows of {wl.name} per step "
+                         "sample": f"{min(rows_per_step, wl.N)} seeded random output rows of {wl.name} per step "
                                    f"(of {wl.N}); direct fp64 Conv3d, OpenMP over rows"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
