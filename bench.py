@@ -493,6 +493,65 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def merger_weights(E: int, H: int, seed: int = 77):
+    """Synthetic PatchMerger weights on the CPU (bf16), for m = 2, D = 4E:
+    gamma ~ 1 + N(0, 0.1), beta ~ N(0, 0.05), w1 [D, D] and w2 [H, D] ~ N(0, 1/D),
+    b1, b2 ~ N(0, 0.02).  Returns (gamma, beta, w1, b1, w2, b2)."""
+    D = 4 * E
+    gen = torch.Generator().manual_seed(seed)
+    mk = lambda *shape, std: (torch.randn(*shape, generator=gen) * std).to(torch.bfloat16)  # noqa: E731
+    gamma = (1.0 + torch.randn(E, generator=gen) * 0.1).to(torch.bfloat16)
+    beta, b1, b2 = mk(E, std=0.05), mk(D, std=0.02), mk(H, std=0.02)
+    w1, w2 = mk(D, D, std=D ** -0.5), mk(H, D, std=D ** -0.5)
+    return gamma, beta, w1, b1, w2, b2
+
+
+MERGER_METRIC = "PatchMerger patches/s and TFLOP/s (% of B200 dense bf16 peak), 1 GPU"
+
+
+def run_reference_merger(args, rank, world):
+    """--impl reference --merger: the CPU PatchMerger oracle on sampled merged
+    rows of an input shaped like the workload's PatchEmbed output (seeded
+    N(0, 0.5) rows; the values do not change the work), the merger arm's
+    weights, metric and unit."""
+    import oracle
+    if rank != 0:
+        return 0
+    wl = workloads.ALL[args.workload]()
+    E, H = wl.E, 1536
+    V = wl.N // 4
+    x = (torch.randn(V * 4, E, generator=torch.Generator().manual_seed(78)) * 0.5).to(torch.bfloat16)
+    gamma, beta, w1, b1, w2, b2 = merger_weights(E, H)
+    per_step = max(1, min(args.ref_rows // 4, V))
+
+    def sample(n, seed):
+        rng = np.random.default_rng(seed)
+        mask = np.zeros(V, np.uint8)
+        mask[rng.choice(V, size=min(n, V), replace=False)] = 1
+        t0 = time.perf_counter()
+        oracle.patch_merger(x, 4, gamma, beta, 1e-6, w1, b1, w2, b2, v_mask=mask)
+        return time.perf_counter() - t0
+    for _ in range(args.warmup):
+        sample(max(1, per_step // 8), 3000)
+    times = [sample(per_step, 4000 + s) for s in range(args.steps)]
+    total = sum(times)
+    value = 4 * per_step * args.steps / total
+    threads = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": MERGER_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(config_of(wl, world), merger="LayerNorm, 2x2 concat, GELU MLP "
+                                            f"{4 * E} -> {4 * E} -> {H}", merged_rows=V),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{per_step} seeded random merged rows ({4 * per_step} patch rows) of {V} per "
+                                   "step; fp64 LayerNorm and MLP with bf16 roundings, OpenMP over rows"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_merger(args, rank, world, local):
     """--merger: the PatchMerger (LayerNorm, 2x2 concat, GELU MLP 5120 -> 5120 ->
     1536, synthetic N(0, 1/sqrt(D)) weights) on the workload's PatchEmbed output
@@ -520,11 +579,7 @@ def run_merger(args, rank, world, local):
     E, D = wl.E, wl.E * 4
     V = x.shape[0] // 4
     x = x[: V * 4]
-    gen = torch.Generator().manual_seed(77)
-    mk = lambda *shape, std: (torch.randn(*shape, generator=gen) * std).to(torch.bfloat16).to(dev)
-    gamma = (1.0 + torch.randn(E, generator=gen) * 0.1).to(torch.bfloat16).to(dev)
-    beta, b1, b2 = mk(E, std=0.05), mk(D, std=0.02), mk(H, std=0.02)
-    w1, w2 = mk(D, D, std=D ** -0.5), mk(H, D, std=D ** -0.5)
+    gamma, beta, w1, b1, w2, b2 = (t.to(dev) for t in merger_weights(E, H))
     pm = vp.PatchMerger(E, m, H, 1e-6)
     pm.set_weights(gamma, beta, w1, b1, w2, b2)
     out = torch.empty((V, H), dtype=torch.bfloat16, device=dev)
@@ -563,7 +618,7 @@ def run_merger(args, rank, world, local):
         fc1_ms = statistics.mean(fc1)
         achieved = 2.0 * V * D * D / (fc1_ms / 1e3) / 1e12
         print(json.dumps({
-            "metric": "PatchMerger patches/s and TFLOP/s (% of B200 dense bf16 peak), 1 GPU", "value": value,
+            "metric": MERGER_METRIC, "value": value,
             "unit": "patches/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (PatchEmbed output of the workload, "
@@ -614,7 +669,7 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     rank, world, local = dist_env()
     if args.impl == "reference":
-        return run_reference(args, rank, world)
+        return run_reference_merger(args, rank, world) if args.merger else run_reference(args, rank, world)
     if args.merger:
         return run_merger(args, rank, world, local)
     return run_ours(args, rank, world, local)

@@ -10,6 +10,7 @@ import socket
 import sys
 
 import pytest
+import torch
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -110,3 +111,21 @@ def test_clock_sampler_finds_the_cuda_device_among_all_gpus():
     assert bench.nvml_handle_for(nv, _props(0, 0x52, 0)) == (2, "pci")
     assert bench.nvml_handle_for(nv, _props(0, 0x99, 0, "cccc")) == (2, "uuid")
     assert bench.nvml_handle_for(nv, _props(0, 0x99, 0)) == (None, None)
+
+
+def test_reference_arm_for_the_merger():
+    """--impl reference --merger times the CPU PatchMerger oracle with the merger
+    arm's metric and unit."""
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        assert bench.main(["--impl", "reference", "--merger", "--workload", "image_224x896", "--ref-rows", "8",
+                           "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(buf.getvalue().strip())
+    assert line["impl"] == "reference" and line["metric"] == bench.MERGER_METRIC and line["unit"] == "patches/s"
+    assert line["value"] > 0 and line["config"]["merged_rows"] == 256
+
+
+def test_merger_weights_are_seeded():
+    a, b = bench.merger_weights(64, 32), bench.merger_weights(64, 32)
+    assert [t.shape for t in a] == [(64,), (64,), (256, 256), (256,), (32, 256), (32,)]
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
