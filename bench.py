@@ -216,9 +216,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle arm
 
-def oracle_sample_rate(wl, n_rows: int, seed: int):
-    """Time the CPU oracle on n_rows sampled output rows of the workload.
-    Returns (rows/s, seconds, threads)."""
+def oracle_sample_rate(wl, n_rows: int, seed: int, fp32_form: bool = False):
+    """Time the CPU oracle on n_rows sampled output rows of the workload
+    (fp32_form: the unrounded fp32 Conv3d that the tf32 path is checked
+    against, for fp32 patch rows).  Returns (rows/s, seconds, threads)."""
     import oracle
     rng = np.random.default_rng(seed)
     rows = rng.choice(wl.N, size=min(n_rows, wl.N), replace=False)
@@ -226,7 +227,8 @@ def oracle_sample_rate(wl, n_rows: int, seed: int):
     mask[rows] = 1
     t0 = time.perf_counter()
     if wl.patches is not None:
-        oracle.conv3d_patches(wl.patches, wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
+        form = oracle.conv3d_patches_fp32 if fp32_form else oracle.conv3d_patches
+        form(wl.patches, wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
     else:
         oracle.conv3d_grouped([(it.frames, it.grid) for it in wl.items], wl.merge, wl.mean, wl.std,
                               wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
@@ -239,12 +241,13 @@ def run_reference(args, rank, world):
         return 0
     wl = workloads.ALL[args.workload]()
     rows_per_step = args.ref_rows
+    fp32_form = bool(args.tf32 and wl.patches is not None and wl.patches.dtype == torch.float32)
     for _ in range(args.warmup):
-        oracle_sample_rate(wl, max(16, rows_per_step // 8), 1000)
+        oracle_sample_rate(wl, max(16, rows_per_step // 8), 1000, fp32_form)
     times, nrows = [], 0
     threads = 1
     for s in range(args.steps):
-        r, dt, threads = oracle_sample_rate(wl, rows_per_step, 2000 + s)
+        r, dt, threads = oracle_sample_rate(wl, rows_per_step, 2000 + s, fp32_form)
         times.append(dt)
         nrows += int(round(r * dt))
     total = sum(times)
@@ -256,7 +259,9 @@ def run_reference(args, rank, world):
         "data": "synthetic", "config": config_of(wl, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{min(rows_per_step, wl.N)} seeded random output rows of {wl.name} per step "
-                                   f"(of {wl.N}); direct fp64 Conv3d, OpenMP over rows"},
+                                   f"(of {wl.N}); direct fp64 Conv3d"
+                                   + (" on the unrounded fp32 inputs (the tf32 path's reference)" if fp32_form else "")
+                                   + ", OpenMP over rows"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

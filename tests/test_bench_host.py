@@ -129,3 +129,12 @@ def test_merger_weights_are_seeded():
     a, b = bench.merger_weights(64, 32), bench.merger_weights(64, 32)
     assert [t.shape for t in a] == [(64,), (64,), (256, 256), (256,), (32, 256), (32,)]
     assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+def test_reference_arm_for_tf32_times_the_fp32_form():
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        assert bench.main(["--impl", "reference", "--tf32", "--workload", "patches_fp32_1024", "--ref-rows", "8",
+                           "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(buf.getvalue().strip())
+    assert line["value"] > 0 and "unrounded fp32" in line["cpu_baseline"]["sample"]
