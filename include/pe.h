@@ -194,21 +194,32 @@ pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int
  *              README §3.2 PatchMerger and §4.1; Qwen2.5VL语言模型 MRoPE example:
  *              merged grid row-major, h outer).  gh and gw must be multiples of m.
  *   out      : dev [gt*gh*gw, E] of dtype out_dt.
- * Requires p even and p <= PE_MAX_PATCH.  Three execution paths, all within
- * the same tolerance of the exact result:
- *   fused    one kernel; the normalised [N, K] patch matrix only ever exists
- *            tile by tile in shared memory (fp32 frames, tp != 2, p not in
- *            {14, 16}, and the allocation-free call);
- *   staged   (default for bf16 frames with tp = 2 and p in {14, 16}) a prepare
- *            kernel writes the normalised rows once into the handle's
+ * Requires p even and p <= PE_MAX_PATCH.  Execution paths, all within the
+ * same tolerance of the exact result:
+ *   resident A  (default when every item is a single frame, bf16 frames,
+ *            tp = 2 and the C*p*p-column A block fits in shared memory beside
+ *            the weight ring: C = 3 with p <= 14) one kernel; each 256-row
+ *            block's normalised patches are gathered from the frames once into
+ *            shared memory, in merge order, and every weight tile streams past
+ *            them; both temporal slices of the weight meet the one frame.  No
+ *            workspace; the [N, K] patch matrix never exists in memory;
+ *   fused    one kernel that gathers each A tile again for every weight tile
+ *            (fp32 frames, tp != 2, p not in {14, 16} with video items, and
+ *            the allocation-free call's video groups);
+ *   staged   (default for other bf16 frames with tp = 2 and p in {14, 16}) a
+ *            prepare kernel writes the normalised rows once into the handle's
  *            grow-only workspace, then the TMA-fed contraction reads them back;
  *   streamed one cooperative kernel: producer warps write the same rows while
  *            the contraction consumes the completed row blocks (an option:
  *            slower than staged on B200).
- * When every item is a single frame, the streamed and staged paths store one
- * temporal slice per row and multiply it by both temporal slices of the
- * weight.  The environment variable PE_FRAMES_PATH=fused|streamed|staged
- * overrides the choice.
+ * The resident-A path issues, row by row, the same MMAs in the same order as
+ * the staged path on single images, so the two give identical bits.  The
+ * environment variable PE_FRAMES_PATH=fused|streamed|staged selects another
+ * path instead of the default.  PE_TEST_WAIT_NS=n (a test hook) gives the
+ * resident-A kernel's pipeline waits a limit of n ns instead of 2 s, so that a
+ * test can make them run out and exercise the kernel's unwinding: the call
+ * then leaves an incomplete output and pe_last_error reports
+ * PE_ERR_DEVICE_TIMEOUT.
  * Errors: as pe_forward_patches plus PE_ERR_SHAPE, PE_ERR_UNSUPPORTED.
  */
 pe_status pe_forward_frames(pe_handle *h, const void *frames, pe_dtype f_dt, int T, int H,
@@ -263,11 +274,16 @@ pe_status pe_forward_frames_grouped_pos(pe_handle *h, int n, const void *const *
  *
  * Arguments, layouts and results are those of pe_forward_frames_grouped.
  * n > PE_NOALLOC_MAX_ITEMS returns PE_ERR_UNSUPPORTED before anything runs.
+ * With more than PE_INLINE_ITEMS items the descriptors are written into the
+ * table by small kernels on `stream` whose launch parameters carry them (up to
+ * 64 per launch), so no host staging buffer is used and the host never waits.
  * The first call on a device (with more than PE_INLINE_ITEMS items) looks up
  * the table's device address; make that first call before any stream capture.
  * All calls share the one table and it keeps the last call's contents, so calls
  * that can overlap on the GPU (different streams) race; calls on one stream
- * are ordered and safe.
+ * are ordered and safe.  Groups of single images take the one-launch
+ * resident-A kernel, which needs no workspace; other groups take the fused
+ * kernel (never the staged path, whose row buffer is allocated on first use).
  */
 pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *const *frames, pe_dtype f_dt,
                                             const int32_t *THW, const int32_t *grid_thw, int merge,
@@ -340,15 +356,16 @@ int64_t pe_num_patches(const int32_t *grid_thw, int n);
 
 /*
  * pe_profile_begin / pe_profile_end -- device time of each forward call's
- * contraction kernel (the fused kernel, or the GEMM that follows the prepare
- * or cast kernel), recorded with a CUDA event pair on the call's stream
+ * contraction kernel (the resident-A or fused kernel, or the GEMM that follows
+ * the prepare or cast kernel), recorded with a CUDA event pair on the call's stream
  * around that launch.  pe_profile_begin creates event pairs for up to
  * max_calls calls (0..1e6; 0 records no events and only counts launches) and
  * starts recording; pe_profile_end waits for the recorded events, writes the
  * elapsed milliseconds of the first min(*n, recorded) calls to host ms[] and
  * that count to *n, writes to *launches (if not NULL) how many kernels the
  * forward calls launched in the window (two per call on the staged frames
- * path and for fp32 patch rows, one otherwise), then frees the events and
+ * path and for fp32 patch rows, one otherwise, plus the item-table fills of
+ * the allocation-free call), then frees the events and
  * stops recording.  Profiling is a measurement aid: it allocates events and must not
  * overlap another profiling window on the same handle.  An event recorded
  * between two kernels of one call serialises them, so a window with events

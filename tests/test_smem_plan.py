@@ -10,7 +10,11 @@ the mode accepts, and for a range of N:
     either ring's depth;
   - the epilogue staging area sits past the rings and inside the allocation;
   - the grid is whole CTA pairs, at most one CTA per SM and no more pairs than
-    tiles; the tile width is 64, 128 or 256 and covers E."""
+    tiles; the tile width is 64, 128 or 256 and covers E;
+  - the resident-A kernel's plan, for every (C, p) with tp = 2: it declines
+    when A does not fit and must fit for C = 3, p = 14; otherwise the weight
+    ring, the resident A, the staging boxes and the barriers lie in order
+    inside the allocation, and the chunk and weight-stage counts cover K."""
 from __future__ import annotations
 
 import os
@@ -58,6 +62,47 @@ int main() {
                     if ((size_t)P.epi_offset + 4 * 8192 + 1024 > total) fail("epilogue area", mode, C, tp, p, 0);
                 }
             }
+    /* resident-A kernel: every (C, p) with tp = 2 and even p; the plan either
+       declines (A too large) or fits with its regions in order and in bounds */
+    for (int C = 1; C <= 4; ++C)
+        for (int p = 2; p <= 32; p += 2) {
+            const int K = C * 2 * p * p;
+            if (K > 8192) continue;
+            h.E = 1280; h.C = C; h.tp = 2; h.p = p; h.K = K;
+            h.Kpad = (K + 63) / 64 * 64;
+            h.Kh = (C * p * p + 15) / 16 * 16;
+            h.Kw = 64 * ((h.Kh + 31) / 32);
+            for (int bn : {64, 128, 256})
+                for (int of : {0, 1}) {
+                    FwdParams P;
+                    fill_common(&h, P);
+                    P.bn = bn;
+                    P.out_f32 = of;
+                    const size_t total = plan_astat(&h, P);
+                    ++cases;
+                    if (total == 0) {
+                        if (C == 3 && p == 14) fail("resident A must fit C=3 p=14", 100, C, 2, p, bn);
+                        continue;
+                    }
+                    const size_t box = of ? 4096 : 2048;
+                    const size_t bars = (size_t)(2 * P.nb + 2 * P.n_achunks + 5) * 8 + (size_t)(2 * P.nb + 2) * 4;
+                    if (total > (size_t)h.smem_optin) fail("astat shared memory", 100, C, 2, p, bn);
+                    if (P.nb < 2 || P.n_iss < 1 || P.n_iss > P.nb || P.n_iss > 3) fail("astat ring", 100, C, 2, p, bn);
+                    if (P.epi_bufs < 1 || P.epi_bufs > 2) fail("astat staging", 100, C, 2, p, bn);
+                    if (P.b_slot_bytes != bn / 2 * 128) fail("astat slot", 100, C, 2, p, bn);
+                    if ((size_t)P.a_offset < (size_t)P.nb * P.b_slot_bytes || P.a_offset %% 1024) fail("astat A offset", 100, C, 2, p, bn);
+                    if ((size_t)P.epi_offset < (size_t)P.a_offset + (size_t)(h.Kh / 8) * 2048 || P.epi_offset %% 1024)
+                        fail("astat staging offset", 100, C, 2, p, bn);
+                    if ((size_t)P.bar_offset < (size_t)P.epi_offset + 4 * P.epi_bufs * box || P.bar_offset %% 8)
+                        fail("astat barrier offset", 100, C, 2, p, bn);
+                    if ((size_t)P.bar_offset + bars + 1024 > total) fail("astat barriers in bounds", 100, C, 2, p, bn);
+                    if (P.num_ksteps * 16 != h.Kh || P.n_achunks * kAsChunkKs < P.num_ksteps ||
+                        (P.n_achunks - 1) * kAsChunkKs >= P.num_ksteps || P.n_achunks > kAsMaxChunks)
+                        fail("astat chunks", 100, C, 2, p, bn);
+                    if (64 * P.n_b_stages != h.Kw || 2 * P.n_b_stages < P.num_ksteps || P.cpp != C * p * p)
+                        fail("astat weight stages", 100, C, 2, p, bn);
+                }
+        }
     for (int E : {16, 40, 200, 1152, 1280, 5120})
         for (long long N : {1LL, 129LL, 1024LL, 18944LL, 59204LL, 131072LL, 3000000LL}) {
             h.E = E;

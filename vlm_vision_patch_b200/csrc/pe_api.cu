@@ -19,6 +19,7 @@
 #include "../../include/pe.h"
 #include "pe_host_plan.h"
 #include "pe_kernels.cuh"
+#include "pe_astat.cuh"
 
 using namespace pe;
 
@@ -32,6 +33,8 @@ struct pe_handle {
     uint16_t *wpack_f = nullptr; // dev [E, Kpad] bf16, k order of the frames producer
     uint16_t *wpack_t = nullptr; // dev [E, 2*Kh] bf16, slice-major (tp == 2 only)
     uint16_t *wpack_fold = nullptr; // dev [E, Kh] bf16, both slices summed (tp == 2 only)
+    uint16_t *wpack_i = nullptr; // dev [E, Kw] bf16, slice-interleaved 64-column tiles (tp == 2 only)
+    int Kw = 0;                 // 64 * ceil(Kh / 32)
     bool fold = false;          // pe_set_temporal_fold
     uint32_t *wpack32 = nullptr; // dev [E, Kp32] fp32 words, tf32-rounded, view order
     int Kp32 = 0;               // K rounded up to 32
@@ -44,6 +47,7 @@ struct pe_handle {
     CUtensorMap tmap_wf[3];     // same for the frames-order weight
     CUtensorMap tmap_wt[3];     // same for the slice-major weight
     CUtensorMap tmap_wfold[3];  // same for the folded weight
+    CUtensorMap tmap_wi[3];     // same for the slice-interleaved weight
     CUtensorMap tmap_w32[3];    // same for the tf32 weight (32 fp32 columns per box)
     int num_sms = 0;
     int smem_optin = 0;
@@ -567,6 +571,99 @@ pe_status run_frames_streamed(pe_handle *h, FwdParams &P, void *out, bool all_sc
     return finish(e);
 }
 
+int env_int(const char *name, int dflt) {
+    const char *s = std::getenv(name);
+    return s ? std::atoi(s) : dflt;
+}
+
+// Resident-A kernel (pe_astat_kernel): weight ring depth, staging boxes and
+// shared-memory offsets.  Returns the dynamic shared memory size, or 0 when
+// the resident A does not fit beside a ring of two weight stages.
+// PE_ASTAT_NB / PE_ASTAT_EPIBUFS pin the ring depth / staging boxes.
+size_t plan_astat(const pe_handle *h, FwdParams &P) {
+    if (P.Kh % 16 != 0 || P.Kh > 16 * kAsChunkKs * kAsMaxChunks) return 0;
+    P.num_ksteps = P.Kh / 16;
+    P.n_achunks = (P.num_ksteps + kAsChunkKs - 1) / kAsChunkKs;
+    P.cpp = P.C * P.P * P.P;
+    P.n_b_stages = (P.Kh + 31) / 32;           // slice-interleaved tiles: two k-steps of both slices each
+    P.b_slot_bytes = (P.bn / 2) * 128;          // this CTA's half of one 64-column tile
+    P.ksub = 1;
+    const size_t a_bytes = (size_t)(P.Kh / 8) * 2048;
+    const size_t box = P.out_f32 ? 4096 : 2048;
+    auto up = [](size_t v) { return (v + 1023) / 1024 * 1024; };
+    auto bars = [&](int nb) { return (size_t)(2 * nb + 2 * P.n_achunks + 5) * 8 + (size_t)(2 * nb + 2) * 4; };
+    auto total = [&](int nb, int bufs) {
+        return 1024 + up((size_t)nb * P.b_slot_bytes) + up(a_bytes) + 4 * (size_t)bufs * box + bars(nb);
+    };
+    const int nb_pin = env_int("PE_ASTAT_NB", 0), bufs_pin = env_int("PE_ASTAT_EPIBUFS", 0);
+    for (int nb = 8; nb >= 2; --nb) {
+        if (nb_pin && nb != nb_pin) continue;
+        for (int bufs = 2; bufs >= 1; --bufs) {
+            if (bufs_pin && bufs != bufs_pin) continue;
+            const size_t t = total(nb, bufs);
+            if (t > (size_t)h->smem_optin) continue;
+            P.nb = nb;
+            P.na = 0;
+            P.epi_bufs = bufs;
+            P.n_iss = std::min(3, nb);
+            P.a_offset = (int)up((size_t)nb * P.b_slot_bytes);
+            P.epi_offset = P.a_offset + (int)up(a_bytes);
+            P.bar_offset = P.epi_offset + 4 * bufs * (int)box;
+            return t;
+        }
+    }
+    return 0;
+}
+
+// Single images (every item T = 1), tp = 2, bf16 frames: the resident-A kernel
+// applies when the handle has the slice-interleaved weight and A fits.
+bool astat_eligible(const pe_handle *h, const FwdParams &P, int f_dt) {
+    return f_dt == PE_BF16 && h->tp == 2 && P.all_t1 && h->wpack_i && (h->p & 1) == 0;
+}
+
+template <int PT, int NORM>
+cudaError_t launch_astat(const CUtensorMap &tw, const CUtensorMap &to, const FwdParams &P, size_t smem, int grid,
+                         cudaStream_t st) {
+    auto kern = pe_astat_kernel<PT, NORM>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    pe_handle *h = t_prof_handle;
+    const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
+    if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
+    kern<<<grid, kAsThreads, smem, st>>>(tw, to, P);
+    e = cudaGetLastError();
+    if (prof) {
+        cudaEventRecord(h->prof_ev[2 * h->prof_n + 1], st);
+        ++h->prof_n;
+    }
+    if (h && h->prof_on) ++h->prof_launches;
+    return e;
+}
+
+// One launch from raw frames to embeddings; allocates nothing.  Returns
+// PE_ERR_UNSUPPORTED (nothing launched) when the resident A does not fit.
+pe_status run_frames_astat(pe_handle *h, FwdParams &P, void *out, cudaStream_t st) {
+    int grid = 0;
+    bool ok = true;
+    plan_tiles(h, P, P.N, grid, ok);
+    if (!ok) return PE_ERR_UNSUPPORTED;
+    const size_t smem = plan_astat(h, P);
+    if (smem == 0) return PE_ERR_UNSUPPORTED;
+    const uint64_t wl = (uint64_t)env_int("PE_TEST_WAIT_NS", 0);
+    P.wait_ns = wl;
+    CUtensorMap to;
+    if (!make_out_tmap(&to, out, P.out_f32, P.N, P.E)) return PE_ERR_CUDA;
+    const CUtensorMap &tw = h->tmap_wi[bn_index(P.bn)];
+    bool all_scaled = true;
+    for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
+    cudaError_t e;
+    if (h->p == 14)
+        e = all_scaled ? launch_astat<14, 1>(tw, to, P, smem, grid, st) : launch_astat<14, 2>(tw, to, P, smem, grid, st);
+    else
+        e = launch_astat<0, 2>(tw, to, P, smem, grid, st);
+    return finish(e);
+}
+
 pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt, cudaStream_t st,
                      bool allow_staged = true) {
     P.out_f32 = out_dt == PE_F32;
@@ -577,6 +674,16 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
         bool all_scaled = true;
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
         return run_frames_staged(h, P, out, all_scaled, true, st, true);
+    }
+    // Single images: one resident-A launch (PE_FRAMES_PATH=staged|streamed|fused
+    // selects another path instead).
+    const char *fp = std::getenv("PE_FRAMES_PATH");
+    const bool other = fp && (std::strcmp(fp, "staged") == 0 || std::strcmp(fp, "streamed") == 0 ||
+                              std::strcmp(fp, "fused") == 0);
+    if (!other && astat_eligible(h, P, f_dt)) {
+        FwdParams A = P;
+        const pe_status sa = run_frames_astat(h, A, out, st);
+        if (sa != PE_ERR_UNSUPPORTED) return sa;
     }
     const int lp = allow_staged ? frames_path(h, f_dt) : 0;
     if (lp != 0) {
@@ -693,8 +800,10 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
     if (ok && h->has_bias) ok = cudaMalloc(&h->bias, sizeof(float) * E) == cudaSuccess;
     h->Kp32 = (int)((K + 31) / 32 * 32);
     if (ok) ok = cudaMalloc(&h->wpack32, sizeof(uint32_t) * (size_t)E * h->Kp32) == cudaSuccess;
+    h->Kw = 64 * ((h->Kh + 31) / 32);
     if (ok && tp == 2) ok = cudaMalloc(&h->wpack_t, sizeof(uint16_t) * (size_t)E * 2 * h->Kh) == cudaSuccess &&
-                            cudaMalloc(&h->wpack_fold, sizeof(uint16_t) * (size_t)E * h->Kh) == cudaSuccess;
+                            cudaMalloc(&h->wpack_fold, sizeof(uint16_t) * (size_t)E * h->Kh) == cudaSuccess &&
+                            cudaMalloc(&h->wpack_i, sizeof(uint16_t) * (size_t)E * h->Kw) == cudaSuccess;
     if (ok) {
         const uint32_t boxes[3] = {32, 64, 128};   // half of BN = 64, 128, 256
         for (int i = 0; i < 3 && ok; ++i)
@@ -706,6 +815,8 @@ pe_status pe_create(int E, int C, int tp, int p, int has_bias, pe_handle **out) 
                                                 (uint64_t)(2 * h->Kh), boxes[i])) &&
                  (!h->wpack_fold || make_tmap_bf16(&h->tmap_wfold[i], h->wpack_fold, (uint64_t)E, (uint64_t)h->Kh,
                                                    (uint64_t)h->Kh, boxes[i])) &&
+                 (!h->wpack_i || make_tmap_bf16(&h->tmap_wi[i], h->wpack_i, (uint64_t)E, (uint64_t)h->Kw,
+                                                (uint64_t)h->Kw, boxes[i])) &&
                  make_tmap(&h->tmap_w32[i], h->wpack32, true, (uint64_t)E, (uint64_t)h->Kp32, (uint64_t)h->Kp32,
                            boxes[i], 32, CU_TENSOR_MAP_SWIZZLE_128B);
     }
@@ -722,6 +833,7 @@ void pe_destroy(pe_handle *h) {
     if (h->wpack_f) cudaFree(h->wpack_f);
     if (h->wpack_t) cudaFree(h->wpack_t);
     if (h->wpack_fold) cudaFree(h->wpack_fold);
+    if (h->wpack_i) cudaFree(h->wpack_i);
     if (h->wpack32) cudaFree(h->wpack32);
     if (h->bias) cudaFree(h->bias);
     if (h->err) cudaFree(h->err);
@@ -766,6 +878,11 @@ pe_status pe_set_weight(pe_handle *h, const void *w, pe_dtype w_dt, const void *
     if (h->wpack_fold) {
         pe_pack_weight_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_fold,
                                                           nullptr, h->E, h->C, h->tp, h->p, h->Kh, 3, h->Kh);
+        if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
+    }
+    if (h->wpack_i) {
+        pe_pack_weight_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, nullptr, b_dt == PE_F32, h->wpack_i,
+                                                          nullptr, h->E, h->C, h->tp, h->p, h->Kw, 4, h->Kh);
         if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
     }
     pe_pack_weight_tf32_kernel<<<blocks, threads, 0, st>>>(w, w_dt == PE_F32, h->wpack32, h->E, h->K, h->Kp32);
@@ -1075,21 +1192,23 @@ pe_status pe_forward_frames_grouped_noalloc(pe_handle *h, int n, const void *con
     if (n > PE_INLINE_ITEMS) {
         ItemDesc *table = nullptr;
         if (noalloc_table(h->dev, &table) != cudaSuccess) return PE_ERR_CUDA;
-        // Upload in stack-sized chunks; a pageable-source copy returns once the
-        // chunk has been staged, so the stack buffer can be reused at once.
-        ItemDesc chunk[64];
+        // Upload in groups of kItemsPerFill descriptors, each passed by value in
+        // the parameter block of a one-block kernel: stream-ordered, no host
+        // staging buffer, and the host never waits.
+        ItemBatch batch;
         int64_t r0 = 0;
-        for (int base = 0; base < n; base += 64) {
-            const int m = std::min(64, n - base);
+        for (int base = 0; base < n; base += kItemsPerFill) {
+            const int m = std::min(kItemsPerFill, n - base);
+            std::memset(&batch, 0, sizeof(batch));
             for (int j = 0; j < m; ++j) {
                 const int i = base + j;
                 make_item(h, frames[i], THW[3 * i], THW[3 * i + 1], THW[3 * i + 2], grid_thw + 3 * i, merge, r0,
-                          chunk[j]);
+                          batch.d[j]);
                 r0 += (int64_t)grid_thw[3 * i] * grid_thw[3 * i + 1] * grid_thw[3 * i + 2];
             }
-            if (cudaMemcpyAsync(table + base, chunk, sizeof(ItemDesc) * (size_t)m, cudaMemcpyHostToDevice, st) !=
-                cudaSuccess)
-                return PE_ERR_CUDA;
+            pe_fill_items_kernel<<<1, kItemsPerFill, 0, st>>>(batch, table + base, m);
+            if (h->prof_on) ++h->prof_launches;
+            if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
         }
         P.items_dev = table;
     }

@@ -119,6 +119,12 @@ struct FwdParams {
     uint32_t *ready_next;             // the next call's counters, zeroed by this call
     uint32_t ready_target;            // count that marks an M-block complete
     int32_t n_mblocks;
+    // pe_astat_kernel (resident A)
+    int32_t a_offset, bar_offset;     // shared-memory offsets of the resident A and of the barriers
+    int32_t n_achunks;                // A chunks of kAsChunkKs k-steps
+    int32_t epi_bufs;                 // staging boxes per epilogue warp
+    int32_t cpp;                      // C*p*p: columns of one temporal slice
+    uint64_t wait_ns;                 // pipeline wait limit in ns (0: kWaitTimeoutNs)
 };
 
 // ------------------------------------------------------------ row decoding
@@ -1262,7 +1268,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
 //      one A row across the temporal slices;
 //   3  folded: column (c*p + i)*p + j holds bf16_rne(Ŵ[e,c,0,i,j] + Ŵ[e,c,1,i,j])
 //      (the two bf16-rounded slices summed in fp32, rounded once), zero past
-//      C*p*p: single-frame rows meet both slices in one product (tp = 2).
+//      C*p*p: single-frame rows meet both slices in one product (tp = 2);
+//   4  slice-interleaved (tp = 2): 64-column tile s holds slice 0's in-slice
+//      columns 32s..32s+31 followed by slice 1's same columns (in-slice column
+//      (c*p + i)*p + j, zero past C*p*p), so one 128-byte-swizzled tile feeds
+//      two k-steps of both slices against one resident single-frame A.
 __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias, int b_f32,
                                       uint16_t *wpack, float *bias32, int E, int C, int TP, int P,
                                       int ld, int order, int Kh) {
@@ -1283,6 +1293,13 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
             }
         } else if (order == 2) {
             const int t = kd / Kh, kk = kd - t * Kh;
+            if (t < TP && kk < C * P * P) {
+                const int j = kk % P, i = (kk / P) % P, c = kk / (P * P);
+                k = ((c * TP + t) * P + i) * P + j;
+            }
+        } else if (order == 4) {
+            // 64-column tile s = [slice 0, columns 32s..32s+31 | slice 1, the same columns]
+            const int s = kd >> 6, w = kd & 63, t = w >> 5, kk = 32 * s + (w & 31);
             if (t < TP && kk < C * P * P) {
                 const int j = kk % P, i = (kk / P) % P, c = kk / (P * P);
                 k = ((c * TP + t) * P + i) * P + j;
@@ -1551,6 +1568,18 @@ __global__ void pe_patchify_kernel(const __grid_constant__ FwdParams P, void *ro
             *reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(rows) + R * P.K + k) = w;
         }
     }
+}
+
+// Item-table upload without a host staging buffer: up to kItemsPerFill
+// descriptors travel in the launch's parameter block (copied when the launch
+// is queued) and one thread per descriptor writes it to dst[0..n).
+constexpr int kItemsPerFill = 64;
+struct ItemBatch {
+    ItemDesc d[kItemsPerFill];
+};
+__global__ void pe_fill_items_kernel(const __grid_constant__ ItemBatch b, ItemDesc *dst, int n) {
+    const int i = threadIdx.x;
+    if (i < n) dst[i] = b.d[i];
 }
 
 // Failure-path self-test.  One warp waits, through the same bounded wait the
