@@ -196,6 +196,12 @@ def patch_merger(x, m2: int, gamma, beta, eps: float, w1, b1, w2, b2, v_mask=Non
 def conv3d_frames(frames, grid: Sequence[int], merge: int, mean, std, w, bias,
                   C: int, tp: int, p: int, row_mask=None) -> Tuple[np.ndarray, np.ndarray]:
     """Frames form for one item (frames [T,C,H,W]). Returns (out, absdot) [N,E] fp64."""
+    return _frames(frames, grid, merge, mean, std, w, bias, C, tp, p, row_mask, True)
+
+
+def _frames(frames, grid, merge, mean, std, w, bias, C, tp, p, row_mask, fill):
+    """conv3d_frames; with fill=False the rows a row_mask leaves out are left
+    unwritten (np.empty: pages that nothing touches cost nothing)."""
     f = _f32(frames)
     T, Cf, H, W = f.shape
     assert Cf == C
@@ -206,8 +212,9 @@ def conv3d_frames(frames, grid: Sequence[int], merge: int, mean, std, w, bias,
     mu = _f32(np.asarray(mean, dtype=np.float32).reshape(C))
     sd = _f32(np.asarray(std, dtype=np.float32).reshape(C))
     b = None if bias is None else _f32(bias)
-    out = np.full((N, E), np.nan)
-    mag = np.full((N, E), np.nan)
+    make = (lambda shape: np.full(shape, np.nan)) if fill or row_mask is None else np.empty
+    out = make((N, E))
+    mag = make((N, E))
     m = _mask(row_mask, N)
     rc = _load().oracle_conv3d_frames(
         _p(f, ctypes.c_float), T, H, W, gt, gh, gw, merge, _p(mu, ctypes.c_float),
@@ -219,18 +226,33 @@ def conv3d_frames(frames, grid: Sequence[int], merge: int, mean, std, w, bias,
 
 
 def conv3d_grouped(items, merge: int, mean, std, w, bias, C: int, tp: int, p: int,
-                   row_mask=None) -> Tuple[np.ndarray, np.ndarray]:
+                   row_mask=None, compact: bool = False) -> Tuple[np.ndarray, np.ndarray]:
     """Grouped frames form: items' rows concatenated in list order.
-    ``items`` is a sequence of (frames, grid)."""
+    ``items`` is a sequence of (frames, grid).  With ``compact`` (and a
+    row_mask) only the selected rows are returned, in row order, and items
+    without a selected row are not computed at all; the arithmetic of every
+    computed row is the same."""
+    w = _f32(w)                                    # converted once for all items
+    bias = None if bias is None else _f32(bias)
+    mask = None if row_mask is None else np.asarray(row_mask, dtype=np.uint8)
+    compact = compact and mask is not None
     outs, mags = [], []
     off = 0
     for frames, grid in items:
         n = int(grid[0]) * int(grid[1]) * int(grid[2])
-        sub = None if row_mask is None else np.asarray(row_mask)[off:off + n]
-        o, m = conv3d_frames(frames, grid, merge, mean, std, w, bias, C, tp, p, sub)
+        sub = None if mask is None else mask[off:off + n]
+        off += n
+        if compact and not sub.any():
+            continue
+        o, m = _frames(frames, grid, merge, mean, std, w, bias, C, tp, p, sub, not compact)
+        if compact:
+            sel = np.flatnonzero(sub)
+            o, m = o[sel], m[sel]
         outs.append(o)
         mags.append(m)
-        off += n
+    if not outs:
+        E = int(w.shape[0])
+        return np.empty((0, E)), np.empty((0, E))
     return np.concatenate(outs, 0), np.concatenate(mags, 0)
 
 
