@@ -1,29 +1,37 @@
-"""Benchmark of the fused frames -> embedding PatchEmbed on B200.
+"""Benchmark of the vision PatchEmbed on B200: raw frames (or patch rows) in,
+embeddings out.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step is one pass of the whole hot path over one batch of synthetic input:
-host plan, then either one fused kernel (patchify, normalise, merge-order rows,
-bf16 tcgen05 contraction, bias/cast epilogue) or, for large frame batches, the
+host plan, then the kernels of the path the library takes for the workload,
+over every item.  For groups of single images (the default workload, 16
+images in one grouped call) that is one launch of the resident-A kernel: each
+256-row block's patches are gathered from the frames, normalised and placed in
+merge order once in shared memory, and every weight tile streams past them
+(tcgen05 pair MMAs, bias/cast epilogue, TMA stores).  Video items take the
 staged pair (a prepare kernel that writes the normalised rows once, then the
-TMA-fed contraction kernel with the same epilogue), over every item of the
-workload.  The default workload is the grouped batch of 16 images.
+TMA-fed contraction); patch rows take the TMA-fed contraction.
 
-The roofline object describes the contraction kernel alone: in a second timed
+The roofline object describes the dominant kernel alone: in a second timed
 pass of the same K steps the library records a CUDA event pair around it on
 the launching stream in every step (pe_profile_begin / pe_profile_end), and
 bench divides 2*N*K*E by the mean of those durations.  The headline value
 comes from the first pass, which has no events between the kernels of a step
 (an event there serialises the staged path's two kernels).
 
-For N > 1 (torchrun, one process per GPU) every rank embeds its own copy of the
-workload (weak scaling, no data-path collective); the value is all patches of
-all ranks divided by the slowest rank's device time.
+For N > 1 (torchrun, one process per GPU, --gpus N must equal the number of
+ranks) the global batch is N copies of the workload, cut into contiguous
+output-row ranges at whole items or temporal patches (one range per rank,
+weight replicated, no collective on the data path): weak scaling.  The value is
+all ranks' patches over the slowest rank's device time.
 
 Rank 0 prints one JSON line.  Timing: W untimed warm-up steps; K timed steps,
 each bracketed by CUDA events on the launching stream, with an L2 flush (a
 write larger than L2) before every step outside the events; barrier +
-synchronize around the timed region; max over ranks.
+synchronize around the timed region; max over ranks.  The e2e value goes
+through the library's host-buffer call (pinned host frames in, host
+embeddings out, copies inside the timed region).
 """
 from __future__ import annotations
 
@@ -63,13 +71,13 @@ def load_peaks():
 # SHA-256 of the kernel sources it was taken on.  A changed kernel invalidates
 # the figure (reported as null) until it is captured again.
 TRAFFIC = {
-    # profiles/pe_fwd_kernel_grouped_16_images.md, profiles/pe_fwd_kernel_long_video_64x896.md
     ("grouped_16_images", "staged"): {"bytes": 94770944 + 97856256, "kernel_sha": "2d0b9a5fb46fd12c"},
     ("long_video_64x896", "staged"): {"bytes": 381790464 + 282007296, "kernel_sha": "2d0b9a5fb46fd12c"},
-    # profiles/pe_fwd_kernel_merger_fc1_grouped_16_images.md (the PatchMerger's fc1 + GELU)
+    # the PatchMerger's fc1 + GELU
     ("patch_merger_grouped_16_images", "fc1"): {"bytes": 614624768 + 134967040, "kernel_sha": "2d0b9a5fb46fd12c"},
 }
-KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh")
+KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh",
+                  "vlm_vision_patch_b200/csrc/pe_astat.cuh")
 
 
 def code_digest(texts):
@@ -216,22 +224,36 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle arm
 
+def oracle_inputs(wl):
+    """The workload's tensors as fp32 numpy arrays for the oracle (bf16 widens
+    exactly), converted once per workload, outside every timed region: input
+    marshalling, not the oracle's work."""
+    if getattr(wl, "_oracle_in", None) is None:
+        f32 = lambda t: None if t is None else np.ascontiguousarray(t.float().numpy())  # noqa: E731
+        wl._oracle_in = {"patches": f32(wl.patches), "weight": f32(wl.weight), "bias": f32(wl.bias),
+                         "items": [(f32(it.frames), it.grid) for it in wl.items]}
+    return wl._oracle_in
+
+
 def oracle_sample_rate(wl, n_rows: int, seed: int, fp32_form: bool = False):
     """Time the CPU oracle on n_rows sampled output rows of the workload
     (fp32_form: the unrounded fp32 Conv3d that the tf32 path is checked
-    against, for fp32 patch rows).  Returns (rows/s, seconds, threads)."""
+    against, for fp32 patch rows).  Only the sampled rows are computed and
+    returned (patch rows: the selected rows; frames: the oracle's compact
+    row-mask form).  Returns (rows/s, seconds, threads)."""
     import oracle
+    inp = oracle_inputs(wl)
     rng = np.random.default_rng(seed)
-    rows = rng.choice(wl.N, size=min(n_rows, wl.N), replace=False)
-    mask = np.zeros(wl.N, np.uint8)
-    mask[rows] = 1
+    rows = np.sort(rng.choice(wl.N, size=min(n_rows, wl.N), replace=False))
     t0 = time.perf_counter()
     if wl.patches is not None:
         form = oracle.conv3d_patches_fp32 if fp32_form else oracle.conv3d_patches
-        form(wl.patches, wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
+        form(inp["patches"][rows], inp["weight"], inp["bias"], wl.C, wl.tp, wl.p)
     else:
-        oracle.conv3d_grouped([(it.frames, it.grid) for it in wl.items], wl.merge, wl.mean, wl.std,
-                              wl.weight, wl.bias, wl.C, wl.tp, wl.p, row_mask=mask)
+        mask = np.zeros(wl.N, np.uint8)
+        mask[rows] = 1
+        oracle.conv3d_grouped(inp["items"], wl.merge, wl.mean, wl.std, inp["weight"], inp["bias"],
+                              wl.C, wl.tp, wl.p, row_mask=mask, compact=True)
     dt = time.perf_counter() - t0
     return len(rows) / dt, dt, oracle.num_threads()
 
@@ -292,11 +314,35 @@ def library_context(wl, dev, flush_buf, reps=20):
                                    "shape": [wl.N, wl.K, wl.E]}}
 
 
+E2E_PATHS = {"host": "pe_forward_frames_grouped_host / pe_forward_patches_host (C ABI, host buffers): chunked "
+                     "copies in both directions pipelined with the contraction",
+             "serial": "pinned copy_ in, the device-pointer call, copy_ out, one stream"}
+
+
+def local_shard(wl, world, rank):
+    """This rank's part of a global batch made of `world` copies of the
+    workload, cut into contiguous output-row ranges at whole items or whole
+    temporal patches (vlm_vision_patch_b200.shard): about one copy's rows per
+    rank (weak scaling), no exchange on the data path.  The workload itself at
+    world 1; patch rows shard to exactly one copy per rank."""
+    if world == 1 or wl.patches is not None:
+        return wl
+    import dataclasses
+    from vlm_vision_patch_b200.shard import shard_rows
+    n = len(wl.items)
+    pieces = shard_rows([it.frames.shape[0] for it in wl.items] * world, [it.grid for it in wl.items] * world,
+                        wl.tp, world)[rank]
+    items = [workloads.Item(wl.items[pc.item % n].frames[pc.f0:pc.f1], pc.grid) for pc in pieces]
+    return dataclasses.replace(wl, items=items)
+
+
 def config_of(wl, world):
     cfg = {"workload": wl.name, "N_patches": wl.N, "K": wl.K, "E": wl.E, "patch": wl.p,
            "temporal_patch": wl.tp, "merge": wl.merge, "items": max(1, len(wl.items)),
            "out_dtype": "bf16" if wl.out_dtype == torch.bfloat16 else "f32",
-           "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
+           "parallelism": (f"row shards x{world}: {world} copies of the workload split into contiguous output-row "
+                           "ranges at whole items / temporal patches, weight replicated, no data-path collective")
+                          if world > 1 else "1 gpu",
            "l2": "flushed before every timed step (write of 2x L2 outside the events)"}
     return cfg
 
@@ -312,7 +358,9 @@ def run_ours(args, rank, world, local):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
-    wl = workloads.ALL[args.workload]()
+    wl_global = workloads.ALL[args.workload]()
+    wl = local_shard(wl_global, world, rank)
+    total_rows = world * wl_global.N            # every rank's rows of the global batch
     pe = vp.PatchEmbed(wl.E, wl.C, wl.tp, wl.p, wl.bias is not None)
     pe.set_weight(wl.weight.to(dev), None if wl.bias is None else wl.bias.to(dev))
     pe.set_norm(wl.mean, wl.std)
@@ -386,12 +434,13 @@ def run_ours(args, rank, world, local):
     if pe.last_error() != 0:
         raise RuntimeError("device pipeline timeout during the timed steps")
     total_max_ms = max_over_ranks(sum(times), pg, dev)
-    value = weak_scaling_value(wl.N, args.steps, world, total_max_ms)
+    value = total_rows * args.steps / (total_max_ms / 1e3)
 
     # end to end through the public API with host buffers (pinned), per step:
-    # H2D of the step's frames, the forward, D2H of the embeddings.  "serial":
-    # copy_ in, the device-pointer call, copy_ out, one stream; "host": the
-    # host-buffer call, which pipelines the copies and the contraction in chunks.
+    # H2D of the step's frames, the forward, D2H of the embeddings.  "host"
+    # (the headline): the C-ABI host-buffer call, which pipelines the copies in
+    # both directions with the contraction in chunks; "serial" (context):
+    # copy_ in, the device-pointer call, copy_ out, one stream.
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
     if wl.patches is not None:
         host_in = [wl.patches.pin_memory()]
@@ -401,8 +450,8 @@ def run_ours(args, rank, world, local):
         dev_in = frames_dev
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
 
-    def e2e_step():
-        if args.e2e == "host":
+    def e2e_step(mode):
+        if mode == "host":
             if wl.patches is not None:
                 pe.forward_patches_host(host_in[0], out=host_out, stream=stream, blocking=False)
             else:
@@ -413,18 +462,25 @@ def run_ours(args, rank, world, local):
             d_.copy_(h_, non_blocking=True)
         step()
         host_out.copy_(out, non_blocking=True)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    if pg:
-        pg.barrier()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_value = weak_scaling_value(wl.N, e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), pg, dev))
+
+    def e2e_rate(mode):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            e2e_step(mode)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step(mode)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return total_rows * e2e_steps / (max_over_ranks(e0.elapsed_time(e1), pg, dev) / 1e3)
+    other = "serial" if args.e2e == "host" else "host"
+    e2e_value = e2e_rate(args.e2e)
+    e2e_other = e2e_rate(other)
+    if pe.last_error() != 0:
+        raise RuntimeError("device pipeline timeout during the end-to-end steps")
 
     result = None
     if rank == 0:
@@ -441,11 +497,16 @@ def run_ours(args, rank, world, local):
         # dense tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s)
         peak = float(peaks["bf16_tflops"]) * (1.1 / 2.25 if tf32 else 1.0)
         staged = launches == 2 * args.steps
+        kernel = "pe_fwd_kernel (contraction)"
         if wl.patches is not None:
             path = ("patches: fp32 rows cast to bf16 by a kernel, then the TMA-fed pair GEMM"
                     if wl.patches.dtype == torch.float32 else "patches: bf16 rows, TMA-fed pair GEMM")
         elif staged:
             path = "staged: prepare kernel writes the normalised rows, then the TMA-fed pair GEMM"
+        elif wl.tp == 2 and all(it.frames.shape[0] == 1 for it in wl.items):
+            path = ("fused, resident A: one kernel from frames to embeddings (each 256-row block gathered once "
+                    "into shared memory, the weight streamed past it)")
+            kernel = "pe_astat_kernel (fused frames -> embeddings)"
         else:
             path = "fused: one kernel from frames to embeddings"
         cpu = None
@@ -454,7 +515,7 @@ def run_ours(args, rank, world, local):
             cpu = {"value": r, "unit": UNIT, "cores": th, "kind": "oracle",
                    "sample": f"{min(args.cpu_rows, wl.N)} seeded random output rows of {wl.name} (of {wl.N}), "
                              f"{dt:.1f} s; direct fp64 Conv3d, OpenMP over rows"}
-        traffic = measured_traffic(wl.name, "staged" if staged else "single")
+        traffic = measured_traffic(wl.name, "staged" if staged else ("astat" if "resident A" in path else "single"))
         context = None if (args.no_context or world > 1) else library_context(wl, dev, flush_buf)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -476,17 +537,14 @@ def run_ours(args, rank, world, local):
                           "rest_of_step_mean": statistics.mean(times_k) - gemm_ms},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "pe_fwd_kernel (contraction), 2*N*K*E flop per launch over its own "
-                                   "CUDA-event duration",
+                         "kernel": kernel + ", 2*N*K*E flop per launch over its own CUDA-event duration",
                          "peak_source": (f"{src} bf16 dense (burst), MEASURED_PEAKS.json" if src == "measured"
                                          else "fallback 1590 TFLOP/s bf16")
                                         + (" x 1.1/2.25 (nominal tf32/bf16)" if tf32 else "")},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
-                    "d2h_bytes_per_step": out_bytes,
-                    "path": ("host-buffer call: chunked copies in both directions pipelined with the contraction"
-                             if args.e2e == "host" else
-                             "serial: pinned copy_ in, the device-pointer call, copy_ out, one stream")},
+                    "d2h_bytes_per_step": out_bytes, "path": E2E_PATHS[args.e2e],
+                    other: {"value": e2e_other, "unit": UNIT, "path": E2E_PATHS[other]}},
             "gpu_launches": launches,
             "context": context,
             "clocks": clk.summary(),
@@ -527,7 +585,7 @@ def run_reference_merger(args, rank, world):
     V = wl.N // 4
     x = (torch.randn(V * 4, E, generator=torch.Generator().manual_seed(78)) * 0.5).to(torch.bfloat16)
     gamma, beta, w1, b1, w2, b2 = merger_weights(E, H)
-    per_step = max(1, min(args.ref_rows // 4, V))
+    per_step = max(1, min(args.ref_rows // 32, V))   # 256 merged rows (about 17 GFLOP fp64) at the default
 
     def sample(n, seed):
         rng = np.random.default_rng(seed)
@@ -655,11 +713,12 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=65536,
                     help="output rows in the CPU oracle's timed sample (capped at the workload's N): about "
                          "10-30 s on the host cores")
-    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=8192,
+                    help="output rows the reference arm's oracle computes per step (capped at the workload's N)")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--e2e", default="serial", choices=["serial", "host"],
-                    help="how the end-to-end number moves host data: serial copies around the device-pointer "
-                         "call, or the library's pipelined host-buffer call")
+    ap.add_argument("--e2e", default="host", choices=["serial", "host"],
+                    help="which end-to-end form is the headline e2e value (the other is reported beside it): "
+                         "the library's pipelined host-buffer call, or serial copies around the device-pointer call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the cuBLAS context timing")
     ap.add_argument("--merger", action="store_true",
@@ -673,6 +732,9 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, world, local = dist_env()
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} but {world} process(es) were launched: run N > 1 ranks with "
+                 f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py --gpus {args.gpus} ...")
     if args.impl == "reference":
         return run_reference_merger(args, rank, world) if args.merger else run_reference(args, rank, world)
     if args.merger:

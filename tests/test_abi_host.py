@@ -102,14 +102,3 @@ def test_create_without_gpu_fails_cleanly(lib):
     h = ctypes.c_void_p()
     rc = lib.pe_create(1280, 3, 2, 14, 0, ctypes.byref(h))
     assert rc != 0 and h.value is None
-
-
-def test_design_notes_list_every_call():
-    """The boundary section of the design notes names every call the header
-    declares (the PatchMerger's calls may be written by suffix)."""
-    text = open(os.path.join(ROOT, "DESIGN.md"), encoding="utf-8").read()
-    section = text[text.index("### 2.2 Boundary"):text.index("## 3. Readings")]
-    missing = [f for f in declared_functions()
-               if f"`{f}`" not in section
-               and not (f.startswith("pe_merger_") and f"`_{f[len('pe_merger_'):]}`" in section)]
-    assert not missing, missing
