@@ -183,18 +183,13 @@ def test_frames_small_shapes(T, gh, gw, merge, p, tp, E, bias):
     assert_within_tolerance(out, ref, mag, what=wl.name)
 
 
-def test_grouped_16_images_sampled_rows():
-    """The 16-image grouped workload at full size, checked on sampled rows
-    (every item boundary included)."""
+def test_grouped_16_images_all_rows():
+    """The 16-image grouped workload at full size (59204 rows, the benchmark's
+    launch), every element against the oracle."""
     wl = workloads.grouped_16_images()
-    bounds, off = [], 0
-    for it in wl.items:
-        n = it.grid[0] * it.grid[1] * it.grid[2]
-        bounds += [off, off + 1, off + n - 1]
-        off += n
-    rows = sample_rows(wl.N, 3000, 60, bounds)
-    _, out, ref, mag = _run_frames(wl, rows=rows)
-    assert_within_tolerance(out, ref, mag, rows=rows, what=wl.name)
+    _, out, ref, mag = _run_frames(wl)
+    r = assert_within_tolerance(out, ref, mag, what=wl.name)
+    print(f"grouped_16_images: worst |err| / tolerance = {r:.3f}")
 
 
 def test_grouped_small_items_all_rows():
@@ -391,19 +386,20 @@ def _folded_weight(w: torch.Tensor) -> torch.Tensor:
     return out
 
 
-@pytest.mark.parametrize("case", ["image_224x896", "grouped_small", "p16_raster_bias", "grouped_16_sampled"])
+@pytest.mark.parametrize("case", ["image_224x896", "grouped_small", "p16_raster_bias", "grouped_16_images"])
 def test_temporal_fold(case):
     """Opt-in folding: (1) within the parity tolerance of the oracle run with the
     folded weight (the same products, any summation order); (2) within the
-    folding bound 2^-8 * sum|x̂ ŵ| (+ fp32 accumulation and one bf16 ulp) of the
-    exact, unfolded result."""
+    parity tolerance 1e-3 * sum|x̂ ŵ| (+ one bf16 ulp) of the exact, unfolded
+    Conv3d on every row, the 59204-row group included.  The folded weight
+    carries one more bf16 rounding per term (at most 2^-9 of |Ŵ0 + Ŵ1|); its
+    errors have random signs over the C*p*p terms of a row, so on these inputs
+    they stay well inside the bound (the worst ratio is printed)."""
     rows = None
     if case == "image_224x896":
         wl = workloads.image_224x896()
-    elif case == "grouped_16_sampled":
+    elif case == "grouped_16_images":
         wl = workloads.grouped_16_images()
-        offs = np.cumsum([0] + [g[0] * g[1] * g[2] for g in (it.grid for it in wl.items)])
-        rows = sample_rows(wl.N, 600, 77, extra=offs[1:-1])
     else:
         C, tp = 3, 2
         if case == "grouped_small":
@@ -432,8 +428,8 @@ def test_temporal_fold(case):
     assert_within_tolerance(out, ref_f, mag_f, rows=rows, what=f"{case} folded-weight oracle")
     ref, mag = oracle.conv3d_grouped(its, wl.merge, wl.mean, wl.std, wl.weight, wl.bias,
                                      wl.C, wl.tp, wl.p, row_mask=mask)
-    assert_within_tolerance(out, ref, mag, rows=rows, what=f"{case} exact oracle, folding bound",
-                            rel=2.0 ** -8 + 1e-3)
+    r = assert_within_tolerance(out, ref, mag, rows=rows, what=f"{case} exact oracle, parity tolerance")
+    print(f"fold {case}: worst |err| / tolerance against the exact Conv3d = {r:.3f}")
 
 
 def test_temporal_fold_leaves_video_and_off_state_alone():
@@ -620,12 +616,13 @@ def _merger_case(E, m, H, V, bias, wdt, seed):
     (64, 1, 128, 300, True, torch.bfloat16, torch.float32),       # m = 1
 ])
 def test_patch_merger(E, m, H, V, bias, wdt, out_dtype):
-    """GPU PatchMerger vs the oracle.  Tolerance: the GPU rounds the LayerNorm
-    and GELU outputs to bf16 like the oracle, but from fp32 rather than fp64
-    values, so an element of either may land one bf16 ulp away; through fc2
-    that is at most 2^-8 * sum|g w2| per output, doubled for the fc1 stage and
-    widened for fp32 accumulation: |err| <= 1e-2 * sum|g w2| (+ 1 bf16 ulp for
-    bf16 output).  The typical error must also stay well inside it."""
+    """GPU PatchMerger vs the oracle at the parity tolerance 1e-3 * sum|g w2|
+    (+ 1 bf16 ulp for bf16 output), g the bf16 GELU output.  The GPU rounds the
+    LayerNorm and GELU outputs to bf16 like the oracle, but from fp32 rather
+    than fp64 values: an element lands one bf16 ulp away only when its fp32 and
+    fp64 values straddle a rounding boundary (a few per row), and one such term
+    moves an output by about 2^-8 of one of the D terms of sum|g w2|.  The
+    worst ratio is printed."""
     x, gamma, beta, w1, b1, w2, b2 = _merger_case(E, m, H, V, bias, wdt, 500 + E + V)
     pm = PatchMerger(E, m, H, 1e-6)
     dev = lambda t: None if t is None else t.to(DEV).contiguous()
@@ -634,10 +631,8 @@ def test_patch_merger(E, m, H, V, bias, wdt, out_dtype):
     torch.cuda.synchronize()
     assert pm.last_error() == 0
     ref, mag = oracle.patch_merger(x, m * m, gamma, beta, 1e-6, w1, b1, w2, b2)
-    r = assert_within_tolerance(out, ref, mag, what=f"merger {E},{m},{H},{V}", rel=1e-2)
-    err = np.abs(out.detach().cpu().double().numpy() - ref) / np.maximum(mag, 1e-30)
-    assert np.median(err) < 1e-3, np.median(err)
-    assert r <= 1.0
+    r = assert_within_tolerance(out, ref, mag, what=f"merger {E},{m},{H},{V}")
+    print(f"merger {E},{m},{H},{V}: worst |err| / tolerance = {r:.3f}")
     pm.close()
 
 
@@ -654,7 +649,8 @@ def test_patch_merger_full_size_sampled():
     assert pm.last_error() == 0
     rows = sample_rows(V, 24, 601)
     ref, mag = oracle.patch_merger(x, 4, gamma, beta, 1e-6, w1, b1, w2, b2, v_mask=mask_of(rows, V))
-    assert_within_tolerance(out, ref, mag, rows=rows, what="merger full size", rel=1e-2)
+    r = assert_within_tolerance(out, ref, mag, rows=rows, what="merger full size")
+    print(f"merger full size: worst |err| / tolerance = {r:.3f}")
     pm.close()
 
 
@@ -678,8 +674,8 @@ def test_patch_merger_errors():
                                   "tf32_with_pos"])
 def test_more_path_combinations(case, monkeypatch):
     """Combinations of options and ragged shapes on the default paths, each
-    against the oracle at the parity tolerance (the folded case at the folding
-    bound, the tf32 case against the unrounded oracle at the tf32 bound)."""
+    against the oracle at the parity tolerance (the tf32 case against the
+    unrounded oracle at the tf32 bound)."""
     C, tp = 3, 2
     if case.startswith("tf32"):
         p, E, N = 14, 256, 200
@@ -715,9 +711,47 @@ def test_more_path_combinations(case, monkeypatch):
     torch.cuda.synchronize()
     assert pe.last_error() == 0
     ref, mag = oracle.conv3d_grouped(items, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
-    rel = 1e-3
     if pos is not None:
         pv = pos.double().numpy()
         ref, mag = ref + pv, mag + np.abs(pv)
-        rel = 2.0 ** -8 + 1e-3
-    assert_within_tolerance(out, ref, mag, what=case, rel=rel)
+    assert_within_tolerance(out, ref, mag, what=case)
+
+
+# ----------------------------------------------- Qwen3-VL PatchEmbed shape
+
+QWEN3 = dict(C=3, tp=2, p=16, E=1024)   # Optimize VLM PatchEmbed: Qwen3VLVisionPatchEmbed, bias=True, 2B hidden size
+
+
+def test_qwen3_vl_shape_frames():
+    """Qwen3VLVisionPatchEmbed's shape (patch 16, temporal 2, hidden 1024, with
+    bias) on frames: an image and a video with an odd frame count in one
+    grouped call, merge order, every row against the oracle."""
+    C, tp, p, E = QWEN3["C"], QWEN3["tp"], QWEN3["p"], QWEN3["E"]
+    grids, Ts = [(1, 12, 16), (2, 8, 10)], [1, 3]
+    items = [(workloads.uniform01((T, C, g[1] * p, g[2] * p), 800 + i), g) for i, (T, g) in enumerate(zip(Ts, grids))]
+    w = workloads.normal((E, C, tp, p, p), 801, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 802, std=0.02, dtype=torch.bfloat16)
+    pe = _pe((E, C, tp, p), w, b, workloads.CLIP_MEAN, workloads.CLIP_STD)
+    for od in (torch.bfloat16, torch.float32):
+        out = pe.forward_frames_grouped([f.to(DEV) for f, _ in items], grids, 2, out_dtype=od)
+        torch.cuda.synchronize()
+        assert pe.last_error() == 0
+        ref, mag = oracle.conv3d_grouped(items, 2, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
+        assert_within_tolerance(out, ref, mag, what=f"Qwen3-VL frames {od}")
+
+
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
+def test_qwen3_vl_shape_patches(x_dtype):
+    """The same shape on patch rows [N, 1536] (the processor's pixel_values),
+    N ragged against the 256-row tiles."""
+    C, tp, p, E = QWEN3["C"], QWEN3["tp"], QWEN3["p"], QWEN3["E"]
+    K = C * tp * p * p
+    x = workloads.normal((777, K), 810)
+    w = workloads.normal((E, C, tp, p, p), 811, std=0.02)
+    b = workloads.normal((E,), 812, std=0.02)
+    pe = _pe((E, C, tp, p), w, b)
+    out = pe.forward_patches(x.to(x_dtype).to(DEV), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    ref, mag = oracle.conv3d_patches(x.to(x_dtype), w, b, C, tp, p)
+    assert_within_tolerance(out, ref, mag, what=f"Qwen3-VL patches {x_dtype}")
