@@ -196,26 +196,28 @@ pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int
  *   out      : dev [gt*gh*gw, E] of dtype out_dt.
  * Requires p even and p <= PE_MAX_PATCH.  Execution paths, all within the
  * same tolerance of the exact result:
- *   resident A  (default when every item is a single frame, bf16 frames,
- *            tp = 2 and the C*p*p-column A block fits in shared memory beside
- *            the weight ring: C = 3 with p <= 14) one kernel; each 256-row
- *            block's normalised patches are gathered from the frames once into
- *            shared memory, in merge order, and every weight tile streams past
- *            them; both temporal slices of the weight meet the one frame.  No
- *            workspace; the [N, K] patch matrix never exists in memory;
- *   fused    one kernel that gathers each A tile again for every weight tile
- *            (fp32 frames, tp != 2, p not in {14, 16} with video items, and
- *            the allocation-free call's video groups);
- *   staged   (default for other bf16 frames with tp = 2 and p in {14, 16}) a
- *            prepare kernel writes the normalised rows once into the handle's
+ *   staged   (default for bf16 frames with tp = 2 and p in {14, 16}) a prepare
+ *            kernel writes the normalised rows once into the handle's
  *            grow-only workspace, then the TMA-fed contraction reads them back;
+ *   resident A  (PE_FRAMES_PATH=astat, and the allocation-free call, when
+ *            every item is a single frame, the frames are bf16, tp = 2 and the
+ *            C*p*p-column A block fits in shared memory beside the weight
+ *            ring) one kernel; each 256-row block's normalised patches are
+ *            gathered from the frames once into shared memory, in merge order,
+ *            and every weight tile streams past them; both temporal slices of
+ *            the weight meet the one frame.  No workspace; the [N, K] patch
+ *            matrix never exists in memory.  It issues, row by row, the same
+ *            MMAs in the same order as the staged path, so the two give
+ *            identical bits.  On B200 it runs slower than the staged pair (the
+ *            resident A leaves the weight ring too little shared memory);
+ *   fused    one kernel that gathers each A tile again for every weight tile
+ *            (fp32 frames, tp != 2, p not in {14, 16}, and the allocation-free
+ *            call's other groups);
  *   streamed one cooperative kernel: producer warps write the same rows while
  *            the contraction consumes the completed row blocks (an option:
  *            slower than staged on B200).
- * The resident-A path issues, row by row, the same MMAs in the same order as
- * the staged path on single images, so the two give identical bits.  The
- * environment variable PE_FRAMES_PATH=fused|streamed|staged selects another
- * path instead of the default.  PE_TEST_WAIT_NS=n (a test hook) gives the
+ * The environment variable PE_FRAMES_PATH=staged|astat|fused|streamed selects
+ * a path instead of the default.  PE_TEST_WAIT_NS=n (a test hook) gives the
  * resident-A kernel's pipeline waits a limit of n ns instead of 2 s, so that a
  * test can make them run out and exercise the kernel's unwinding: the call
  * then leaves an incomplete output and pe_last_error reports

@@ -23,7 +23,8 @@ from __future__ import annotations
 
 import pytest
 
-CHUNK_KS = 4          # kAsChunkKs: k-steps per resident-A chunk
+# k-steps per resident-A chunk: 8 image-row segments of p columns = p/2
+# k-steps (7 for p = 14); parametrised below
 
 
 class Bar:
@@ -64,10 +65,10 @@ def parity_wait(bar: Bar, parity: int, phase: int):
         yield
 
 
-def simulate(num_passes, ntn, npairs_cap, nb, n_iss, nks, bug=None):
+def simulate(num_passes, ntn, npairs_cap, nb, n_iss, nks, bug=None, cks=7):
     npairs = min(num_passes, npairs_cap)
-    nst = (nks + 1) // 2
-    nch = (nks + CHUNK_KS - 1) // CHUNK_KS
+    nst = (nks + 3) // 4          # weight stages of 4 k-steps
+    nch = (nks + cks - 1) // cks
     for pair in range(npairs):
         q0 = num_passes * pair // npairs
         q1 = num_passes * (pair + 1) // npairs
@@ -109,26 +110,22 @@ def simulate(num_passes, ntn, npairs_cap, nb, n_iss, nks, bug=None):
                 new_a = q == q0 or n == 0
                 last_a = q == q1 - 1 or n == ntn - 1
                 yield from parity_wait(tempty[acc], accph ^ 1, ause[acc] - 1)
-                next_wait = 0 if new_a else nks
-                next_rel = CHUNK_KS - 1 if last_a else nks + 1
-                hw = hr = 0
+                hw = 0 if new_a else nch          # next A chunk to await (first pass over a block)
+                hr = 0 if last_a else nch         # next A chunk to release (last pass over a block)
                 for j in range(nst):
+                    s0 = 4 * j
+                    slast = min(s0 + 3, nks - 1)
+                    while hw < nch and hw * cks <= slast:   # the chunks this stage reads
+                        yield from parity_wait(full_a[hw], aph, gathers)
+                        hw += 1
                     yield from parity_wait(full_w[ws], wph, wuse[ws])
                     wuse[ws] += 1
-                    for kk in range(2):
-                        s = 2 * j + kk
-                        if s >= nks:
-                            continue
-                        if s == next_wait:
-                            yield from parity_wait(full_a[hw], aph, gathers)
-                            hw += 1
-                            next_wait += CHUNK_KS
-                        if s == next_rel or (last_a and s == nks - 1):
-                            if not (bug == "no_last_release" and hr == nch - 1):
-                                empty_a[hr].arrive()
-                            hr += 1
-                            next_rel += CHUNK_KS
                     empty_w[ws].arrive()
+                    # chunks whose last k-step is issued go back to the producers
+                    while hr < nch and min((hr + 1) * cks, nks) - 1 <= slast:
+                        if not (bug == "no_last_release" and hr == nch - 1):
+                            empty_a[hr].arrive()
+                        hr += 1
                     ws += 1
                     if ws == nb:
                         ws, wph = 0, wph ^ 1
@@ -190,11 +187,11 @@ SHAPES = [(232, 5, 74), (4, 10, 74), (4, 5, 74), (1, 1, 74), (3, 5, 2), (7, 3, 4
 
 @pytest.mark.parametrize("mt,ntn,npairs", SHAPES)
 @pytest.mark.parametrize("nb,n_iss", [(2, 2), (3, 3), (4, 3), (8, 3), (5, 2)])
-@pytest.mark.parametrize("nks", [37, 12, 1, 48])
-def test_protocol_completes_on_the_intended_phases(mt, ntn, npairs, nb, n_iss, nks):
+@pytest.mark.parametrize("nks,cks", [(37, 7), (12, 3), (1, 1), (48, 8), (27, 6)])
+def test_protocol_completes_on_the_intended_phases(mt, ntn, npairs, nb, n_iss, nks, cks):
     if mt * ntn > 400 and (nb, n_iss) != (4, 3):
         pytest.skip("the full-size grouped case runs with the default ring only")
-    simulate(mt * ntn, ntn, npairs, nb, n_iss, nks)
+    simulate(mt * ntn, ntn, npairs, nb, n_iss, nks, cks=cks)
 
 
 @pytest.mark.parametrize("bug,exc", [("producer_skips_wait", Lapped), ("no_last_release", Deadlock),

@@ -1,7 +1,8 @@
 """The resident-A frames kernel (single images, one launch) vs the CPU oracle.
 
-Groups whose items are all single frames (T = 1, duplicated to tp = 2) run by
-default through pe_astat_kernel: each 256-row block's normalised A is built
+Groups whose items are all single frames (T = 1, duplicated to tp = 2) run
+through pe_astat_kernel with PE_FRAMES_PATH=astat and in the allocation-free
+call: each 256-row block's normalised A is built
 once in shared memory from the raw frames and every weight tile streams past
 it, so the [N, K] patch matrix never exists in global memory (patch详解 §4.3,
 the Conv3d cuts and projects in one step).  Checked here:
@@ -48,10 +49,7 @@ def _pe(wl):
 
 
 def _forward(pe, wl, frames, out_dtype, path, monkeypatch, pos=None):
-    if path == "astat":
-        monkeypatch.delenv("PE_FRAMES_PATH", raising=False)
-    else:
-        monkeypatch.setenv("PE_FRAMES_PATH", path)
+    monkeypatch.setenv("PE_FRAMES_PATH", path)
     B.pe_profile_begin(pe.h, 0)
     out = pe.forward_frames_grouped(frames, [it.grid for it in wl.items], wl.merge, out_dtype=out_dtype, pos=pos)
     _, launches = B.pe_profile_end(pe.h, 0)
@@ -105,14 +103,16 @@ def test_astat_every_tile_width(bn, monkeypatch):
     assert torch.equal(out_a, out_s)
 
 
-@pytest.mark.parametrize("nb,bufs", [(2, 1), (2, 2), (3, 1), (3, 2), (4, 1)])
-def test_astat_ring_depths_and_staging(nb, bufs, monkeypatch):
-    """Every weight-ring depth and staging count the planner can choose at
-    BN = 256 gives the same bits (the pipeline shape changes no arithmetic)."""
+@pytest.mark.parametrize("bn,nb,bufs", [("256", 2, 0), ("128", 2, 2), ("128", 3, 1), ("128", 4, 0),
+                                         ("64", 2, 2), ("64", 6, 2), ("64", 5, 0)])
+def test_astat_ring_depths_and_staging(bn, nb, bufs, monkeypatch):
+    """Weight-ring depths and epilogue forms the planner can choose (staging
+    boxes for TMA stores, or stores straight from registers when no boxes fit)
+    give the same bits (the pipeline shape changes no arithmetic)."""
     wl = _wl([(1, 20, 24), (1, 16, 10), (1, 6, 14)], E=1280, seed=230)
     pe = _pe(wl)
     frames = [it.frames.to(DEV) for it in wl.items]
-    monkeypatch.setenv("PE_BN", "256")
+    monkeypatch.setenv("PE_BN", bn)
     base, _ = _forward(pe, wl, frames, torch.bfloat16, "staged", monkeypatch)
     monkeypatch.setenv("PE_ASTAT_NB", str(nb))
     monkeypatch.setenv("PE_ASTAT_EPIBUFS", str(bufs))
@@ -195,13 +195,17 @@ def test_astat_many_items_device_table(monkeypatch):
     assert_within_tolerance(out, ref, mag, what="resident A, 40 items")
 
 
-def test_p16_images_fall_back_to_staged(monkeypatch):
-    """p = 16 (a 768-column A, 192 KB) leaves no room for the weight ring: the
-    call runs the staged pair, still within tolerance."""
-    wl = _wl([(1, 6, 8)], E=1024, p=16, seed=290)
+@pytest.mark.parametrize("bn,launches", [("64", 1), ("256", 2)])
+def test_p16_images_resident_when_the_ring_fits(bn, launches, monkeypatch):
+    """p = 16 makes a 768-column A (192 KB): beside 64-wide weight tiles (4 KB
+    stages) it still fits and the call is one resident-A launch; with 256-wide
+    tiles (16 KB stages) it does not, and the call runs the staged pair.  Both
+    within tolerance of the oracle."""
+    monkeypatch.setenv("PE_BN", bn)
+    wl = _wl([(1, 6, 8), (1, 4, 10)], E=1024, p=16, seed=290)
     pe = _pe(wl)
     frames = [it.frames.to(DEV) for it in wl.items]
-    out, launches = _forward(pe, wl, frames, torch.bfloat16, "astat", monkeypatch)
-    assert launches == 2
+    out, n = _forward(pe, wl, frames, torch.bfloat16, "astat", monkeypatch)
+    assert n == launches
     ref, mag = _oracle(wl)
-    assert_within_tolerance(out, ref, mag, what="p=16 images")
+    assert_within_tolerance(out, ref, mag, what=f"p=16 images, BN={bn}")

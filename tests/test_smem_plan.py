@@ -88,18 +88,26 @@ int main() {
                     const size_t bars = (size_t)(2 * P.nb + 2 * P.n_achunks + 5) * 8 + (size_t)(2 * P.nb + 2) * 4;
                     if (total > (size_t)h.smem_optin) fail("astat shared memory", 100, C, 2, p, bn);
                     if (P.nb < 2 || P.n_iss < 1 || P.n_iss > P.nb || P.n_iss > 3) fail("astat ring", 100, C, 2, p, bn);
-                    if (P.epi_bufs < 1 || P.epi_bufs > 2) fail("astat staging", 100, C, 2, p, bn);
-                    if (P.b_slot_bytes != bn / 2 * 128) fail("astat slot", 100, C, 2, p, bn);
+                    if (P.epi_bufs < 0 || P.epi_bufs > 2) fail("astat staging", 100, C, 2, p, bn);
+                    if (P.b_slot_bytes != kAsWTiles * (bn / 2) * 128) fail("astat slot", 100, C, 2, p, bn);
                     if ((size_t)P.a_offset < (size_t)P.nb * P.b_slot_bytes || P.a_offset %% 1024) fail("astat A offset", 100, C, 2, p, bn);
-                    if ((size_t)P.epi_offset < (size_t)P.a_offset + (size_t)(h.Kh / 8) * 2048 || P.epi_offset %% 1024)
+                    if ((size_t)P.epi_offset < (size_t)P.a_offset + (size_t)((h.Kh + 63) / 64) * kAsTileBytes ||
+                        P.epi_offset %% 1024)
                         fail("astat staging offset", 100, C, 2, p, bn);
                     if ((size_t)P.bar_offset < (size_t)P.epi_offset + 4 * P.epi_bufs * box || P.bar_offset %% 8)
                         fail("astat barrier offset", 100, C, 2, p, bn);
                     if ((size_t)P.bar_offset + bars + 1024 > total) fail("astat barriers in bounds", 100, C, 2, p, bn);
-                    if (P.num_ksteps * 16 != h.Kh || P.n_achunks * kAsChunkKs < P.num_ksteps ||
-                        (P.n_achunks - 1) * kAsChunkKs >= P.num_ksteps || P.n_achunks > kAsMaxChunks)
-                        fail("astat chunks", 100, C, 2, p, bn);
-                    if (64 * P.n_b_stages != h.Kw || 2 * P.n_b_stages < P.num_ksteps || P.cpp != C * p * p)
+                    {   /* chunks of 8 segments = p/2 k-steps: the MMA's and the producers' counts agree */
+                        const int cks = kAsChunkSegs * p / 16;
+                        if (P.num_ksteps * 16 != h.Kh || cks < 1 || P.n_achunks > kAsMaxChunks ||
+                            P.n_achunks != (C * p + kAsChunkSegs - 1) / kAsChunkSegs ||
+                            P.n_achunks != (P.num_ksteps + cks - 1) / cks)
+                            fail("astat chunks", 100, C, 2, p, bn);
+                    }
+                    /* stage j loads weight tiles 2j, 2j + 1 (k-steps 4j .. 4j + 3); the last
+                       tile any stage loads lies inside the packed weight's Kw columns */
+                    if (P.n_b_stages != (h.Kh + 63) / 64 || 4 * P.n_b_stages < P.num_ksteps || P.cpp != C * p * p ||
+                        64 * (2 * (P.n_b_stages - 1) + ((P.num_ksteps - 4 * (P.n_b_stages - 1)) >= 3 ? 2 : 1)) > h.Kw)
                         fail("astat weight stages", 100, C, 2, p, bn);
                 }
         }

@@ -581,25 +581,29 @@ int env_int(const char *name, int dflt) {
 // the resident A does not fit beside a ring of two weight stages.
 // PE_ASTAT_NB / PE_ASTAT_EPIBUFS pin the ring depth / staging boxes.
 size_t plan_astat(const pe_handle *h, FwdParams &P) {
-    if (P.Kh % 16 != 0 || P.Kh > 16 * kAsChunkKs * kAsMaxChunks) return 0;
+    if (P.Kh % 16 != 0 || (P.P & 1)) return 0;
     P.num_ksteps = P.Kh / 16;
-    P.n_achunks = (P.num_ksteps + kAsChunkKs - 1) / kAsChunkKs;
+    P.n_achunks = (P.C * P.P + kAsChunkSegs - 1) / kAsChunkSegs;   // chunks of 8 segments (8p columns)
+    const int cks = kAsChunkSegs * P.P / 16;                          // k-steps per chunk
+    if (P.n_achunks > kAsMaxChunks || cks < 1 || (P.num_ksteps + cks - 1) / cks != P.n_achunks) return 0;
     P.cpp = P.C * P.P * P.P;
-    P.n_b_stages = (P.Kh + 31) / 32;           // slice-interleaved tiles: two k-steps of both slices each
-    P.b_slot_bytes = (P.bn / 2) * 128;          // this CTA's half of one 64-column tile
+    P.n_b_stages = (P.Kh + 63) / 64;           // 2 slice-interleaved tiles (4 k-steps of both slices) per stage
+    P.b_slot_bytes = kAsWTiles * (P.bn / 2) * 128;   // this CTA's half of the stage's tiles
     P.ksub = 1;
-    const size_t a_bytes = (size_t)(P.Kh / 8) * 2048;
+    const size_t a_bytes = (size_t)((P.Kh + 63) / 64) * kAsTileBytes;   // 64-column swizzled tiles
     const size_t box = P.out_f32 ? 4096 : 2048;
     auto up = [](size_t v) { return (v + 1023) / 1024 * 1024; };
     auto bars = [&](int nb) { return (size_t)(2 * nb + 2 * P.n_achunks + 5) * 8 + (size_t)(2 * nb + 2) * 4; };
     auto total = [&](int nb, int bufs) {
         return 1024 + up((size_t)nb * P.b_slot_bytes) + up(a_bytes) + 4 * (size_t)bufs * box + bars(nb);
     };
-    const int nb_pin = env_int("PE_ASTAT_NB", 0), bufs_pin = env_int("PE_ASTAT_EPIBUFS", 0);
+    const int nb_pin = env_int("PE_ASTAT_NB", 0), bufs_pin = env_int("PE_ASTAT_EPIBUFS", -1);
+    // staging boxes (TMA stores) when they fit beside two weight stages; else
+    // the epilogue stores straight from registers (bufs = 0)
     for (int nb = 8; nb >= 2; --nb) {
         if (nb_pin && nb != nb_pin) continue;
-        for (int bufs = 2; bufs >= 1; --bufs) {
-            if (bufs_pin && bufs != bufs_pin) continue;
+        for (int bufs = 2; bufs >= 0; --bufs) {
+            if (bufs_pin >= 0 && bufs != bufs_pin) continue;
             const size_t t = total(nb, bufs);
             if (t > (size_t)h->smem_optin) continue;
             P.nb = nb;
@@ -651,6 +655,7 @@ pe_status run_frames_astat(pe_handle *h, FwdParams &P, void *out, cudaStream_t s
     if (smem == 0) return PE_ERR_UNSUPPORTED;
     const uint64_t wl = (uint64_t)env_int("PE_TEST_WAIT_NS", 0);
     P.wait_ns = wl;
+    P.out = out;
     CUtensorMap to;
     if (!make_out_tmap(&to, out, P.out_f32, P.N, P.E)) return PE_ERR_CUDA;
     const CUtensorMap &tw = h->tmap_wi[bn_index(P.bn)];
@@ -675,12 +680,13 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
         return run_frames_staged(h, P, out, all_scaled, true, st, true);
     }
-    // Single images: one resident-A launch (PE_FRAMES_PATH=staged|streamed|fused
-    // selects another path instead).
+    // Single images: the resident-A kernel when asked for (PE_FRAMES_PATH=astat)
+    // and for the allocation-free call (it needs no workspace); otherwise the
+    // staged pair, which measured faster on B200 (the resident A leaves the
+    // weight ring too little shared memory to hide its latency).
     const char *fp = std::getenv("PE_FRAMES_PATH");
-    const bool other = fp && (std::strcmp(fp, "staged") == 0 || std::strcmp(fp, "streamed") == 0 ||
-                              std::strcmp(fp, "fused") == 0);
-    if (!other && astat_eligible(h, P, f_dt)) {
+    const bool want_astat = (fp && std::strcmp(fp, "astat") == 0) || !allow_staged;
+    if (want_astat && astat_eligible(h, P, f_dt)) {
         FwdParams A = P;
         const pe_status sa = run_frames_astat(h, A, out, st);
         if (sa != PE_ERR_UNSUPPORTED) return sa;

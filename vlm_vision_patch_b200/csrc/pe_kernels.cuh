@@ -121,8 +121,9 @@ struct FwdParams {
     int32_t n_mblocks;
     // pe_astat_kernel (resident A)
     int32_t a_offset, bar_offset;     // shared-memory offsets of the resident A and of the barriers
-    int32_t n_achunks;                // A chunks of kAsChunkKs k-steps
-    int32_t epi_bufs;                 // staging boxes per epilogue warp
+    int32_t n_achunks;                // A chunks of 8 image-row segments (p/2 k-steps)
+    int32_t epi_bufs;                 // staging boxes per epilogue warp (0: stores straight from registers)
+    void *out;                        // [N, E] output (the direct-store epilogue)
     int32_t cpp;                      // C*p*p: columns of one temporal slice
     uint64_t wait_ns;                 // pipeline wait limit in ns (0: kWaitTimeoutNs)
 };
