@@ -66,7 +66,9 @@ typedef enum {
     PE_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed                    */
     PE_ERR_UNSUPPORTED = 7,    /* valid request outside what the kernels implement     */
     PE_ERR_DEVICE_TIMEOUT = 8, /* a kernel gave up waiting on its pipeline (bounded wait) */
-    PE_ERR_HOST_MEMORY = 9     /* a host allocation (item table, chunk plan) failed    */
+    PE_ERR_HOST_MEMORY = 9,    /* a host allocation (item table, chunk plan) failed    */
+    PE_ERR_DEVICE_BOUNDS = 10  /* the bounds-checking debug build found a kernel index
+                                  outside its buffer (the access was skipped)          */
 } pe_status;
 
 typedef enum { PE_F32 = 0, PE_BF16 = 1 } pe_dtype;

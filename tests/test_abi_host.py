@@ -61,12 +61,12 @@ def test_build_tracks_every_source():
 def test_status_strings(lib):
     from vlm_vision_patch_b200 import _binding
     seen = set()
-    for code in range(10):
+    for code in range(11):
         s = _binding.status_string(code)
         assert s and s != "unknown status"
         seen.add(s)
-    assert len(seen) == 10
-    assert set(_binding.STATUS) == set(range(10))
+    assert len(seen) == 11
+    assert set(_binding.STATUS) == set(range(11))
     assert _binding.status_string(99) == "unknown status"
 
 

@@ -12,13 +12,15 @@ import os
 from typing import Optional, Sequence
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpe.so")
+# PE_LIB selects another build of the same library (the bounds-checking
+# libpe_debug.so); by default the in-tree libpe.so
+LIB_PATH = os.environ.get("PE_LIB") or os.path.join(HERE, "libpe.so")
 
 PE_F32, PE_BF16 = 0, 1
 STATUS = {
     0: "PE_OK", 1: "PE_ERR_INVALID_ARG", 2: "PE_ERR_SHAPE", 3: "PE_ERR_DTYPE",
     4: "PE_ERR_ALIGN", 5: "PE_ERR_NO_WEIGHT", 6: "PE_ERR_CUDA", 7: "PE_ERR_UNSUPPORTED",
-    8: "PE_ERR_DEVICE_TIMEOUT", 9: "PE_ERR_HOST_MEMORY",
+    8: "PE_ERR_DEVICE_TIMEOUT", 9: "PE_ERR_HOST_MEMORY", 10: "PE_ERR_DEVICE_BOUNDS",
 }
 PE_INLINE_ITEMS = 16
 PE_MAX_PATCH = 32

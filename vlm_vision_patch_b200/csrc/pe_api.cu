@@ -752,6 +752,7 @@ const char *pe_status_string(pe_status s) {
         case PE_ERR_UNSUPPORTED: return "unsupported configuration";
         case PE_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
         case PE_ERR_HOST_MEMORY: return "host memory allocation failed";
+        case PE_ERR_DEVICE_BOUNDS: return "a kernel index fell outside its buffer (bounds-checking build)";
     }
     return "unknown status";
 }

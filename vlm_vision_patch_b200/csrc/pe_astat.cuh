@@ -110,9 +110,11 @@ __device__ __forceinline__ void as_emit(const FwdParams &P, const CUtensorMap *t
             const int c0 = col0 + q * (P.pos_f32 ? 4 : 8);
             if (q < nq && r < P.N && c0 < P.E) {
                 const char *a = reinterpret_cast<const char *>(P.pos) + (r * P.E + c0) * (int64_t)(P.pos_f32 ? 4 : 2);
-                asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
-                             : "l"(a));
+                const char *plo = reinterpret_cast<const char *>(P.pos);
+                if (PE_IN(a, 16, plo, plo + P.N * (int64_t)P.E * (P.pos_f32 ? 4 : 2), P.err))
+                    asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
+                                 : "l"(a));
             }
         }
     }
@@ -177,6 +179,10 @@ __device__ __forceinline__ void as_emit_direct(const FwdParams &P, const uint32_
                                                int lane) {
     const int64_t r = row0 + lane;
     if (r >= P.N || col0 >= P.E) return;
+    const int osz = P.out_f32 ? 4 : 2;
+    const char *olo = static_cast<const char *>(P.out), *ohi = olo + P.N * (int64_t)P.E * osz;
+    const char *plo = static_cast<const char *>(P.pos), *phi = plo + P.N * (int64_t)P.E * (P.pos_f32 ? 4 : 2);
+    (void)olo; (void)ohi; (void)plo; (void)phi;
     float f[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
@@ -191,6 +197,7 @@ __device__ __forceinline__ void as_emit_direct(const FwdParams &P, const uint32_
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 if (col0 + 4 * q >= P.E) break;
+                if (!PE_IN(pr + q, 16, plo, phi, P.err)) continue;
                 const float4 a = __ldg(pr + q);
                 f[4 * q] += a.x; f[4 * q + 1] += a.y; f[4 * q + 2] += a.z; f[4 * q + 3] += a.w;
             }
@@ -199,6 +206,7 @@ __device__ __forceinline__ void as_emit_direct(const FwdParams &P, const uint32_
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 if (col0 + 8 * q >= P.E) break;
+                if (!PE_IN(pr + q, 16, plo, phi, P.err)) continue;
                 const uint4 a = __ldg(pr + q);
                 const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
@@ -213,14 +221,14 @@ __device__ __forceinline__ void as_emit_direct(const FwdParams &P, const uint32_
         float *o = reinterpret_cast<float *>(P.out) + r * P.E + col0;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-            if (col0 + 4 * q < P.E)
+            if (col0 + 4 * q < P.E && PE_IN(o + 4 * q, 16, olo, ohi, P.err))
                 st_global_v4(o + 4 * q, __float_as_uint(f[4 * q]), __float_as_uint(f[4 * q + 1]),
                              __float_as_uint(f[4 * q + 2]), __float_as_uint(f[4 * q + 3]));
     } else {
         uint16_t *o = reinterpret_cast<uint16_t *>(P.out) + r * P.E + col0;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            if (col0 + 8 * q < P.E)
+            if (col0 + 8 * q < P.E && PE_IN(o + 8 * q, 16, olo, ohi, P.err))
                 st_global_v4(o + 8 * q, pack_bf16x2(f[8 * q], f[8 * q + 1]), pack_bf16x2(f[8 * q + 2], f[8 * q + 3]),
                              pack_bf16x2(f[8 * q + 4], f[8 * q + 5]), pack_bf16x2(f[8 * q + 6], f[8 * q + 7]));
     }
@@ -274,6 +282,7 @@ __device__ __forceinline__ void as_produce(const FwdParams &P, uint8_t *a_buf, u
         jw2[v] = 2 * jw;
     }
     const char *src[MAXIT];
+    const char *dlo[MAXIT], *dhi[MAXIT];   // frame buffers (bounds-checking build)
     int32_t sW[MAXIT], sHW[MAXIT];   // bytes
     uint32_t raw[2][kAsStageSegs][MAXIT];
 
@@ -282,9 +291,12 @@ __device__ __forceinline__ void as_produce(const FwdParams &P, uint8_t *a_buf, u
         for (int v = 0; v < MAXIT; ++v) {
             const int64_t R = (int64_t)mb * (2 * kBM) + rank * kBM + rr[v];
             sp[v] = nullptr;
+            dlo[v] = dhi[v] = nullptr;
             w[v] = hw[v] = 0;
             if (uok[v] && R < P.N) {
                 const RowSrc rs = locate_row(P, R, 2);
+                dlo[v] = rs.lo;
+                dhi[v] = rs.hi;
                 sp[v] = rs.base + jw2[v] * 2;
                 w[v] = rs.W * 2;
                 hw[v] = rs.HW * 2;
@@ -322,7 +334,8 @@ __device__ __forceinline__ void as_produce(const FwdParams &P, uint8_t *a_buf, u
                 raw[b][qq][v] = 0u;
                 if (seg < nseg && src[v]) {
                     const char *a = src[v] + (int64_t)c * sHW[v] + (int64_t)i * sW[v];
-                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][v]) : "l"(a));
+                    if (PE_IN(a, 4, dlo[v], dhi[v], P.err))
+                        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][v]) : "l"(a));
                 }
             }
         }

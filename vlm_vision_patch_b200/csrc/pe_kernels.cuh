@@ -128,6 +128,30 @@ struct FwdParams {
     uint64_t wait_ns;                 // pipeline wait limit in ns (0: kWaitTimeoutNs)
 };
 
+// ------------------------------------------------------------ debug bounds
+//
+// Built with -DPE_DEBUG_BOUNDS (libpe_debug.so, vlm_vision_patch_b200.build
+// --debug-bounds): each data-dependent global access of the kernels (pixel
+// gathers through the item table, streamed patch-row stores, position-table
+// loads, register-to-global output stores) first checks that its address
+// range lies inside the buffer it indexes.  An access outside records
+// PE_ERR_DEVICE_BOUNDS in the kernel's error word and is skipped (a load
+// reads zero).  TMA accesses are range-checked by the hardware against their
+// tensor maps; the elementwise kernels index inside their own loop bounds.
+// Without the macro PE_IN is the constant true and the checks compile to
+// nothing.
+#ifdef PE_DEBUG_BOUNDS
+__device__ __forceinline__ bool dbg_in(const void *a, int64_t bytes, const void *lo, const void *hi, int *err) {
+    const char *q = static_cast<const char *>(a);
+    if (q >= static_cast<const char *>(lo) && q + bytes <= static_cast<const char *>(hi)) return true;
+    if (err) atomicExch(err, (int)PE_ERR_DEVICE_BOUNDS);
+    return false;
+}
+#define PE_IN(a, n, lo, hi, err) ::pe::dbg_in((a), (n), (lo), (hi), (err))
+#else
+#define PE_IN(a, n, lo, hi, err) ((void)(lo), (void)(hi), true)
+#endif
+
 // ------------------------------------------------------------ row decoding
 
 __device__ __forceinline__ const ItemDesc &item_at(const FwdParams &P, int i) {
@@ -153,6 +177,7 @@ struct RowSrc {
     int32_t HW;         // elements per channel plane
     int32_t CHW;        // elements per frame
     int32_t tmax;       // last usable temporal offset: min(t, tmax) frames past tau0
+    const char *lo, *hi;  // the item's frame buffer (filled in the bounds-checking build only)
 };
 
 __device__ __forceinline__ RowSrc locate_row(const FwdParams &P, int64_t R, int esize) {
@@ -183,6 +208,11 @@ __device__ __forceinline__ RowSrc locate_row(const FwdParams &P, int64_t R, int 
     s.tmax = (int32_t)(it.T - 1 - tau0);
     const int64_t el = (tau0 * P.C * it.H + g_h * P.P) * (int64_t)it.W + g_w * P.P;
     s.base = reinterpret_cast<const char *>(it.frames) + el * esize;
+    s.lo = s.hi = nullptr;
+#ifdef PE_DEBUG_BOUNDS
+    s.lo = reinterpret_cast<const char *>(it.frames);
+    s.hi = s.lo + (int64_t)it.T * P.C * it.H * it.W * esize;
+#endif
     return s;
 }
 
@@ -256,16 +286,18 @@ __device__ __forceinline__ uint32_t norm_pair_bf16(uint32_t w, const NormConst &
 template <bool F32IN> struct PixPair;
 template <> struct PixPair<false> {
     uint32_t w;
-    __device__ __forceinline__ void load(const char *p) {
-        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w) : "l"(p));
+    __device__ __forceinline__ void load(const char *p, const char *lo, const char *hi, int *err) {
+        w = 0u;
+        if (PE_IN(p, 4, lo, hi, err)) asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w) : "l"(p));
     }
     __device__ __forceinline__ void zero() { w = 0u; }
     __device__ __forceinline__ uint32_t norm(const NormConst &n) const { return norm_pair_bf16(w, n); }
 };
 template <> struct PixPair<true> {
     float a, b;
-    __device__ __forceinline__ void load(const char *p) {
-        asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "l"(p));
+    __device__ __forceinline__ void load(const char *p, const char *lo, const char *hi, int *err) {
+        a = b = 0.f;
+        if (PE_IN(p, 8, lo, hi, err)) asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "l"(p));
     }
     __device__ __forceinline__ void zero() { a = b = 0.f; }
     __device__ __forceinline__ uint32_t norm(const NormConst &n) const { return norm_pair_f32(a, b, n); }
@@ -372,6 +404,7 @@ __device__ __forceinline__ void produce_frames_reg(const FwdParams &P, const Pro
 
     // load side: row sources of the tile being loaded
     const char *src[MAXIT];
+    const char *dlo[MAXIT], *dhi[MAXIT];          // frame buffers (bounds-checking build)
     int32_t sW[MAXIT], sHW[MAXIT], sT1[MAXIT];   // sT1: byte offset of the t = 1 slice (0: same frame)
     int ld_lt = 0, ld_s = 0;
     uint32_t rokb[2] = {0u, 0u}, dupb[2] = {0u, 0u};
@@ -391,6 +424,8 @@ __device__ __forceinline__ void produce_frames_reg(const FwdParams &P, const Pro
                 if (!(uok[v] && m0 + rr[v] < P.N)) continue;
                 const RowSrc rs = locate_row(P, m0 + rr[v], 2);
                 src[v] = rs.base + (int64_t)kw[v] * 2;
+                dlo[v] = rs.lo;
+                dhi[v] = rs.hi;
                 sW[v] = rs.W * 2;
                 sHW[v] = rs.HW * 2;
                 sT1[v] = rs.tmax > 0 ? rs.CHW * 2 : 0;
@@ -413,9 +448,10 @@ __device__ __forceinline__ void produce_frames_reg(const FwdParams &P, const Pro
                 for (int t = 0; t < NT; ++t) raw[b][qq][t][v] = 0u;
                 if (ci < nci && (rokb[b] >> v & 1u)) {
                     const char *a = src[v] + (int64_t)c * sHW[v] + (int64_t)i * sW[v];
-                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][0][v]) : "l"(a));
+                    if (PE_IN(a, 4, dlo[v], dhi[v], P.err))
+                        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][0][v]) : "l"(a));
                     if constexpr (!DUPALL) {
-                        if (sT1[v] != 0)
+                        if (sT1[v] != 0 && PE_IN(a + sT1[v], 4, dlo[v], dhi[v], P.err))
                             asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][qq][NT - 1][v]) : "l"(a + sT1[v]));
                     }
                 }
@@ -514,16 +550,20 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, const ProdCtx
         const int uW = itd.W, uHW = itd.H * itd.W;
 
         const char *src[MAXIT];
+        const char *dlo[MAXIT], *dhi[MAXIT];     // frame buffers (bounds-checking build)
         int32_t sW[MAXIT], sHW[MAXIT], sCHW[MAXIT], sTm[MAXIT];
         bool rok[MAXIT];
 #pragma unroll
         for (int v = 0; v < MAXIT; ++v) {
             rok[v] = uok[v] && (m0 + rr[v] < P.N);
             src[v] = nullptr;
+            dlo[v] = dhi[v] = nullptr;
             sW[v] = sHW[v] = sCHW[v] = sTm[v] = 0;
             if (rok[v]) {
                 const RowSrc s = locate_row(P, m0 + rr[v], esize);
                 src[v] = s.base + (int64_t)kw[v] * esize;
+                dlo[v] = s.lo;
+                dhi[v] = s.hi;
                 sW[v] = s.W;
                 sHW[v] = s.HW;
                 sCHW[v] = s.CHW;
@@ -548,10 +588,10 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, const ProdCtx
                         px[qq][0][v].zero();
                         px[qq][1][v].zero();
                         if (live && rok[v]) {
-                            px[qq][0][v].load(src[v] + uoff);
+                            px[qq][0][v].load(src[v] + uoff, dlo[v], dhi[v], P.err);
                             if (!dup) {
                                 const int64_t t1 = (sTm[v] > 0 ? (int64_t)sCHW[v] : 0) * esize;
-                                px[qq][1][v].load(src[v] + uoff + t1);
+                                px[qq][1][v].load(src[v] + uoff + t1, dlo[v], dhi[v], P.err);
                             }
                         }
                     }
@@ -586,7 +626,7 @@ __device__ __forceinline__ void produce_frames(const FwdParams &P, const ProdCtx
                         if (live && rok[v]) {
                             const int tt = t < sTm[v] ? t : sTm[v];
                             const int64_t off = (int64_t)tt * sCHW[v] + (int64_t)cc * sHW[v] + (int64_t)ii * sW[v];
-                            px[q][v].load(src[v] + off * esize);
+                            px[q][v].load(src[v] + off * esize, dlo[v], dhi[v], P.err);
                         }
                     }
                 }
@@ -781,10 +821,13 @@ __device__ __forceinline__ void produce_rows_stream(const FwdParams &P, int pw, 
             const int64_t row = (int64_t)m * (2 * kBM) + (it & 7) * 32 + lane;
             const bool live = row < P.N;
             const char *base0 = nullptr, *base1 = nullptr;
+            const char *dlo = nullptr, *dhi = nullptr;   // frame buffer (bounds-checking build)
             int sW = 0, sHW = 0;
             uint16_t *dst = P.a_rows;
             if (live) {
                 const RowSrc rs = locate_row(P, row, 2);
+                dlo = rs.lo;
+                dhi = rs.hi;
                 base0 = rs.base;
                 base1 = rs.tmax > 0 ? rs.base + (int64_t)rs.CHW * 2 : rs.base;
                 sW = rs.W * 2;
@@ -814,10 +857,13 @@ __device__ __forceinline__ void produce_rows_stream(const FwdParams &P, int pw, 
                     const char *s2 = bt + (int64_t)c2 * sHW + (int64_t)i2 * sW;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        if (2 * k < n1)
-                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[u][k]) : "l"(s1 + 4 * k));
-                        else if (c2 < C)
-                            asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[u][k]) : "l"(s2 + (2 * k - n1) * 2));
+                        if (2 * k < n1) {
+                            if (PE_IN(s1 + 4 * k, 4, dlo, dhi, P.err))
+                                asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[u][k]) : "l"(s1 + 4 * k));
+                        } else if (c2 < C) {
+                            if (PE_IN(s2 + (2 * k - n1) * 2, 4, dlo, dhi, P.err))
+                                asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[u][k]) : "l"(s2 + (2 * k - n1) * 2));
+                        }
                     }
                 }
 #pragma unroll
@@ -837,7 +883,8 @@ __device__ __forceinline__ void produce_rows_stream(const FwdParams &P, int pw, 
                             else if (c + 1 < C) w[u][k] = norm_word<NORM>(w[u][k], n2c);
                         }
                     }
-                    st_global_v4(dst + col[u], w[u][0], w[u][1], w[u][2], w[u][3]);
+                    if (PE_IN(dst + col[u], 16, P.a_rows, P.a_rows + P.N * (int64_t)row_elems, P.err))
+                        st_global_v4(dst + col[u], w[u][0], w[u][1], w[u][2], w[u][3]);
                 }
             }
         }
@@ -1120,9 +1167,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     if (q < nq && r < P.N && c0 < P.E) {
                         const char *a = reinterpret_cast<const char *>(P.pos) +
                                         (r * P.E + c0) * (int64_t)(P.pos_f32 ? 4 : 2);
-                        asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
-                                     : "l"(a));
+                        const char *plo = reinterpret_cast<const char *>(P.pos);
+                        if (PE_IN(a, 16, plo, plo + P.N * (int64_t)P.E * (P.pos_f32 ? 4 : 2), P.err))
+                            asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
+                                         : "l"(a));
                     }
                 }
             }
@@ -1370,6 +1419,7 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
         const char *src = rs.base + 4 * jw;
         const int sW = rs.W * 2, sHW = rs.HW * 2;
         const int sT1 = (!SHARED && rs.tmax > 0) ? rs.CHW * 2 : 0;
+        const char *dlo = rs.lo, *dhi = rs.hi;   // frame buffer (bounds-checking build)
         // One channel (p image rows, every temporal slice) per register buffer;
         // the loads of channel c + 1 are in flight while channel c is stored.
         uint32_t raw[2][NT][p];
@@ -1377,10 +1427,12 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
             const char *a = src + (int64_t)c * sHW;
 #pragma unroll
             for (int i = 0; i < p; ++i) {
-                asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][0][i]) : "l"(a + (int64_t)i * sW));
+                raw[b][0][i] = 0u;
+                if (PE_IN(a + (int64_t)i * sW, 4, dlo, dhi, P.err))
+                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(raw[b][0][i]) : "l"(a + (int64_t)i * sW));
                 if constexpr (!SHARED) {
                     raw[b][NT - 1][i] = 0u;
-                    if (sT1 != 0)
+                    if (sT1 != 0 && PE_IN(a + (int64_t)i * sW + sT1, 4, dlo, dhi, P.err))
                         asm volatile("ld.global.nc.b32 %0, [%1];"
                                      : "=r"(raw[b][NT - 1][i]) : "l"(a + (int64_t)i * sW + sT1));
                 }
@@ -1410,8 +1462,11 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
                 if (c >= C) break;
                 const char *a = src + (int64_t)c * sHW;
 #pragma unroll
-                for (int i = 0; i < p; ++i)
-                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(all[c][i]) : "l"(a + (int64_t)i * sW));
+                for (int i = 0; i < p; ++i) {
+                    all[c][i] = 0u;
+                    if (PE_IN(a + (int64_t)i * sW, 4, dlo, dhi, P.err))
+                        asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(all[c][i]) : "l"(a + (int64_t)i * sW));
+                }
             }
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -1558,7 +1613,7 @@ __global__ void pe_patchify_kernel(const __grid_constant__ FwdParams P, void *ro
         const int tt = t < s.tmax ? t : s.tmax;
         const int64_t off = (int64_t)tt * s.CHW + (int64_t)c * s.HW + (int64_t)i * s.W + 2 * jw;
         PixPair<F32IN> px;
-        px.load(s.base + off * esize);
+        px.load(s.base + off * esize, s.lo, s.hi, P.err);
         const uint32_t w = px.norm(norm_const(P, c));
         const int64_t k = 2 * (int64_t)wk;
         if (rows_f32) {
