@@ -293,26 +293,73 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ our arm
 
-def library_context(wl, dev, flush_buf, reps=20):
-    """cuBLAS (torch.nn.functional.linear, bf16) on the same [N, K] x [E, K]^T
-    contraction, timed like the steps (L2 flushed, CUDA events): context for
-    the contraction kernel's number, not part of the path."""
-    x = torch.randn(wl.N, wl.K, device=dev).to(torch.bfloat16)
-    w = torch.randn(wl.E, wl.K, device=dev).to(torch.bfloat16) * 0.02
+def torch_patch_rows(frames, grid, merge, mean, std, tp, p):
+    """Normalised patch rows [N, C*tp*p*p] (bf16) of one [T, C, H, W] item in
+    output-row order, written with torch tensor ops: the frames padded to
+    tp*g_t by repeating the last one, bf16(fp32(fp32(x - mean) / std)) per
+    channel, then a view/permute to (g_t, window row, window column, dh, dw)
+    rows of (c, t, i, j) columns (raster rows for merge 1).  The eager-torch
+    form of the path, timed as context only."""
+    T, C, H, W = frames.shape
+    gt, gh, gw = (int(v) for v in grid)
+    idx = torch.clamp(torch.arange(gt * tp, device=frames.device), max=T - 1)
+    f = frames[idx].float()
+    mu = torch.tensor(mean, dtype=torch.float32, device=frames.device).view(1, C, 1, 1)
+    sd = torch.tensor(std, dtype=torch.float32, device=frames.device).view(1, C, 1, 1)
+    f = ((f - mu) / sd).to(torch.bfloat16)
+    m = merge
+    f = f.view(gt, tp, C, gh // m, m, p, gw // m, m, p)
+    # -> (gt, gh/m, gw/m, dh, dw, C, tp, i, j)
+    f = f.permute(0, 3, 6, 4, 7, 2, 1, 5, 8)
+    return f.reshape(gt * gh * gw, C * tp * p * p)
+
+
+def _event_ms(fn, flush_buf, dev, reps):
     for _ in range(3):
-        torch.nn.functional.linear(x, w)
+        fn()
     ts = []
     for _ in range(reps):
         flush_buf.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        torch.nn.functional.linear(x, w)
+        fn()
         b.record()
         torch.cuda.synchronize(dev)
         ts.append(a.elapsed_time(b))
-    ms = statistics.median(ts)
-    return {"cublas_linear_bf16": {"ms": ms, "tflops": 2.0 * wl.N * wl.K * wl.E / (ms / 1e3) / 1e12,
-                                   "shape": [wl.N, wl.K, wl.E]}}
+    return statistics.median(ts)
+
+
+def library_context(wl, dev, flush_buf, reps=20):
+    """Library and eager-torch forms of the same work, timed like the steps
+    (L2 flushed, CUDA events): context for the path's numbers, not part of it.
+      cublas_linear_bf16   torch.nn.functional.linear on [N, K] x [E, K]^T
+      cudnn_conv3d_bf16    torch.nn.functional.conv3d on the rows viewed as
+                           [N, C, tp, p, p] against the [E, C, tp, p, p] weight
+      torch_frames_bf16    frames workloads: torch_patch_rows per item, cat,
+                           then linear (+ bias): raw frames to embeddings"""
+    flop = 2.0 * wl.N * wl.K * wl.E
+    x = torch.randn(wl.N, wl.K, device=dev).to(torch.bfloat16)
+    w = torch.randn(wl.E, wl.K, device=dev).to(torch.bfloat16) * 0.02
+    ctx = {}
+    ms = _event_ms(lambda: torch.nn.functional.linear(x, w), flush_buf, dev, reps)
+    ctx["cublas_linear_bf16"] = {"ms": ms, "tflops": flop / (ms / 1e3) / 1e12, "shape": [wl.N, wl.K, wl.E]}
+    x5 = x.view(wl.N, wl.C, wl.tp, wl.p, wl.p)
+    w5 = w.view(wl.E, wl.C, wl.tp, wl.p, wl.p)
+    ms = _event_ms(lambda: torch.nn.functional.conv3d(x5, w5, stride=(wl.tp, wl.p, wl.p)), flush_buf, dev, reps)
+    ctx["cudnn_conv3d_bf16"] = {"ms": ms, "tflops": flop / (ms / 1e3) / 1e12}
+    if wl.patches is None:
+        frames = [it.frames.to(dev) for it in wl.items]
+        wt = wl.weight.to(dev).to(torch.bfloat16).reshape(wl.E, wl.K)
+        bias = None if wl.bias is None else wl.bias.to(dev).to(torch.bfloat16)
+
+        def eager():
+            rows = torch.cat([torch_patch_rows(f, it.grid, wl.merge, wl.mean, wl.std, wl.tp, wl.p)
+                              for f, it in zip(frames, wl.items)])
+            return torch.nn.functional.linear(rows, wt, bias)
+        ms = _event_ms(eager, flush_buf, dev, reps)
+        ctx["torch_frames_bf16"] = {"ms": ms, "patches_per_s": wl.N / (ms / 1e3), "tflops": flop / (ms / 1e3) / 1e12}
+        del frames
+    return ctx
 
 
 E2E_PATHS = {"host": "pe_forward_frames_grouped_host / pe_forward_patches_host (C ABI, host buffers): chunked "

@@ -138,3 +138,20 @@ def test_reference_arm_for_tf32_times_the_fp32_form():
                            "--steps", "1", "--warmup", "3"]) == 0
     line = json.loads(buf.getvalue().strip())
     assert line["value"] > 0 and "unrounded fp32" in line["cpu_baseline"]["sample"]
+
+
+@pytest.mark.parametrize("T,gh,gw,merge,tp,p", [(1, 4, 6, 2, 2, 14), (3, 2, 4, 2, 2, 4), (5, 6, 2, 2, 2, 3),
+                                                 (2, 3, 5, 1, 2, 2), (4, 2, 2, 2, 1, 6)])
+def test_eager_torch_rows_match_the_oracle_patchify(T, gh, gw, merge, tp, p):
+    """The eager-torch context form of the path builds the oracle's rows bit
+    for bit (normalisation, temporal padding, merge order)."""
+    import numpy as np
+    import oracle
+    import workloads
+    C = 3
+    frames = workloads.uniform01((T, C, gh * p, gw * p), 77 + T)
+    grid = (-(-T // tp), gh, gw)
+    got = bench.torch_patch_rows(frames, grid, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, tp, p)
+    ref = oracle.patchify(frames, grid, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, C, tp, p)
+    assert got.dtype == torch.bfloat16
+    assert np.array_equal(got.float().numpy().view(np.uint32), ref.view(np.uint32))
