@@ -58,6 +58,7 @@ FRAME_CASES = {
     "fused_p8": ("fused", [(2, 6, 8), (1, 4, 4)], 8, 256, False, torch.bfloat16, torch.bfloat16, False, {}),
     "streamed_video": ("streamed", [(4, 6, 10), (3, 4, 8), (1, 10, 6)], 14, 1280, True, torch.bfloat16,
                        torch.bfloat16, False, {}),
+    "fused_p32": ("fused", [(3, 2, 4), (1, 4, 2)], 32, 128, True, torch.bfloat16, torch.float32, True, {}),
     "many_items": ("staged", [(1 + (i % 3), 2 + 2 * (i % 4), 2 + 2 * (i % 5)) for i in range(40)], 14, 256,
                    True, torch.bfloat16, torch.bfloat16, True, {}),
 }
@@ -95,6 +96,23 @@ def run_patches():
     return {"out": out.cpu()}, pe.last_error()
 
 
+def run_patches_edges():
+    """The largest K (C = 4, p = 32: 8192) and the largest E (65528) the ABI takes."""
+    res = {}
+    err = 0
+    for C, tp, p, E, N in ((4, 2, 32, 256, 300), (3, 2, 2, 65528, 130)):
+        K = C * tp * p * p
+        pe = PatchEmbed(E, C, tp, p, True)
+        pe.set_weight(workloads.normal((E, C, tp, p, p), 710 + p, std=0.02, dtype=torch.bfloat16).to(DEV),
+                      workloads.normal((E,), 711, std=0.02, dtype=torch.bfloat16).to(DEV))
+        x = workloads.normal((N, K), 712 + p, dtype=torch.bfloat16).to(DEV)
+        out = pe.forward_patches(x, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        res[f"K{K}_E{E}"] = out.cpu()
+        err = err or pe.last_error()
+    return res, err
+
+
 def run_merger():
     E, m, H = 256, 2, 512
     mg = PatchMerger(E, m, H)
@@ -116,6 +134,7 @@ def main(dst):
     for name in FRAME_CASES:
         res[name], errs[name] = run_frames(name)
     res["patches"], errs["patches"] = run_patches()
+    res["patches_edges"], errs["patches_edges"] = run_patches_edges()
     res["merger"], errs["merger"] = run_merger()
     torch.save({"lib": B.LIB_PATH, "out": res, "err": errs}, dst)
 
