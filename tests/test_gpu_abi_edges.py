@@ -64,3 +64,26 @@ def test_frames_p32(T, gh, gw, merge, E):
     assert pe.last_error() == 0
     ref, mag = oracle.conv3d_frames(frames, grid, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
     assert_within_tolerance(out, ref, mag, what=f"frames p=32 T={T} grid={grid} merge={merge}")
+
+
+@pytest.mark.parametrize("C", [1, 2, 4])
+@pytest.mark.parametrize("path", ["staged", "fused", "astat"])
+def test_frames_other_channel_counts(C, path, monkeypatch):
+    """Grayscale (C = 1), two-channel and four-channel frames (pe_create takes
+    C up to 4) through every frames path: a group of images and, for the
+    staged and fused paths, a video item; against the oracle."""
+    tp, p, E = 2, 14, 256
+    monkeypatch.setenv("PE_FRAMES_PATH", path)
+    items = [(1, 6, 8), (1, 4, 10)] if path == "astat" else [(1, 6, 8), (3, 4, 6), (1, 2, 2)]
+    frames = [workloads.uniform01((T, C, gh * p, gw * p), 920 + 7 * C + i) for i, (T, gh, gw) in enumerate(items)]
+    grids = [(-(-T // tp), gh, gw) for T, gh, gw in items]
+    w = workloads.normal((E, C, tp, p, p), 921 + C, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 922, std=0.02, dtype=torch.bfloat16)
+    mean, std = (0.5, 0.45, 0.4, 0.35)[:C], (0.25, 0.26, 0.27, 0.28)[:C]
+    pe = _pe(E, C, tp, p, w, b)
+    pe.set_norm(mean, std)
+    out = pe.forward_frames_grouped([f.to(DEV) for f in frames], grids, 2, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    ref, mag = oracle.conv3d_grouped(list(zip(frames, grids)), 2, mean, std, w, b, C, tp, p)
+    assert_within_tolerance(out, ref, mag, what=f"C={C} {path}")
