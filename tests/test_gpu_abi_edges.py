@@ -87,3 +87,22 @@ def test_frames_other_channel_counts(C, path, monkeypatch):
     assert pe.last_error() == 0
     ref, mag = oracle.conv3d_grouped(list(zip(frames, grids)), 2, mean, std, w, b, C, tp, p)
     assert_within_tolerance(out, ref, mag, what=f"C={C} {path}")
+
+
+@pytest.mark.parametrize("T,tp,p,merge", [(5, 3, 14, 2), (1, 3, 8, 2), (6, 4, 6, 1), (3, 4, 14, 2)])
+def test_frames_temporal_patch_3_and_4(T, tp, p, merge):
+    """Temporal patch sizes above 2 (pe_create takes tp up to 4) run the fused
+    frames kernel: the last frame repeated up to a multiple of tp (T = 1 with
+    tp = 3 is one image three times), against the oracle."""
+    C, E, gh, gw = 3, 192, 4, 6
+    frames = workloads.uniform01((T, C, gh * p, gw * p), 930 + T + tp)
+    w = workloads.normal((E, C, tp, p, p), 931 + tp, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 932, std=0.02, dtype=torch.bfloat16)
+    pe = _pe(E, C, tp, p, w, b)
+    pe.set_norm(workloads.CLIP_MEAN, workloads.CLIP_STD)
+    grid = (-(-T // tp), gh, gw)
+    out = pe.forward_frames(frames.to(DEV), grid, merge, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    ref, mag = oracle.conv3d_frames(frames, grid, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
+    assert_within_tolerance(out, ref, mag, what=f"tp={tp} T={T} p={p}")
