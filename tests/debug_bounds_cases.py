@@ -55,6 +55,8 @@ FRAME_CASES = {
     "fused_video": ("fused", [(4, 6, 10), (3, 4, 8), (1, 10, 6)], 14, 1280, True, torch.bfloat16,
                     torch.bfloat16, True, {}),
     "fused_f32_frames": ("fused", [(2, 6, 4), (1, 4, 6)], 14, 256, True, torch.float32, torch.float32, False, {}),
+    "staged_f32_images": ("staged", [(1, 6, 8), (1, 4, 10)], 14, 256, True, torch.float32, torch.float32, True, {}),
+    "staged_f32_video": ("staged", [(4, 6, 8), (3, 4, 6)], 14, 256, True, torch.float32, torch.bfloat16, False, {}),
     "fused_p8": ("fused", [(2, 6, 8), (1, 4, 4)], 8, 256, False, torch.bfloat16, torch.bfloat16, False, {}),
     "streamed_video": ("streamed", [(4, 6, 10), (3, 4, 8), (1, 10, 6)], 14, 1280, True, torch.bfloat16,
                        torch.bfloat16, False, {}),

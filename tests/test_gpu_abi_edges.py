@@ -106,3 +106,33 @@ def test_frames_temporal_patch_3_and_4(T, tp, p, merge):
     assert pe.last_error() == 0
     ref, mag = oracle.conv3d_frames(frames, grid, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
     assert_within_tolerance(out, ref, mag, what=f"tp={tp} T={T} p={p}")
+
+
+@pytest.mark.parametrize("items,p,merge", [([(1, 6, 8), (1, 4, 10), (1, 2, 2)], 14, 2),      # single frames
+                                           ([(4, 6, 8), (3, 4, 6), (1, 2, 4)], 14, 2),      # video rows
+                                           ([(1, 4, 6), (2, 2, 4)], 16, 1)])
+def test_fp32_frames_staged_and_fused(items, p, merge, monkeypatch):
+    """fp32 frames take the staged pair (the prepare kernel's fp32 form, two
+    launches) by default and the fused kernel when asked for; both within
+    tolerance of the oracle."""
+    from vlm_vision_patch_b200 import _binding as B
+    C, tp, E = 3, 2, 256
+    frames = [workloads.uniform01((T, C, gh * p, gw * p), 940 + i, dtype=torch.float32)
+              for i, (T, gh, gw) in enumerate(items)]
+    grids = [(-(-T // tp), gh, gw) for T, gh, gw in items]
+    w = workloads.normal((E, C, tp, p, p), 941, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 942, std=0.02, dtype=torch.bfloat16)
+    pe = _pe(E, C, tp, p, w, b)
+    pe.set_norm(workloads.CLIP_MEAN, workloads.CLIP_STD)
+    ref, mag = oracle.conv3d_grouped(list(zip(frames, grids)), merge, workloads.CLIP_MEAN, workloads.CLIP_STD,
+                                     w, b, C, tp, p)
+    dev_frames = [f.to(DEV) for f in frames]
+    for path, launches in (("staged", 2), ("fused", 1)):
+        monkeypatch.setenv("PE_FRAMES_PATH", path)
+        B.pe_profile_begin(pe.h, 0)
+        out = pe.forward_frames_grouped(dev_frames, grids, merge, out_dtype=torch.float32)
+        _, n = B.pe_profile_end(pe.h, 0)
+        torch.cuda.synchronize()
+        assert pe.last_error() == 0
+        assert n == launches, (path, n)
+        assert_within_tolerance(out, ref, mag, what=f"fp32 frames {path} p={p}")

@@ -423,7 +423,7 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
 // 59k), so it runs whenever it can: bf16 frames, tp = 2, p in {14, 16}.
 
 bool staged_eligible(const pe_handle *h, int f_dt) {
-    return f_dt == PE_BF16 && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
+    return (f_dt == PE_BF16 || f_dt == PE_F32) && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
 }
 
 // bf16 frames with tp = 2 and p in {14, 16}: 0 = fused kernel, 1 = staged
@@ -437,13 +437,13 @@ int frames_path(const pe_handle *h, int f_dt) {
     if (!staged_eligible(h, f_dt)) return 0;
     const char *e = std::getenv("PE_FRAMES_PATH");
     if (e && std::strcmp(e, "fused") == 0) return 0;
-    if (e && std::strcmp(e, "streamed") == 0) return 2;
+    if (e && std::strcmp(e, "streamed") == 0 && f_dt == PE_BF16) return 2;   // its producers read bf16 words
     return 1;
 }
 
-template <int PT, int NORM, bool SHARED>
+template <int PT, int NORM, bool SHARED, bool F32IN = false>
 cudaError_t launch_prep_rows(const FwdParams &P, uint16_t *A, int row_elems, cudaStream_t st) {
-    auto kern = pe_prep_rows_kernel<PT, NORM, SHARED>;
+    auto kern = pe_prep_rows_kernel<PT, NORM, SHARED, F32IN>;
     const int smem = kPrepRows * row_elems * 2;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -453,8 +453,11 @@ cudaError_t launch_prep_rows(const FwdParams &P, uint16_t *A, int row_elems, cud
 }
 
 template <int PT>
-cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool shared, uint16_t *A, int row_elems,
+cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool shared, bool f32, uint16_t *A, int row_elems,
                         cudaStream_t st) {
+    if (f32)   // fp32 frames: the normalisation mode is read per channel
+        return shared ? launch_prep_rows<PT, 2, true, true>(P, A, row_elems, st)
+                      : launch_prep_rows<PT, 2, false, true>(P, A, row_elems, st);
     if (all_scaled)
         return shared ? launch_prep_rows<PT, 1, true>(P, A, row_elems, st)
                       : launch_prep_rows<PT, 1, false>(P, A, row_elems, st);
@@ -465,8 +468,8 @@ cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool shared, uint16
 // shared: every row is a single frame (tp == 2), so A holds one slice per row
 // (A[N, Kh]) and the contraction meets it with the slice-major weight.
 // fold: single-frame rows against the folded weight (one product per pixel).
-pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, cudaStream_t st,
-                            bool fold = false) {
+pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, bool f32,
+                            cudaStream_t st, bool fold = false) {
     const int row_elems = shared ? h->Kh : h->K;
     const size_t need = (size_t)P.N * row_elems * 2;
     if (need > h->stage_bytes) {
@@ -495,8 +498,8 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
         return PE_ERR_CUDA;
     if (!make_out_tmap(&to, out, G.out_f32, G.N, G.E)) return PE_ERR_CUDA;
-    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, h->stage_rows, row_elems, st)
-                                 : launch_prep<16>(P, all_scaled, shared, h->stage_rows, row_elems, st);
+    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st)
+                                 : launch_prep<16>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st);
     if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
     if (fold)
@@ -678,7 +681,7 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
     if (allow_staged && h->fold && h->wpack_fold && P.all_t1 && staged_eligible(h, f_dt)) {
         bool all_scaled = true;
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
-        return run_frames_staged(h, P, out, all_scaled, true, st, true);
+        return run_frames_staged(h, P, out, all_scaled, true, f_dt == PE_F32, st, true);
     }
     // Single images: the resident-A kernel when asked for (PE_FRAMES_PATH=astat)
     // and for the allocation-free call (it needs no workspace); otherwise the
@@ -697,7 +700,7 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
         const bool shared = h->tp == 2 && P.all_t1 && h->wpack_t;
         if (lp == 2) return run_frames_streamed(h, P, out, all_scaled, shared, st);
-        return run_frames_staged(h, P, out, all_scaled, shared, st);
+        return run_frames_staged(h, P, out, all_scaled, shared, f_dt == PE_F32, st);
     }
     int grid = 0;
     bool ok = true;

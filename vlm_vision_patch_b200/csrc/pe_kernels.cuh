@@ -1388,7 +1388,7 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
 
 // Staged frames path, prepare step: normalised patch rows written once for
 // the TMA-fed contraction, through shared memory so that both sides of the
-// copy are coalesced.  A CTA owns kPrepRows consecutive output rows and one
+// copy are coalesced.  bf16 frames, or fp32 frames (F32IN, prep_unit_f32).  A CTA owns kPrepRows consecutive output rows and one
 // (row, word) unit per thread; consecutive threads read consecutive words of
 // one image row.  Each thread loads its word of the p image rows of every
 // channel (single-frame rows: all channels at once; otherwise one channel of
@@ -1401,7 +1401,59 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
 //           last frame repeated where a temporal patch runs past T.
 constexpr int kPrepRows = 16;
 
-template <int PT, int NORM, bool SHARED>
+// fp32 frames: one (row, word) unit of the prepare kernel.  The same rows
+// as the bf16 form (two pixels per unit, 8-byte loads: an image row starts
+// 56-byte aligned and a unit at 8 bytes), normalised from the fp32 values.
+template <int PT, bool SHARED>
+__device__ __forceinline__ void prep_unit_f32(const FwdParams &P, int64_t R, int jw, uint32_t srow, int row_elems,
+                                              int nci) {
+    constexpr int p = PT, NT = SHARED ? 1 : 2;
+    const RowSrc rs = locate_row(P, R, 4);
+    const char *src = rs.base + 8 * jw;
+    const int64_t sW = (int64_t)rs.W * 4, sHW = (int64_t)rs.HW * 4;
+    const int64_t sT1 = (!SHARED && rs.tmax > 0) ? (int64_t)rs.CHW * 4 : 0;
+    const char *dlo = rs.lo, *dhi = rs.hi;   // frame buffer (bounds-checking build)
+    PixPair<true> px[2][NT][p];
+    auto load = [&](const int b, const int c) {
+        const char *a = src + (int64_t)c * sHW;
+#pragma unroll
+        for (int i = 0; i < p; ++i) {
+            px[b][0][i].load(a + (int64_t)i * sW, dlo, dhi, P.err);
+            if constexpr (!SHARED) {
+                px[b][NT - 1][i].zero();
+                if (sT1 != 0) px[b][NT - 1][i].load(a + (int64_t)i * sW + sT1, dlo, dhi, P.err);
+            }
+        }
+    };
+    auto store = [&](const int b, const int c) {
+        const NormConst nc = norm_const(P, c);
+#pragma unroll
+        for (int i = 0; i < p; ++i) {
+            const int ci = c * p + i;
+            const uint32_t w0 = px[b][0][i].norm(nc);
+            if constexpr (SHARED) {
+                sts32(srow + (uint32_t)((ci * p + 2 * jw) * 2), w0);
+            } else {
+                const uint32_t w1 = sT1 ? px[b][NT - 1][i].norm(nc) : w0;
+                sts32(srow + (uint32_t)((ci * 2 * p + 2 * jw) * 2), w0);
+                sts32(srow + (uint32_t)((ci * 2 * p + p + 2 * jw) * 2), w1);
+            }
+        }
+    };
+    const int C = P.C;
+    load(0, 0);
+    for (int c = 0; c < C; c += 2) {
+        if (c + 1 < C) load(1, c + 1);
+        store(0, c);
+        if (c + 1 >= C) break;
+        if (c + 2 < C) load(0, c + 2);
+        store(1, c + 1);
+    }
+    if (SHARED && 2 * jw < row_elems - nci * p)   // zero columns up to Kh
+        sts32(srow + (uint32_t)((nci * p + 2 * jw) * 2), 0u);
+}
+
+template <int PT, int NORM, bool SHARED, bool F32IN = false>
 __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const __grid_constant__ FwdParams P,
                                                                         uint16_t *A, int row_elems) {
     constexpr int p = PT, ws = p / 2, NT = SHARED ? 1 : 2;
@@ -1414,7 +1466,9 @@ __global__ void __launch_bounds__(kPrepRows *PT / 2) pe_prep_rows_kernel(const _
     int r, jw;
     unit_to_row_word<kPrepRows>((int)threadIdx.x, ws, P.merge, r, jw);
     const uint32_t srow = smem_addr(prep_smem) + (uint32_t)(r * row_elems * 2);
-    if (r < rows) {
+    if constexpr (F32IN) {
+        if (r < rows) prep_unit_f32<PT, SHARED>(P, m0 + r, jw, srow, row_elems, nci);
+    } else if (r < rows) {
         const RowSrc rs = locate_row(P, m0 + r, 2);
         const char *src = rs.base + 4 * jw;
         const int sW = rs.W * 2, sHW = rs.HW * 2;
