@@ -419,8 +419,9 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
 // Staged frames path: prepare kernel writes A once, then the TMA-fed pair
 // GEMM reads it back.  The fused producer repeats its gather for every weight
 // tile of a row block; measured on B200 the staged pair is faster at every
-// size (about 2x at ~1000 patches, where both are latency-bound, 1.8x at
-// 59k), so it runs whenever it can: bf16 frames, tp = 2, p in {14, 16}.
+// size (about 2x at ~1000 patches, where both are latency-bound, 3x at 59k
+// patches; 6.8x for fp32 frames), so it runs whenever it can: bf16 or fp32
+// frames, tp = 2, p in {14, 16}.
 
 bool staged_eligible(const pe_handle *h, int f_dt) {
     return (f_dt == PE_BF16 || f_dt == PE_F32) && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
