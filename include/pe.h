@@ -198,7 +198,7 @@ pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int
  *   out      : dev [gt*gh*gw, E] of dtype out_dt.
  * Requires p even and p <= PE_MAX_PATCH.  Execution paths, all within the
  * same tolerance of the exact result:
- *   staged   (default for bf16 or fp32 frames with tp = 2 and p in {14, 16}) a prepare
+ *   staged   (default for bf16 or fp32 frames with tp in {1, 2} and p in {14, 16}) a prepare
  *            kernel writes the normalised rows once into the handle's
  *            grow-only workspace, then the TMA-fed contraction reads them back;
  *   resident A  (PE_FRAMES_PATH=astat, and the allocation-free call, when
@@ -213,7 +213,7 @@ pe_status pe_forward_patches_pos(pe_handle *h, const void *x, pe_dtype x_dt, int
  *            identical bits.  On B200 it runs slower than the staged pair (the
  *            resident A leaves the weight ring too little shared memory);
  *   fused    one kernel that gathers each A tile again for every weight tile
- *            (tp != 2, p not in {14, 16}, and the allocation-free
+ *            (tp in {3, 4}, p not in {14, 16}, and the allocation-free
  *            call's other groups);
  *   streamed one cooperative kernel: producer warps write the same rows while
  *            the contraction consumes the completed row blocks (an option for

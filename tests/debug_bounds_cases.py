@@ -23,9 +23,9 @@ DEV = "cuda:0"
 C, TP = 3, 2
 
 
-def _pe(E, p, bias, seed):
-    pe = PatchEmbed(E, C, TP, p, bias)
-    w = workloads.normal((E, C, TP, p, p), seed, std=0.02, dtype=torch.bfloat16).to(DEV)
+def _pe(E, p, bias, seed, tp=TP):
+    pe = PatchEmbed(E, C, tp, p, bias)
+    w = workloads.normal((E, C, tp, p, p), seed, std=0.02, dtype=torch.bfloat16).to(DEV)
     b = workloads.normal((E,), seed + 1, std=0.02, dtype=torch.bfloat16).to(DEV) if bias else None
     pe.set_weight(w, b)
     pe.set_norm(workloads.CLIP_MEAN, workloads.CLIP_STD)
@@ -38,8 +38,8 @@ def _frames(items, p, seed, dtype=torch.bfloat16):
             for i, (T, gh, gw) in enumerate(items)]
 
 
-def _grids(items):
-    return [((T + TP - 1) // TP, gh, gw) for T, gh, gw in items]
+def _grids(items, tp=TP):
+    return [((T + tp - 1) // tp, gh, gw) for T, gh, gw in items]
 
 
 # name: (frames path, items (T, gh, gw), p, E, bias, frame dtype, out dtype, with pos, extra env)
@@ -57,6 +57,7 @@ FRAME_CASES = {
     "fused_f32_frames": ("fused", [(2, 6, 4), (1, 4, 6)], 14, 256, True, torch.float32, torch.float32, False, {}),
     "staged_f32_images": ("staged", [(1, 6, 8), (1, 4, 10)], 14, 256, True, torch.float32, torch.float32, True, {}),
     "staged_f32_video": ("staged", [(4, 6, 8), (3, 4, 6)], 14, 256, True, torch.float32, torch.bfloat16, False, {}),
+    "staged_tp1": ("staged", [(3, 4, 6), (1, 6, 8)], 14, 192, True, torch.bfloat16, torch.bfloat16, True, {}),
     "fused_p8": ("fused", [(2, 6, 8), (1, 4, 4)], 8, 256, False, torch.bfloat16, torch.bfloat16, False, {}),
     "streamed_video": ("streamed", [(4, 6, 10), (3, 4, 8), (1, 10, 6)], 14, 1280, True, torch.bfloat16,
                        torch.bfloat16, False, {}),
@@ -68,13 +69,14 @@ FRAME_CASES = {
 
 def run_frames(name):
     path, items, p, E, bias, fdt, odt, with_pos, env = FRAME_CASES[name]
+    tp = 1 if name.endswith("_tp1") else TP
     saved = {k: os.environ.get(k) for k in list(env) + ["PE_FRAMES_PATH"]}
     os.environ.update(env)
     os.environ["PE_FRAMES_PATH"] = path
     try:
-        pe = _pe(E, p, bias, 400 + len(name))
+        pe = _pe(E, p, bias, 400 + len(name), tp)
         frames = _frames(items, p, 500 + len(name), fdt)
-        grids = _grids(items)
+        grids = _grids(items, tp)
         n = B.pe_num_patches(grids)
         pos = workloads.normal((n, E), 600, dtype=odt).to(DEV) if with_pos else None
         out = pe.forward_frames_grouped(frames, grids, 2, out_dtype=odt, pos=pos)

@@ -136,3 +136,33 @@ def test_fp32_frames_staged_and_fused(items, p, merge, monkeypatch):
         assert pe.last_error() == 0
         assert n == launches, (path, n)
         assert_within_tolerance(out, ref, mag, what=f"fp32 frames {path} p={p}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("p,merge", [(14, 2), (16, 1)])
+def test_temporal_patch_1_staged_and_fused(p, merge, dtype, monkeypatch):
+    """tp = 1 (one frame per temporal patch, a plain 2-D patch embedding per
+    frame) runs the staged pair (one-slice rows against the frames-order
+    weight) by default and the fused kernel when asked for: a group of a
+    3-frame item and two images, against the oracle."""
+    from vlm_vision_patch_b200 import _binding as B
+    C, tp, E = 3, 1, 192
+    items = [(3, 4, 6), (1, 6, 8), (1, 2, 2)]
+    frames = [workloads.uniform01((T, C, gh * p, gw * p), 950 + i, dtype=dtype) for i, (T, gh, gw) in enumerate(items)]
+    grids = [(T, gh, gw) for T, gh, gw in items]
+    w = workloads.normal((E, C, tp, p, p), 951, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 952, std=0.02, dtype=torch.bfloat16)
+    pe = _pe(E, C, tp, p, w, b)
+    pe.set_norm(workloads.CLIP_MEAN, workloads.CLIP_STD)
+    ref, mag = oracle.conv3d_grouped(list(zip(frames, grids)), merge, workloads.CLIP_MEAN, workloads.CLIP_STD,
+                                     w, b, C, tp, p)
+    dev_frames = [f.to(DEV) for f in frames]
+    for path, launches in (("staged", 2), ("fused", 1)):
+        monkeypatch.setenv("PE_FRAMES_PATH", path)
+        B.pe_profile_begin(pe.h, 0)
+        out = pe.forward_frames_grouped(dev_frames, grids, merge, out_dtype=torch.float32)
+        _, n = B.pe_profile_end(pe.h, 0)
+        torch.cuda.synchronize()
+        assert pe.last_error() == 0
+        assert n == launches, (path, n)
+        assert_within_tolerance(out, ref, mag, what=f"tp=1 {path} p={p} {dtype}")

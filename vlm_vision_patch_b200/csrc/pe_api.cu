@@ -424,7 +424,10 @@ pe_status setup_frames(pe_handle *h, int n, const void *const *frames, int f_dt,
 // frames, tp = 2, p in {14, 16}.
 
 bool staged_eligible(const pe_handle *h, int f_dt) {
-    return (f_dt == PE_BF16 || f_dt == PE_F32) && h->tp == 2 && (h->p == 14 || h->p == 16) && (h->K % 8) == 0;
+    // tp = 1 rows are one slice wide (Kh columns, a multiple of 16); tp = 2
+    // video rows are K wide, so K must keep their rows 16-byte aligned
+    return (f_dt == PE_BF16 || f_dt == PE_F32) && (h->p == 14 || h->p == 16) &&
+           (h->tp == 1 || (h->tp == 2 && (h->K % 8) == 0));
 }
 
 // bf16 frames with tp = 2 and p in {14, 16}: 0 = fused kernel, 1 = staged
@@ -438,7 +441,7 @@ int frames_path(const pe_handle *h, int f_dt) {
     if (!staged_eligible(h, f_dt)) return 0;
     const char *e = std::getenv("PE_FRAMES_PATH");
     if (e && std::strcmp(e, "fused") == 0) return 0;
-    if (e && std::strcmp(e, "streamed") == 0 && f_dt == PE_BF16) return 2;   // its producers read bf16 words
+    if (e && std::strcmp(e, "streamed") == 0 && f_dt == PE_BF16 && h->tp == 2) return 2;   // bf16 words, tp = 2
     return 1;
 }
 
@@ -468,9 +471,11 @@ cudaError_t launch_prep(const FwdParams &P, bool all_scaled, bool shared, bool f
 
 // shared: every row is a single frame (tp == 2), so A holds one slice per row
 // (A[N, Kh]) and the contraction meets it with the slice-major weight.
-// fold: single-frame rows against the folded weight (one product per pixel).
+// wmode 1 (fold): single-frame rows against the folded weight (one product
+// per pixel); wmode 2: tp = 1, whose rows are one frame's patch in the view
+// order, against the frames-order weight (the same order when tp = 1).
 pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scaled, bool shared, bool f32,
-                            cudaStream_t st, bool fold = false) {
+                            cudaStream_t st, int wmode = 0) {
     const int row_elems = shared ? h->Kh : h->K;
     const size_t need = (size_t)P.N * row_elems * 2;
     if (need > h->stage_bytes) {
@@ -493,7 +498,7 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     bool ok = true;
     plan_tiles(h, G, G.N, grid, ok);
     if (!ok) return PE_ERR_UNSUPPORTED;
-    const int amode = (shared && !fold) ? kAModeTmaShared : kAModeTma;
+    const int amode = (shared && wmode == 0) ? kAModeTmaShared : kAModeTma;
     const size_t smem = plan_pipeline(h, G, amode, row_elems);
     CUtensorMap tx, to;
     if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
@@ -503,8 +508,10 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
                                  : launch_prep<16>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st);
     if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
-    if (fold)
+    if (wmode == 1)
         return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wfold[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
+    if (wmode == 2)
+        return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
     if (shared)
         return finish(
             launch_fwd<kAModeTmaShared, 0, false>(h->tmap_wt[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
@@ -682,7 +689,7 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
     if (allow_staged && h->fold && h->wpack_fold && P.all_t1 && staged_eligible(h, f_dt)) {
         bool all_scaled = true;
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
-        return run_frames_staged(h, P, out, all_scaled, true, f_dt == PE_F32, st, true);
+        return run_frames_staged(h, P, out, all_scaled, true, f_dt == PE_F32, st, 1);
     }
     // Single images: the resident-A kernel when asked for (PE_FRAMES_PATH=astat)
     // and for the allocation-free call (it needs no workspace); otherwise the
@@ -701,6 +708,8 @@ pe_status run_frames(pe_handle *h, FwdParams &P, int f_dt, void *out, int out_dt
         for (int c = 0; c < P.C; ++c) all_scaled = all_scaled && P.norm_mode[c] == kNormScaled;
         const bool shared = h->tp == 2 && P.all_t1 && h->wpack_t;
         if (lp == 2) return run_frames_streamed(h, P, out, all_scaled, shared, st);
+        if (h->tp == 1)   // one frame per temporal patch: one-slice rows, frames-order weight
+            return run_frames_staged(h, P, out, all_scaled, true, f_dt == PE_F32, st, 2);
         return run_frames_staged(h, P, out, all_scaled, shared, f_dt == PE_F32, st);
     }
     int grid = 0;
