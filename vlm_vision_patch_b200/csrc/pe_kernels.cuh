@@ -1395,8 +1395,9 @@ __global__ void pe_pack_weight_kernel(const void *w, int w_f32, const void *bias
 // both temporal slices ahead of the one being stored), normalises them and
 // writes them into the CTA's row block in shared memory; one bulk copy then
 // stores the contiguous block of rows.
-//   SHARED  single-frame rows in the slice layout A[N, Kh], column
-//           (c*p + i)*p + j, zero up to Kh (the weight is slice-major);
+//   SHARED  one slice per row, A[N, Kh], column (c*p + i)*p + j, zero up to
+//           Kh: single-frame rows with tp = 2 (met by the slice-major
+//           weight) and every row with tp = 1 (met by the frames-order one);
 //   else    A[N, K] in the frames order k' = ((c*p + i)*tp + t)*p + j, the
 //           last frame repeated where a temporal patch runs past T.
 constexpr int kPrepRows = 16;
