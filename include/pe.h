@@ -380,6 +380,19 @@ pe_status pe_profile_begin(pe_handle *h, int max_calls);
 pe_status pe_profile_end(pe_handle *h, float *ms, int *n, int64_t *launches);
 
 /*
+ * pe_profile_target -- which kernel of a forward call the profiling event
+ * pairs bracket from now on: 0 (the default) the contraction kernel, as
+ * described above; 1 the kernel that runs before it, the prepare kernel of a
+ * staged frames call or the cast / tf32-rounding kernel of an fp32 patches
+ * call (calls without one record nothing).  The patchify read's achieved
+ * memory throughput is the frames bytes over that time.  An event after the
+ * prepare kernel keeps the contraction from starting early, as any event
+ * between the two does.
+ * Errors: PE_ERR_INVALID_ARG (NULL handle, target not 0 or 1).
+ */
+pe_status pe_profile_target(pe_handle *h, int target);
+
+/*
  * pe_selftest_wait_timeout -- test hook for failure detection: one warp waits,
  * through the bounded wait every pipeline uses, on a shared-memory barrier
  * phase that nothing completes.  The wait gives up after its limit (2 s), and

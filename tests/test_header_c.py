@@ -61,6 +61,7 @@ int main(void)
           PE_ERR_INVALID_ARG);
     CHECK(pe_forward_patches_host(NULL, NULL, PE_BF16, 4, NULL, PE_BF16, NULL) == PE_ERR_INVALID_ARG);
     CHECK(pe_selftest_wait_timeout(NULL, NULL) == PE_ERR_INVALID_ARG);
+    CHECK(pe_profile_target(NULL, 0) == PE_ERR_INVALID_ARG);
     pe_destroy(NULL);
     pe_merger_destroy(NULL);
     printf("%%d failed\n", fails);

@@ -34,7 +34,7 @@ EXPORTS = (
     "pe_set_temporal_fold", "pe_forward_patches_pos", "pe_forward_frames_grouped_pos", "pe_set_tf32",
     "pe_merger_create", "pe_merger_set_weights", "pe_merger_forward", "pe_merger_last_error", "pe_merger_destroy",
     "pe_merger_profile_begin", "pe_merger_profile_end", "pe_forward_frames_grouped_host", "pe_forward_patches_host",
-    "pe_selftest_wait_timeout",
+    "pe_selftest_wait_timeout", "pe_profile_target",
 )
 
 
@@ -92,6 +92,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "pe_destroy": ([vp], None),
         "pe_device": ([vp], i32),
         "pe_profile_begin": ([vp, i32], i32),
+        "pe_profile_target": ([vp, i32], i32),
         "pe_profile_end": ([vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(i32),
                             ctypes.POINTER(ctypes.c_int64)], i32),
     }
@@ -230,6 +231,11 @@ def pe_num_patches(grid_thw: Sequence[Sequence[int]]) -> int:
 
 def pe_profile_begin(h: int, max_calls: int) -> None:
     _check("pe_profile_begin", load().pe_profile_begin(h, max_calls))
+
+
+def pe_profile_target(h: int, target: int) -> None:
+    """0: profile the contraction kernel (default); 1: the kernel before it."""
+    _check("pe_profile_target", load().pe_profile_target(h, target))
 
 
 def pe_profile_end(h: int, max_calls: int):

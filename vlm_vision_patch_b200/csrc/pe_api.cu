@@ -68,6 +68,7 @@ struct pe_handle {
     int prof_cap = 0, prof_n = 0;
     int64_t prof_launches = 0;   // kernels launched by forward calls while profiling
     bool prof_on = false;
+    int prof_target = 0;         // 0: the contraction kernel, 1: the kernel before it
     cudaEvent_t items_evt = nullptr;
     bool items_evt_pending = false;
     // host-buffer calls: two input and two output slots in one device buffer,
@@ -201,9 +202,11 @@ cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensor
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     pe_handle *h = t_prof_handle;
-    const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
+    const bool prof = h && h->prof_on && h->prof_target == 0 && h->prof_n < h->prof_cap;
     if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
-    const bool pdl = after_prep && !prof;   // an event between the two kernels serialises them anyway
+    // an event between the two kernels (either profiling target) serialises
+    // them anyway; a window that only counts launches keeps the overlap
+    const bool pdl = after_prep && !(h && h->prof_on && h->prof_cap > 0);
     if (pdl || coop) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid);
@@ -236,6 +239,24 @@ cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensor
     if (h && h->prof_on) ++h->prof_launches;
     return e;
 }
+
+// Event pair around the kernel a call launches before its contraction, when
+// the handle profiles that kernel (pe_profile_target 1).
+struct PreKernelEvents {
+    pe_handle *h;
+    bool on;
+    PreKernelEvents(pe_handle *hh, cudaStream_t st)
+        : h(hh), on(hh && hh->prof_on && hh->prof_target == 1 && hh->prof_n < hh->prof_cap), s(st) {
+        if (on) cudaEventRecord(h->prof_ev[2 * h->prof_n], s);
+    }
+    ~PreKernelEvents() {
+        if (on) {
+            cudaEventRecord(h->prof_ev[2 * h->prof_n + 1], s);
+            ++h->prof_n;
+        }
+    }
+    cudaStream_t s;
+};
 
 struct ProfScope {   // makes the handle's profiling events visible to launch_fwd
     explicit ProfScope(pe_handle *h) { t_prof_handle = h; }
@@ -504,8 +525,12 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     if (!make_tmap_bf16(&tx, h->stage_rows, (uint64_t)G.N, (uint64_t)row_elems, (uint64_t)row_elems, kBM))
         return PE_ERR_CUDA;
     if (!make_out_tmap(&to, out, G.out_f32, G.N, G.E)) return PE_ERR_CUDA;
-    cudaError_t e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st)
-                                 : launch_prep<16>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st);
+    cudaError_t e;
+    {
+        PreKernelEvents pk(h, st);
+        e = (h->p == 14) ? launch_prep<14>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st)
+                         : launch_prep<16>(P, all_scaled, shared, f32, h->stage_rows, row_elems, st);
+    }
     if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
     if (wmode == 1)
@@ -643,7 +668,7 @@ cudaError_t launch_astat(const CUtensorMap &tw, const CUtensorMap &to, const Fwd
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     pe_handle *h = t_prof_handle;
-    const bool prof = h && h->prof_on && h->prof_n < h->prof_cap;
+    const bool prof = h && h->prof_on && h->prof_target == 0 && h->prof_n < h->prof_cap;
     if (prof) cudaEventRecord(h->prof_ev[2 * h->prof_n], st);
     kern<<<grid, kAsThreads, smem, st>>>(tw, to, P);
     e = cudaGetLastError();
@@ -995,8 +1020,11 @@ pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
         if (!make_out_tmap(&to, out, P.out_f32, N, h->E)) return PE_ERR_CUDA;
         const int64_t n4 = (int64_t)N * h->K / 4;
         const int cb = (int)std::min<int64_t>((n4 + 255) / 256, (int64_t)h->num_sms * 8);
-        pe_round_tf32_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(x),
-                                                 reinterpret_cast<uint32_t *>(h->stage_rows), n4);
+        {
+            PreKernelEvents pk(h, st);
+            pe_round_tf32_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(x),
+                                                     reinterpret_cast<uint32_t *>(h->stage_rows), n4);
+        }
         if (h->prof_on) ++h->prof_launches;
         if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
         FwdParams G = P;
@@ -1030,7 +1058,10 @@ pe_status forward_patches(pe_handle *h, const void *x, pe_dtype x_dt, int64_t N,
         if (!make_out_tmap(&to, out, P.out_f32, N, h->E)) return PE_ERR_CUDA;
         const int64_t n8 = (int64_t)N * h->K / 8;
         const int cb = (int)std::min<int64_t>((n8 + 255) / 256, (int64_t)h->num_sms * 8);
-        pe_cast_rows_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(x), h->stage_rows, n8);
+        {
+            PreKernelEvents pk(h, st);
+            pe_cast_rows_kernel<<<cb, 256, 0, st>>>(reinterpret_cast<const float *>(x), h->stage_rows, n8);
+        }
         if (h->prof_on) ++h->prof_launches;
         if (cudaGetLastError() != cudaSuccess) return PE_ERR_CUDA;
         FwdParams G = P;
@@ -1253,6 +1284,12 @@ pe_status pe_profile_begin(pe_handle *h, int max_calls) {
     h->prof_n = 0;
     h->prof_launches = 0;
     h->prof_on = true;
+    return PE_OK;
+}
+
+pe_status pe_profile_target(pe_handle *h, int target) {
+    if (!h || (target != 0 && target != 1)) return PE_ERR_INVALID_ARG;
+    h->prof_target = target;
     return PE_OK;
 }
 
