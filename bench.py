@@ -441,18 +441,21 @@ def run_ours(args, rank, world, local):
     out = torch.empty((wl.N, wl.E), dtype=wl.out_dtype, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # --pos: a [N, E] bf16 position table added in the contraction's epilogue
+    # (device-resident, like a model parameter)
+    pos = workloads.normal((wl.N, wl.E), 97, dtype=torch.bfloat16).to(dev) if args.pos else None
     if wl.patches is not None:
         x_dev = wl.patches.to(dev)
 
         def step():
-            pe.forward_patches(x_dev, out=out)
+            pe.forward_patches(x_dev, out=out, pos=pos)
         in_bytes = wl.patches.numel() * wl.patches.element_size()
     else:
         frames_dev = [it.frames.to(dev) for it in wl.items]
         grids = [it.grid for it in wl.items]
 
         def step():
-            pe.forward_frames_grouped(frames_dev, grids, wl.merge, out=out)
+            pe.forward_frames_grouped(frames_dev, grids, wl.merge, out=out, pos=pos)
         in_bytes = sum(it.frames.numel() * it.frames.element_size() for it in wl.items)
     out_bytes = out.numel() * out.element_size()
 
@@ -551,9 +554,12 @@ def run_ours(args, rank, world, local):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         return total_rows * e2e_steps / (max_over_ranks(e0.elapsed_time(e1), pg, dev) / 1e3)
-    other = "serial" if args.e2e == "host" else "host"
-    e2e_value = e2e_rate(args.e2e)
-    e2e_other = e2e_rate(other)
+    # the host-buffer calls take no position table: with --pos both figures
+    # come from the serial form
+    e2e_mode = "serial" if args.pos else args.e2e
+    other = "serial" if e2e_mode == "host" else "host"
+    e2e_value = e2e_rate(e2e_mode)
+    e2e_other = None if args.pos else e2e_rate(other)
     if pe.last_error() != 0:
         raise RuntimeError("device pipeline timeout during the end-to-end steps")
 
@@ -605,7 +611,8 @@ def run_ours(args, rank, world, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "tf32" if (args.tf32 and wl.patches is not None and wl.patches.dtype == torch.float32) else "bf16",
             "data": "synthetic (seeded U[0,1) frames, N(0,0.02) weights)",
-            "config": dict(config_of(wl, world), **({"temporal_fold": True, "K_contracted": k_eff} if folded else {})),
+            "config": dict(config_of(wl, world), **({"temporal_fold": True, "K_contracted": k_eff} if folded else {}),
+                           **({"position_table": "bf16 [N, E], added in the epilogue"} if args.pos else {})),
             "tflops": step_tflops,
             "pct_of_peak": {f"bf16_burst_{src}": step_tflops / float(peaks["bf16_tflops"]),
                             f"bf16_sustained_{src}": step_tflops / float(peaks.get("bf16_tflops_sustained",
@@ -625,9 +632,10 @@ def run_ours(args, rank, world, local):
                                          else "fallback 1590 TFLOP/s bf16")
                                         + (" x 1.1/2.25 (nominal tf32/bf16)" if tf32 else "")},
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
-                    "d2h_bytes_per_step": out_bytes, "path": E2E_PATHS[args.e2e],
-                    other: {"value": e2e_other, "unit": UNIT, "path": E2E_PATHS[other]}},
+            "e2e": dict({"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
+                         "d2h_bytes_per_step": out_bytes, "path": E2E_PATHS[e2e_mode]},
+                        **({} if args.pos else {other: {"value": e2e_other, "unit": UNIT,
+                                                        "path": E2E_PATHS[other]}})),
             "gpu_launches": launches,
             "context": context,
             "clocks": clk.summary(),
@@ -808,6 +816,9 @@ def main(argv=None):
                     help="time the PatchMerger on the workload's PatchEmbed output instead of the PatchEmbed")
     ap.add_argument("--tf32", action="store_true",
                     help="opt-in tf32 contraction of fp32 patch rows (the fp32 workloads); dtype reads tf32")
+    ap.add_argument("--pos", action="store_true",
+                    help="add a [N, E] bf16 position-embedding table in the contraction's epilogue "
+                         "(pe_forward_*_pos); e2e then times the serial form")
     ap.add_argument("--fold", action="store_true",
                     help="opt-in temporal folding of single-frame items (half the contraction; TFLOP/s then "
                          "counts the folded K)")
