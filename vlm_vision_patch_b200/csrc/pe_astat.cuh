@@ -87,12 +87,8 @@ __device__ __forceinline__ bool mbar_wait_nap(uint32_t bar, uint32_t parity, vol
         }
     }
 }
+
 constexpr uint32_t kAsNapNs = 100;
-
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // One 32-column chunk of an epilogue warp's 32 rows: + bias (+ position
 // table), cast, staged through a swizzled box, stored by TMA (rows past N and
 // columns past E are clipped by the tensor map).

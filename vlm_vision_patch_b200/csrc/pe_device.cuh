@@ -141,6 +141,11 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Hint: bring the 128-byte line holding `p` into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Untiled bulk copy of `bytes` contiguous bytes from shared to global memory
 // (both addresses 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {

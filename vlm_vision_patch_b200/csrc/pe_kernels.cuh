@@ -1233,9 +1233,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         };
         // the tile loop, compiled without options, with the position-embedding
         // add, and with the GELU (the PatchMerger's fc1)
+        // With a position table, each lane asks L2 for its row of the table
+        // for this CTA's next tile (and for the first tile) before waiting for
+        // the accumulator: the MMAs of the tile hide that fetch, and the
+        // per-chunk table loads below then find the rows in L2.
+        auto prefetch_pos = [&](int t) {
+            const int64_t r = (int64_t)(t / P.n_tiles_n) * (2 * kBM) + rank * kBM + wq * 32 + lane;
+            const int c0 = (t % P.n_tiles_n) * P.bn;
+            if (r >= P.N || c0 >= P.E) return;
+            const int es = P.pos_f32 ? 4 : 2;
+            const int nc = (P.E - c0) < P.bn ? (P.E - c0) : P.bn;
+            const uintptr_t a = reinterpret_cast<uintptr_t>(P.pos) + (uintptr_t)((r * P.E + c0) * es);
+            const uintptr_t end = a + (uintptr_t)nc * es;
+            prefetch_l2(reinterpret_cast<const void *>(a));
+            for (uintptr_t q = (a & ~(uintptr_t)127) + 128; q < end; q += 128)
+                prefetch_l2(reinterpret_cast<const void *>(q));
+        };
         auto tiles = [&](auto kPos, auto kAct) {
             for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
                 const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
+                if constexpr (decltype(kPos)::value) {
+                    if (tile == (int)(blockIdx.x >> 1)) prefetch_pos(tile);
+                    if (tile + (int)(gridDim.x >> 1) < P.num_tiles) prefetch_pos(tile + (int)(gridDim.x >> 1));
+                }
                 if (!mbar_wait(smem_addr(&tfull[acc]), accph, abort)) break;
                 tc_fence_after();
                 const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
