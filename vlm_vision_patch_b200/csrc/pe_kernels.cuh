@@ -1149,32 +1149,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         const int nch = P.bn / 32;   // 2, 4 or 8
         int acc = 0, nbuf = 0;
         uint32_t accph = 0;
-        auto emit = [&](auto kPos, auto kAct, const uint32_t (&v)[32], int cc, int64_t row0, int n_blk) {
+        // position-embedding row segment of this lane's row for chunk cc (E % 8
+        // == 0, so a 16-byte piece is either wholly inside the row or wholly past it)
+        auto load_pos = [&](uint4 (&pq)[8], int cc, int64_t row0, int n_blk) {
+            const int col0 = n_blk * P.bn + cc * 32;
+            const int64_t r = row0 + lane;
+            const int nq = P.pos_f32 ? 8 : 4;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                pq[q] = make_uint4(0u, 0u, 0u, 0u);
+                const int c0 = col0 + q * (P.pos_f32 ? 4 : 8);
+                if (q < nq && r < P.N && c0 < P.E) {
+                    const char *a = reinterpret_cast<const char *>(P.pos) +
+                                    (r * P.E + c0) * (int64_t)(P.pos_f32 ? 4 : 2);
+                    const char *plo = reinterpret_cast<const char *>(P.pos);
+                    if (PE_IN(a, 16, plo, plo + P.N * (int64_t)P.E * (P.pos_f32 ? 4 : 2), P.err))
+                        asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
+                                     : "l"(a));
+                }
+            }
+        };
+        // pq holds chunk cc's table segment on entry (loaded one chunk ahead);
+        // once added, it is reloaded with chunk cc + 1's while this chunk is
+        // staged and stored
+        auto emit = [&](auto kPos, auto kAct, const uint32_t (&v)[32], int cc, int64_t row0, int n_blk,
+                        uint4 (&pq)[8]) {
             constexpr bool has_pos = decltype(kPos)::value;
             constexpr bool has_act = decltype(kAct)::value;
             const int col0 = n_blk * P.bn + cc * 32;
             if (row0 >= P.N || col0 >= P.E) return;   // whole box outside: nothing to store
-            // position-embedding row segment of this lane's row (E % 8 == 0, so a
-            // 16-byte piece is either wholly inside the row or wholly past it)
-            uint4 pq[8];
-            if constexpr (has_pos) {
-                const int64_t r = row0 + lane;
-                const int nq = P.pos_f32 ? 8 : 4;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    pq[q] = make_uint4(0u, 0u, 0u, 0u);
-                    const int c0 = col0 + q * (P.pos_f32 ? 4 : 8);
-                    if (q < nq && r < P.N && c0 < P.E) {
-                        const char *a = reinterpret_cast<const char *>(P.pos) +
-                                        (r * P.E + c0) * (int64_t)(P.pos_f32 ? 4 : 2);
-                        const char *plo = reinterpret_cast<const char *>(P.pos);
-                        if (PE_IN(a, 16, plo, plo + P.N * (int64_t)P.E * (P.pos_f32 ? 4 : 2), P.err))
-                            asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                         : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
-                                         : "l"(a));
-                    }
-                }
-            }
             float f[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
@@ -1207,6 +1211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                         }
                     }
                 }
+                if (cc + 1 < nch) load_pos(pq, cc + 1, row0, n_blk);
             }
             uint8_t *buf = stage_buf + (size_t)nbuf * (P.out_f32 ? 4096 : 2048);
             if (P.out_f32) {
@@ -1260,6 +1265,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 tc_fence_after();
                 const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
                 const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
+                uint4 pq[8];
+                if constexpr (decltype(kPos)::value) load_pos(pq, 0, row0, n_blk);
                 if constexpr (kTmaA && AMODE != kAModeTmaStream) {
                     // registers to spare: the next chunk's TMEM load overlaps this chunk's work
                     uint32_t va[32], vb[32];
@@ -1267,17 +1274,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     for (int cc = 0; cc < nch; cc += 2) {
                         tmem_ld_wait();
                         tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 1) * 32, vb);
-                        emit(kPos, kAct, va, cc, row0, n_blk);
+                        emit(kPos, kAct, va, cc, row0, n_blk, pq);
                         tmem_ld_wait();
                         if (cc + 2 < nch) tmem_ld_32x32b_x32(tbase + (uint32_t)(cc + 2) * 32, va);
-                        emit(kPos, kAct, vb, cc + 1, row0, n_blk);
+                        emit(kPos, kAct, vb, cc + 1, row0, n_blk, pq);
                     }
                 } else {
                     uint32_t va[32];
                     for (int cc = 0; cc < nch; ++cc) {
                         tmem_ld_32x32b_x32(tbase + (uint32_t)cc * 32, va);
                         tmem_ld_wait();
-                        emit(kPos, kAct, va, cc, row0, n_blk);
+                        emit(kPos, kAct, va, cc, row0, n_blk, pq);
                     }
                 }
                 tc_fence_before();
