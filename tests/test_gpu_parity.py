@@ -494,6 +494,37 @@ def test_position_embedding_add(form, path, pos_dtype, out_dtype, monkeypatch):
     assert_within_tolerance(out, ref + pv, mag + np.abs(pv), what=f"pos {form} {path}")
 
 
+@pytest.mark.parametrize("form,pos_dtype", [("patches", torch.bfloat16), ("patches", torch.float32),
+                                            ("frames", torch.bfloat16), ("frames", torch.float32)])
+def test_position_embedding_ragged_width(form, pos_dtype):
+    """E = 200 (six whole 32-column chunks and one of 8 columns) with a bias:
+    the last chunk takes the epilogue's guarded table and bias loads, the
+    others the unguarded ones.  Against the oracle's conv plus the table."""
+    C, tp, p, E = 3, 2, 14, 200
+    w = workloads.normal((E, C, tp, p, p), 180, std=0.02, dtype=torch.bfloat16)
+    b = workloads.normal((E,), 181, std=0.5)
+    pe = _pe((E, C, tp, p), w, b, workloads.CLIP_MEAN, workloads.CLIP_STD)
+    if form == "frames":
+        grids = [(1, 6, 10), (2, 4, 6)]
+        items = [(workloads.uniform01((T, C, g[1] * p, g[2] * p), 182 + i), g)
+                 for i, (T, g) in enumerate(zip([1, 3], grids))]
+        N = sum(g[0] * g[1] * g[2] for g in grids)
+        pos = workloads.normal((N, E), 184, std=1.0, dtype=pos_dtype)
+        out = pe.forward_frames_grouped([f.to(DEV) for f, _ in items], grids, 2, out_dtype=torch.float32,
+                                        pos=pos.to(DEV))
+        ref, mag = oracle.conv3d_grouped(items, 2, workloads.CLIP_MEAN, workloads.CLIP_STD, w, b, C, tp, p)
+    else:
+        N = 333
+        x = workloads.normal((N, C * tp * p * p), 185, dtype=torch.bfloat16)
+        pos = workloads.normal((N, E), 186, std=1.0, dtype=pos_dtype)
+        out = pe.forward_patches(x.to(DEV), out_dtype=torch.float32, pos=pos.to(DEV))
+        ref, mag = oracle.conv3d_patches(x, w, b, C, tp, p)
+    torch.cuda.synchronize()
+    assert pe.last_error() == 0
+    pv = pos.double().numpy()
+    assert_within_tolerance(out, ref + pv, mag + np.abs(pv), what=f"pos E=200 {form} {pos_dtype}")
+
+
 def test_position_embedding_argument_errors():
     C, tp, p, E = 3, 2, 14, 64
     pe = _pe((E, C, tp, p), workloads.normal((E, C, tp, p, p), 170, std=0.02), None)

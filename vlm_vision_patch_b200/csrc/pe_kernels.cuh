@@ -1149,24 +1149,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         const int nch = P.bn / 32;   // 2, 4 or 8
         int acc = 0, nbuf = 0;
         uint32_t accph = 0;
-        // position-embedding row segment of this lane's row for chunk cc (E % 8
-        // == 0, so a 16-byte piece is either wholly inside the row or wholly past it)
-        auto load_pos = [&](uint4 (&pq)[8], int cc, int64_t row0, int n_blk) {
+        // position-embedding row segment of this lane's row for chunk cc, PD = 1
+        // for a bf16 table (four 16-byte pieces), 2 for fp32 (eight).  A chunk
+        // wholly inside the table takes unguarded loads; at the edges E % 8 == 0
+        // keeps each 16-byte piece wholly inside the row or wholly past it.
+        auto load_pos = [&](auto kPD, uint4 (&pq)[8], int cc, int64_t row0, int n_blk) {
+            constexpr int PD = decltype(kPD)::value;
+            constexpr int NQ = PD == 2 ? 8 : 4, ES = PD == 2 ? 4 : 2;
             const int col0 = n_blk * P.bn + cc * 32;
             const int64_t r = row0 + lane;
-            const int nq = P.pos_f32 ? 8 : 4;
+            const char *plo = reinterpret_cast<const char *>(P.pos);
+            const char *phi = plo + P.N * (int64_t)P.E * ES;
+            const char *a0 = plo + (r * P.E + col0) * (int64_t)ES;
+            if (r < P.N && col0 + 32 <= P.E) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                pq[q] = make_uint4(0u, 0u, 0u, 0u);
-                const int c0 = col0 + q * (P.pos_f32 ? 4 : 8);
-                if (q < nq && r < P.N && c0 < P.E) {
-                    const char *a = reinterpret_cast<const char *>(P.pos) +
-                                    (r * P.E + c0) * (int64_t)(P.pos_f32 ? 4 : 2);
-                    const char *plo = reinterpret_cast<const char *>(P.pos);
-                    if (PE_IN(a, 16, plo, plo + P.N * (int64_t)P.E * (P.pos_f32 ? 4 : 2), P.err))
+                for (int q = 0; q < NQ; ++q) {
+                    pq[q] = make_uint4(0u, 0u, 0u, 0u);
+                    if (PE_IN(a0 + 16 * q, 16, plo, phi, P.err))
                         asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
-                                     : "l"(a));
+                                     : "l"(a0 + 16 * q));
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                    pq[q] = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < P.N && col0 + q * (16 / ES) < P.E && PE_IN(a0 + 16 * q, 16, plo, phi, P.err))
+                        asm volatile("ld.global.nc.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(pq[q].x), "=r"(pq[q].y), "=r"(pq[q].z), "=r"(pq[q].w)
+                                     : "l"(a0 + 16 * q));
                 }
             }
         };
@@ -1175,7 +1186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         // staged and stored
         auto emit = [&](auto kPos, auto kAct, const uint32_t (&v)[32], int cc, int64_t row0, int n_blk,
                         uint4 (&pq)[8]) {
-            constexpr bool has_pos = decltype(kPos)::value;
+            constexpr int PD = decltype(kPos)::value;
             constexpr bool has_act = decltype(kAct)::value;
             const int col0 = n_blk * P.bn + cc * 32;
             if (row0 >= P.N || col0 >= P.E) return;   // whole box outside: nothing to store
@@ -1183,9 +1194,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
 #pragma unroll
             for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
             if (P.bias) {
+                if (col0 + 32 <= P.E) {   // the bias buffer is the library's own: 16-byte aligned
+                    const float4 *b4 = reinterpret_cast<const float4 *>(P.bias + col0);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 b = __ldg(b4 + i);
+                        f[4 * i] += b.x;
+                        f[4 * i + 1] += b.y;
+                        f[4 * i + 2] += b.z;
+                        f[4 * i + 3] += b.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (col0 + e < P.E) f[e] += __ldg(P.bias + col0 + e);
+                }
             }
             // the buffer must be free of the store issued nbufs chunks ago
             if (lane == 0) {
@@ -1196,14 +1219,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
 #pragma unroll
                 for (int e = 0; e < 32; ++e) f[e] = 0.5f * f[e] * (1.0f + erff(f[e] * 0.70710678118654752f));
             }
-            if constexpr (has_pos) {   // out = acc + bias + pos, in fp32, before the output cast
+            if constexpr (PD != 0) {   // out = acc + bias + pos, in fp32, before the output cast
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int q = 0; q < (PD == 2 ? 8 : 4); ++q) {
                     const uint32_t w4[4] = {pq[q].x, pq[q].y, pq[q].z, pq[q].w};
-                    if (P.pos_f32) {
+                    if constexpr (PD == 2) {
 #pragma unroll
                         for (int u = 0; u < 4; ++u) f[4 * q + u] += __uint_as_float(w4[u]);
-                    } else if (q < 4) {
+                    } else {
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             f[8 * q + 2 * u] += bf16lo_to_f32(w4[u]);
@@ -1211,7 +1234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                         }
                     }
                 }
-                if (cc + 1 < nch) load_pos(pq, cc + 1, row0, n_blk);
+                if (cc + 1 < nch) load_pos(kPos, pq, cc + 1, row0, n_blk);
             }
             uint8_t *buf = stage_buf + (size_t)nbuf * (P.out_f32 ? 4096 : 2048);
             if (P.out_f32) {
@@ -1257,7 +1280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
         auto tiles = [&](auto kPos, auto kAct) {
             for (int tile = blockIdx.x >> 1; tile < P.num_tiles; tile += gridDim.x >> 1) {
                 const int m_blk = tile / P.n_tiles_n, n_blk = tile % P.n_tiles_n;
-                if constexpr (decltype(kPos)::value) {
+                if constexpr (decltype(kPos)::value != 0) {
                     if (tile == (int)(blockIdx.x >> 1)) prefetch_pos(tile);
                     if (tile + (int)(gridDim.x >> 1) < P.num_tiles) prefetch_pos(tile + (int)(gridDim.x >> 1));
                 }
@@ -1266,9 +1289,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 const int64_t row0 = (int64_t)m_blk * (2 * kBM) + rank * kBM + wq * 32;
                 const uint32_t tbase = tmem_base + ((uint32_t)(wq * 32) << 16) + (uint32_t)(acc * kMaxBN);
                 uint4 pq[8];
-                if constexpr (decltype(kPos)::value) load_pos(pq, 0, row0, n_blk);
-                if constexpr (kTmaA && AMODE != kAModeTmaStream) {
+                if constexpr (decltype(kPos)::value != 0) load_pos(kPos, pq, 0, row0, n_blk);
+                if constexpr (kTmaA && AMODE != kAModeTmaStream && decltype(kPos)::value != 2) {
                     // registers to spare: the next chunk's TMEM load overlaps this chunk's work
+                    // (not with an fp32 table, whose 32 registers of look-ahead take their place)
                     uint32_t va[32], vb[32];
                     tmem_ld_32x32b_x32(tbase, va);
                     for (int cc = 0; cc < nch; cc += 2) {
@@ -1293,9 +1317,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 if (++acc == 2) { acc = 0; accph ^= 1; }
             }
         };
-        if (P.pos) tiles(std::true_type{}, std::false_type{});
-        else if (P.act) tiles(std::false_type{}, std::true_type{});
-        else tiles(std::false_type{}, std::false_type{});
+        using PosNone = std::integral_constant<int, 0>;
+        if (P.pos && P.pos_f32) tiles(std::integral_constant<int, 2>{}, std::false_type{});
+        else if (P.pos) tiles(std::integral_constant<int, 1>{}, std::false_type{});
+        else if (P.act) tiles(PosNone{}, std::true_type{});
+        else tiles(PosNone{}, std::false_type{});
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
     } else if (AMODE == kAModeTmaStream && warp >= kStreamProdWarp0 && warp < kStreamProdWarp0 + kStreamProdWarps) {
