@@ -386,7 +386,8 @@ def _folded_weight(w: torch.Tensor) -> torch.Tensor:
     return out
 
 
-@pytest.mark.parametrize("case", ["image_224x896", "grouped_small", "p16_raster_bias", "grouped_16_images"])
+@pytest.mark.parametrize("case", ["image_224x896", "grouped_small", "p16_raster_bias", "grouped_16_images",
+                                  "E200_bias_f32", "E200_bf16"])
 def test_temporal_fold(case):
     """Opt-in folding: (1) within the parity tolerance of the oracle run with the
     folded weight (the same products, any summation order); (2) within the
@@ -396,6 +397,7 @@ def test_temporal_fold(case):
     errors have random signs over the C*p*p terms of a row, so on these inputs
     they stay well inside the bound (the worst ratio is printed)."""
     rows = None
+    od = torch.bfloat16
     if case == "image_224x896":
         wl = workloads.image_224x896()
     elif case == "grouped_16_images":
@@ -405,6 +407,13 @@ def test_temporal_fold(case):
         if case == "grouped_small":
             p, E, merge, bias = 14, 1280, 2, None
             grids = [(1, 12, 18), (1, 20, 10), (1, 8, 8)]
+        elif case.startswith("E200"):
+            # rows of 400 or 800 bytes and a last 8-column chunk: the epilogue's
+            # 16-byte register stores and its partial chunk
+            p, E, merge = 14, 200, 2
+            grids = [(1, 6, 10), (1, 4, 8)]
+            bias = workloads.normal((E,), 133, std=0.5) if case == "E200_bias_f32" else None
+            od = torch.float32 if case == "E200_bias_f32" else torch.bfloat16
         else:
             p, E, merge = 16, 1152, 1
             grids = [(1, 7, 9), (1, 5, 11)]
@@ -418,7 +427,7 @@ def test_temporal_fold(case):
     pe = _pe((wl.E, wl.C, wl.tp, wl.p), wl.weight, wl.bias, wl.mean, wl.std)
     pe.set_temporal_fold(True)
     frames = [it.frames.to(DEV) for it in wl.items]
-    out = pe.forward_frames_grouped(frames, [it.grid for it in wl.items], wl.merge)
+    out = pe.forward_frames_grouped(frames, [it.grid for it in wl.items], wl.merge, out_dtype=od)
     torch.cuda.synchronize()
     assert pe.last_error() == 0
     mask = None if rows is None else mask_of(rows, wl.N)

@@ -195,10 +195,10 @@ thread_local pe_handle *t_prof_handle = nullptr;   // handle of the call being l
 // griddepcontrol.wait before the first load).
 // `coop`: every CTA must be resident at once (CTAs wait for rows that other
 // CTAs produce): cooperative launch.
-template <int AMODE, int PT, bool F32IN, int NORM = 2, bool DUPALL = false>
+template <int AMODE, int PT, bool F32IN, int NORM = 2, bool DUPALL = false, bool REGSTORE = false>
 cudaError_t launch_fwd(const CUtensorMap &tw, const FwdParams &P, const CUtensorMap &tx, const CUtensorMap &to,
                        size_t smem, int grid, cudaStream_t st, bool after_prep = false, bool coop = false) {
-    auto kern = pe_fwd_kernel<AMODE, PT, F32IN, NORM, DUPALL>;
+    auto kern = pe_fwd_kernel<AMODE, PT, F32IN, NORM, DUPALL, REGSTORE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     pe_handle *h = t_prof_handle;
@@ -533,8 +533,14 @@ pe_status run_frames_staged(pe_handle *h, FwdParams &P, void *out, bool all_scal
     }
     if (h->prof_on) ++h->prof_launches;
     if (e != cudaSuccess) return PE_ERR_CUDA;
-    if (wmode == 1)
-        return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wfold[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
+    if (wmode == 1) {
+        // the folded weight halves each tile's MMAs, so the epilogue bounds the
+        // tile: its rows are stored straight from registers
+        G.out = out;
+        G.epi_v8 = reinterpret_cast<uintptr_t>(out) % 32 == 0 && (int64_t)G.E * (G.out_f32 ? 4 : 2) % 32 == 0;
+        return finish(launch_fwd<kAModeTma, 0, false, 2, false, true>(h->tmap_wfold[bn_index(G.bn)], G, tx, to, smem,
+                                                                      grid, st, true));
+    }
     if (wmode == 2)
         return finish(launch_fwd<kAModeTma, 0, false>(h->tmap_wf[bn_index(G.bn)], G, tx, to, smem, grid, st, true));
     if (shared)

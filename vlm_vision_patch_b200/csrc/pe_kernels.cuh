@@ -126,6 +126,7 @@ struct FwdParams {
     void *out;                        // [N, E] output (the direct-store epilogue)
     int32_t cpp;                      // C*p*p: columns of one temporal slice
     uint64_t wait_ns;                 // pipeline wait limit in ns (0: kWaitTimeoutNs)
+    int32_t epi_v8;                   // register-store epilogue: out and its rows are 32-byte aligned
 };
 
 // ------------------------------------------------------------ debug bounds
@@ -995,7 +996,10 @@ __device__ __noinline__ void mma_issue_generic(const FwdParams &P, uint8_t *a_ri
 
 // ------------------------------------------------------------- the kernel
 
-template <int AMODE, int PT, bool F32IN, int NORM, bool DUPALL>
+// REGSTORE: the epilogue writes each lane's row straight from registers
+// (P.out) instead of staging 32 x 32 boxes for TMA stores.  Faster only where
+// the epilogue, not the MMAs, bounds a tile (the folded weight's half-K tiles).
+template <int AMODE, int PT, bool F32IN, int NORM, bool DUPALL, bool REGSTORE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 1)
     pe_fwd_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                   const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ FwdParams P) {
@@ -1211,10 +1215,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 }
             }
             // the buffer must be free of the store issued nbufs chunks ago
-            if (lane == 0) {
-                if (nbufs == 4) bulk_wait_read<3>(); else bulk_wait_read<1>();
+            if constexpr (!REGSTORE) {
+                if (lane == 0) {
+                    if (nbufs == 4) bulk_wait_read<3>(); else bulk_wait_read<1>();
+                }
+                __syncwarp();
             }
-            __syncwarp();
             if constexpr (has_act) {   // exact GELU, 0.5 x (1 + erf(x / sqrt 2)), in fp32
 #pragma unroll
                 for (int e = 0; e < 32; ++e) f[e] = 0.5f * f[e] * (1.0f + erff(f[e] * 0.70710678118654752f));
@@ -1235,6 +1241,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                     }
                 }
                 if (cc + 1 < nch) load_pos(kPos, pq, cc + 1, row0, n_blk);
+            }
+            if constexpr (REGSTORE) {
+                const int64_t r = row0 + lane;
+                if (r >= P.N) return;
+                const bool whole = col0 + 32 <= P.E;
+                char *o = static_cast<char *>(P.out) + (r * P.E + col0) * (int64_t)(P.out_f32 ? 4 : 2);
+                if (!P.out_f32) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(f[2 * c], f[2 * c + 1]);
+                    if (whole && P.epi_v8) {
+                        st_global_v8(o, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                        st_global_v8(o + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)   // E % 8 == 0: a 16-byte piece is wholly in or past the row
+                            if (col0 + 8 * q < P.E)
+                                st_global_v4(o + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    }
+                } else {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(f[c]);
+                    if (whole && P.epi_v8) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            st_global_v8(o + 32 * q, w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3], w[8 * q + 4],
+                                         w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            if (col0 + 4 * q < P.E)
+                                st_global_v4(o + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    }
+                }
+                return;
             }
             uint8_t *buf = stage_buf + (size_t)nbuf * (P.out_f32 ? 4096 : 2048);
             if (P.out_f32) {
