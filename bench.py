@@ -71,11 +71,12 @@ def load_peaks():
 # SHA-256 of the kernel sources it was taken on.  A changed kernel invalidates
 # the figure (reported as null) until it is captured again.
 TRAFFIC = {
-    ("grouped_16_images", "staged"): {"bytes": 105941248 + 96926208, "kernel_sha": "9c4107df61303b2e"},
-    ("grouped_16_images", "astat"): {"bytes": 111334144 + 98161664, "kernel_sha": "9c4107df61303b2e"},
-    ("long_video_64x896", "staged"): {"bytes": 419398656 + 281046784, "kernel_sha": "9c4107df61303b2e"},
+    ("grouped_16_images", "staged"): {"bytes": 111796224 + 97408512, "kernel_sha": "b5936d4a35aabebe"},
+    ("grouped_16_images", "staged_fold"): {"bytes": 86795008 + 97496832, "kernel_sha": "b5936d4a35aabebe"},
+    ("grouped_16_images", "astat"): {"bytes": 111581440 + 98128384, "kernel_sha": "b5936d4a35aabebe"},
+    ("long_video_64x896", "staged"): {"bytes": 528994816 + 281480704, "kernel_sha": "b5936d4a35aabebe"},
     # the PatchMerger's fc1 + GELU
-    ("patch_merger_grouped_16_images", "fc1"): {"bytes": 699528704 + 139933184, "kernel_sha": "9c4107df61303b2e"},
+    ("patch_merger_grouped_16_images", "fc1"): {"bytes": 805690880 + 136922112, "kernel_sha": "b5936d4a35aabebe"},
 }
 KERNEL_SOURCES = ("vlm_vision_patch_b200/csrc/pe_kernels.cuh", "vlm_vision_patch_b200/csrc/pe_device.cuh",
                   "vlm_vision_patch_b200/csrc/pe_astat.cuh")
@@ -603,7 +604,11 @@ def run_ours(args, rank, world, local):
             cpu = {"value": r, "unit": UNIT, "cores": th, "kind": "oracle",
                    "sample": f"{min(args.cpu_rows, wl.N)} seeded random output rows of {wl.name} (of {wl.N}), "
                              f"{dt:.1f} s; direct fp64 Conv3d, OpenMP over rows"}
-        traffic = measured_traffic(wl.name, "staged" if staged else ("astat" if "resident A" in path else "single"))
+        # the counters belong to one kernel form: the folded weight, the
+        # position table and tf32 each launch another
+        variant = ("staged" if staged else ("astat" if "resident A" in path else "single")) + \
+            ("_fold" if folded else "") + ("_pos" if args.pos else "") + ("_tf32" if tf32 else "")
+        traffic = measured_traffic(wl.name, variant)
         context = None if (args.no_context or world > 1) else library_context(wl, dev, flush_buf)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
