@@ -64,6 +64,12 @@ FRAME_CASES = {
     "fused_p32": ("fused", [(3, 2, 4), (1, 4, 2)], 32, 128, True, torch.bfloat16, torch.float32, True, {}),
     "many_items": ("staged", [(1 + (i % 3), 2 + 2 * (i % 4), 2 + 2 * (i % 5)) for i in range(40)], 14, 256,
                    True, torch.bfloat16, torch.bfloat16, True, {}),
+    # temporal folding: the contraction's register-store epilogue (16-byte stores
+    # on 400-byte rows with a partial last chunk; 32-byte stores on fp32 rows)
+    "staged_E200_fold": ("staged", [(1, 6, 10), (1, 4, 8)], 14, 200, True, torch.bfloat16, torch.bfloat16, True,
+                         {}),
+    "staged_f32out_fold": ("staged", [(1, 12, 18), (1, 2, 2)], 14, 1280, True, torch.bfloat16, torch.float32,
+                           False, {}),
 }
 
 
@@ -75,6 +81,8 @@ def run_frames(name):
     os.environ["PE_FRAMES_PATH"] = path
     try:
         pe = _pe(E, p, bias, 400 + len(name), tp)
+        if name.endswith("_fold"):
+            pe.set_temporal_fold(True)
         frames = _frames(items, p, 500 + len(name), fdt)
         grids = _grids(items, tp)
         n = B.pe_num_patches(grids)

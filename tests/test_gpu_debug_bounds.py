@@ -7,9 +7,10 @@ register-to-global output stores) checks its address range against the
 buffer it indexes; an access outside would set PE_ERR_DEVICE_BOUNDS in the
 handle's error word and be skipped.  A child process runs the staged,
 resident-A (staging boxes and direct stores), fused (bf16 and fp32 frames,
-p = 8, p = 32), streamed, device item-table, patch-row (including K = 8192 and
-E = 65528) and merger paths on small ragged shapes, once with each library; the debug run must report no error
-and give the same bits as the product library.
+p = 8, p = 32), streamed, device item-table, folded (the contraction's
+register stores), patch-row (including K = 8192 and E = 65528) and merger
+paths on small ragged shapes, once with each library; the debug run must
+report no error and give the same bits as the product library.
 """
 import os
 import subprocess

@@ -1247,17 +1247,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
                 if (r >= P.N) return;
                 const bool whole = col0 + 32 <= P.E;
                 char *o = static_cast<char *>(P.out) + (r * P.E + col0) * (int64_t)(P.out_f32 ? 4 : 2);
+                const char *olo = static_cast<const char *>(P.out);
+                const char *ohi = olo + P.N * (int64_t)P.E * (P.out_f32 ? 4 : 2);
                 if (!P.out_f32) {
                     uint32_t w[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) w[c] = pack_bf16x2(f[2 * c], f[2 * c + 1]);
                     if (whole && P.epi_v8) {
-                        st_global_v8(o, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
-                        st_global_v8(o + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                        if (PE_IN(o, 64, olo, ohi, P.err)) {
+                            st_global_v8(o, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                            st_global_v8(o + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                        }
                     } else {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)   // E % 8 == 0: a 16-byte piece is wholly in or past the row
-                            if (col0 + 8 * q < P.E)
+                            if (col0 + 8 * q < P.E && PE_IN(o + 16 * q, 16, olo, ohi, P.err))
                                 st_global_v4(o + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                     }
                 } else {
@@ -1265,14 +1269,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(AMODE), 
 #pragma unroll
                     for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(f[c]);
                     if (whole && P.epi_v8) {
+                        if (PE_IN(o, 128, olo, ohi, P.err)) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            st_global_v8(o + 32 * q, w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3], w[8 * q + 4],
-                                         w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]);
+                            for (int q = 0; q < 4; ++q)
+                                st_global_v8(o + 32 * q, w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3],
+                                             w[8 * q + 4], w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]);
+                        }
                     } else {
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
-                            if (col0 + 4 * q < P.E)
+                            if (col0 + 4 * q < P.E && PE_IN(o + 16 * q, 16, olo, ohi, P.err))
                                 st_global_v4(o + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                     }
                 }
