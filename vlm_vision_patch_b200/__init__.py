@@ -26,10 +26,11 @@ def _dt(t: torch.dtype) -> int:
 
 
 def _dev(t: torch.Tensor, name: str, device: Optional[int] = None) -> int:
-    if not t.is_cuda:
+    d = t.get_device()            # -1 for a host tensor
+    if d < 0:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if device is not None and t.device.index != device:
-        raise ValueError(f"{name} is on cuda:{t.device.index}, the handle on cuda:{device}")
+    if device is not None and d != device:
+        raise ValueError(f"{name} is on cuda:{d}, the handle on cuda:{device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
@@ -63,8 +64,15 @@ def _need_frames(frames: Sequence[torch.Tensor], C: int) -> None:
             raise ValueError(f"frames must be [T, {C}, H, W]; got {tuple(f.shape)}")
 
 
+# the current stream's raw handle without building a Stream object (a few
+# microseconds per call otherwise); the public route where torch lacks it
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream) -> int:
     if stream is None:
+        if _raw_stream is not None:
+            return int(_raw_stream(torch.cuda.current_device()))
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
@@ -173,14 +181,28 @@ class PatchEmbed:
         return out
 
     def _items(self, frames, grid_thw):
+        """One pass over the items: the grids, layouts and dtypes checked, and the
+        frame sizes (T, H, W) and grids flattened for the C call.  Returns
+        (patch count, flat THW, flat grids, frames dtype)."""
         if len(frames) == 0 or len(frames) != len(grid_thw):
             raise ValueError(f"{len(frames)} frame tensors for {len(grid_thw)} grids; need one per item, at least one")
-        if any(len(g) != 3 for g in grid_thw):
-            raise ValueError("every grid_thw entry must be (t, h, w)")
-        _need_frames(frames, self.C)
-        if len({f.dtype for f in frames}) != 1:
-            raise TypeError("all items must share one dtype")
-        return sum(int(g[0]) * int(g[1]) * int(g[2]) for g in grid_thw)
+        C = self.C
+        thw, grids, n, dt = [], [], 0, None
+        for f, g in zip(frames, grid_thw):
+            if len(g) != 3:
+                raise ValueError("every grid_thw entry must be (t, h, w)")
+            s = f.shape
+            if len(s) != 4 or s[1] != C:
+                raise ValueError(f"frames must be [T, {C}, H, W]; got {tuple(s)}")
+            if dt is None:
+                dt = f.dtype
+            elif f.dtype != dt:
+                raise TypeError("all items must share one dtype")
+            t, h, w = int(g[0]), int(g[1]), int(g[2])
+            grids += (t, h, w)
+            thw += (s[0], s[2], s[3])
+            n += t * h * w
+        return n, thw, grids, dt
 
     def forward_frames_grouped(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]],
                                merge: int = 2, out: Optional[torch.Tensor] = None,
@@ -188,18 +210,17 @@ class PatchEmbed:
                                pos: Optional[torch.Tensor] = None) -> torch.Tensor:
         """All items in one launch; `pos`, if given, is a [N, E] table in output row
         order added in the same epilogue."""
-        n = self._items(frames, grid_thw)
+        n, thw, grids, fdt = self._items(frames, grid_thw)
         out = self._out(n, out, out_dtype, frames[0].device)
         if pos is not None:
             _need(pos, (n, self.E), "pos")
         d = self.dev
         ptrs = [_dev(f, "frames", d) for f in frames]
-        thw = [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames]
         if pos is None:
-            B.pe_forward_frames_grouped(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
+            B.pe_forward_frames_grouped(self.h, ptrs, _dt(fdt), thw, grids, merge,
                                         _dev(out, "out", d), _dt(out.dtype), _stream(stream))
         else:
-            B.pe_forward_frames_grouped_pos(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
+            B.pe_forward_frames_grouped_pos(self.h, ptrs, _dt(fdt), thw, grids, merge,
                                             _dev(pos, "pos", d), _dt(pos.dtype), _dev(out, "out", d),
                                             _dt(out.dtype), _stream(stream))
         return out
@@ -213,12 +234,11 @@ class PatchEmbed:
         tensors (``pin_memory()``) overlap the copies; the default output is
         pinned.  With ``blocking=False`` the output is complete only once the
         stream has drained."""
-        n = self._items(frames, grid_thw)
+        n, thw, grids, fdt = self._items(frames, grid_thw)
         out = _host_out((n, self.E), out, out_dtype)
         ptrs = [_host(f, "frames") for f in frames]
-        thw = [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames]
         st = _stream(stream)
-        B.pe_forward_frames_grouped_host(self.h, ptrs, _dt(frames[0].dtype), thw, grid_thw, merge,
+        B.pe_forward_frames_grouped_host(self.h, ptrs, _dt(fdt), thw, grids, merge,
                                          _host(out, "out"), _dt(out.dtype), st)
         if blocking:
             _sync(stream)
@@ -241,10 +261,9 @@ class PatchEmbed:
 
     def patchify(self, frames: Sequence[torch.Tensor], grid_thw: Sequence[Sequence[int]], merge: int = 2,
                  rows_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
-        n = self._items(frames, grid_thw)
+        n, thw, grids, fdt = self._items(frames, grid_thw)
         rows = torch.empty((n, self.K), dtype=rows_dtype, device=frames[0].device)
-        B.pe_patchify(self.h, [_dev(f, "frames", self.dev) for f in frames], _dt(frames[0].dtype),
-                      [tuple(f.shape[i] for i in (0, 2, 3)) for f in frames], grid_thw, merge,
+        B.pe_patchify(self.h, [_dev(f, "frames", self.dev) for f in frames], _dt(fdt), thw, grids, merge,
                       _dev(rows, "rows"), _dt(rows.dtype), _stream(stream))
         return rows
 
