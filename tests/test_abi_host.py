@@ -102,3 +102,23 @@ def test_create_without_gpu_fails_cleanly(lib):
     h = ctypes.c_void_p()
     rc = lib.pe_create(1280, 3, 2, 14, 0, ctypes.byref(h))
     assert rc != 0 and h.value is None
+
+
+def test_marshalling_helpers():
+    """The binding's array builders: nested or flat grids, numpy and torch
+    integers, pointers as 64-bit values; out-of-range values are refused rather
+    than wrapped."""
+    import numpy as np
+    from vlm_vision_patch_b200 import _binding as B
+    nested = [(1, 16, 64), (2, 4, 6)]
+    flat = [1, 16, 64, 2, 4, 6]
+    assert list(B._i32rows(nested)) == flat
+    assert list(B._i32rows(flat)) == flat
+    assert list(B._i32rows(np.array(nested))) == flat
+    assert list(B._i32rows([torch.tensor(v) for v in flat])) == flat
+    assert list(B._i32rows([])) == []
+    big = 2**47 + 4096
+    p = B._ptrs([big, 0, 16])
+    assert [p[0], p[1], p[2]] == [big, None, 16]
+    with pytest.raises(OverflowError):
+        B._i32arr([2**31])

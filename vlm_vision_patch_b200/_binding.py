@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import array
 import ctypes
+import operator
 import os
 from typing import Optional, Sequence
 
@@ -123,8 +124,11 @@ def _i32arr(vals: Sequence[int]):
 
 def _i32rows(rows) -> "ctypes.Array":
     """int32 array of [n, 3] values given as n triples or already flat."""
-    if len(rows) and not hasattr(rows[0], "__index__"):
-        rows = [v for r in rows for v in r]
+    if len(rows):
+        try:
+            operator.index(rows[0])          # an integer: already flat
+        except TypeError:
+            rows = [v for r in rows for v in r]
     return _i32arr(rows)
 
 
