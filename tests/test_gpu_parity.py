@@ -712,7 +712,7 @@ def test_patch_merger_errors():
 # ------------------------------------------------------ more path/shape cases
 
 @pytest.mark.parametrize("case", ["staged_E200_bias_f32", "staged_merge1_odd_gw_p16", "fold_with_pos",
-                                  "tf32_with_pos"])
+                                  "fold_with_f32_pos_f32_out", "tf32_with_pos"])
 def test_more_path_combinations(case, monkeypatch):
     """Combinations of options and ragged shapes on the default paths, each
     against the oracle at the parity tolerance (the tf32 case against the
@@ -736,17 +736,19 @@ def test_more_path_combinations(case, monkeypatch):
         p, E, merge, grids, Ts, od = 14, 200, 2, [(2, 6, 8), (1, 4, 10)], [3, 1], torch.float32
     elif case == "staged_merge1_odd_gw_p16":
         p, E, merge, grids, Ts, od = 16, 384, 1, [(1, 5, 7), (2, 3, 9)], [1, 4], torch.bfloat16
-    else:
+    elif case == "fold_with_pos":
         p, E, merge, grids, Ts, od = 14, 512, 2, [(1, 8, 12), (1, 6, 6)], [1, 1], torch.bfloat16
+    else:   # an fp32 table and fp32 rows through the folded path's register stores
+        p, E, merge, grids, Ts, od = 14, 200, 2, [(1, 8, 12), (1, 6, 6)], [1, 1], torch.float32
     items = [(workloads.uniform01((T, C, g[1] * p, g[2] * p), 710 + i), g) for i, (T, g) in enumerate(zip(Ts, grids))]
     w = workloads.normal((E, C, tp, p, p), 720, std=0.02, dtype=torch.bfloat16)
     b = workloads.normal((E,), 721, std=0.02, dtype=torch.bfloat16)
     pe = _pe((E, C, tp, p), w, b, workloads.CLIP_MEAN, workloads.CLIP_STD)
     N = sum(g[0] * g[1] * g[2] for g in grids)
     pos = None
-    if case == "fold_with_pos":
+    if case.startswith("fold_with"):
         pe.set_temporal_fold(True)
-        pos = workloads.normal((N, E), 722, std=0.5, dtype=torch.bfloat16)
+        pos = workloads.normal((N, E), 722, std=0.5, dtype=torch.bfloat16 if case == "fold_with_pos" else torch.float32)
     out = pe.forward_frames_grouped([f.to(DEV) for f, _ in items], grids, merge, out_dtype=od,
                                     pos=None if pos is None else pos.to(DEV))
     torch.cuda.synchronize()
