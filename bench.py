@@ -632,6 +632,9 @@ def run_ours(args, rank, world, local):
             "patchify": patchify_line(wl, pre_times),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
+                         # context: the same against the sustained (power-capped) figure
+                         "frac_sustained": achieved / (float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+                                                       * (1.1 / 2.25 if tf32 else 1.0)),
                          "kernel": kernel + ", 2*N*K*E flop per launch over its own CUDA-event duration",
                          "peak_source": (f"{src} bf16 dense (burst), MEASURED_PEAKS.json" if src == "measured"
                                          else "fallback 1590 TFLOP/s bf16")
