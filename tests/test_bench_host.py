@@ -155,3 +155,22 @@ def test_eager_torch_rows_match_the_oracle_patchify(T, gh, gw, merge, tp, p):
     ref = oracle.patchify(frames, grid, merge, workloads.CLIP_MEAN, workloads.CLIP_STD, C, tp, p)
     assert got.dtype == torch.bfloat16
     assert np.array_equal(got.float().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def test_measured_traffic_belongs_to_one_kernel_form_and_source(monkeypatch):
+    """The per-launch DRAM figure is reported only for the kernel form it was
+    captured on (a folded, position-table or tf32 launch has its own key) and
+    only while the kernel sources still hash to the digest of the capture."""
+    key = ("grouped_16_images", "staged")
+    rec = bench.TRAFFIC[key]
+    sha = bench.kernel_sha()
+    if rec["kernel_sha"] == sha:
+        assert bench.measured_traffic(*key) == rec["bytes"]
+    assert bench.measured_traffic("grouped_16_images", "staged_pos") is None
+    assert bench.measured_traffic("grouped_16_images", "no_such_path") is None
+    monkeypatch.setattr(bench, "kernel_sha", lambda: "0" * 16)
+    assert bench.measured_traffic(*key) is None
+    # comments do not change the digest; code does
+    base = bench.code_digest(["int a; // x\n", "/* y */ int b;"])
+    assert bench.code_digest(["int a;  // other\n", "int b; /* z */"]) == base
+    assert bench.code_digest(["int a = 1;", "int b;"]) != base
